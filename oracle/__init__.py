@@ -1,0 +1,216 @@
+"""CPU oracle for the sparse MoE feed-forward layer.
+
+TEST INFRASTRUCTURE ONLY: the plain, slow, obviously correct CPU definition
+that the CUDA path is checked against. Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import it. It shares no code with the CUDA path (``mixture_experts_ffn_11_b200``)
+and does not import it; both take their inputs from the ``synth`` module.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, fp64 accumulation); this
+module builds it, marshals numpy arrays, and strings the steps together.
+Citations are to the blog post "Mixture of Experts (MoEs) in Transformers".
+
+Parity status per function (what pins it, see tests/test_oracle_pins.py):
+  router_logits  pinned: numpy fp64 matmul; closed-form golden cases
+  topk           pinned: brute-force full sort; golden ties; closed-form weights
+  permute        pinned: numpy stable argsort; invariants (bijection, scan)
+  moe_tokens     pinned: dense-masked brute force over all experts (numpy fp64);
+                 E=1,k=1 dense SwiGLU (torch fp64); identical experts; linearity
+                 in W_down; hand-derived golden values
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_SO = os.path.join(_HERE, "_moe_oracle.so")
+
+ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm": 2}
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _SO) -> str:
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-shared", "-fPIC", "-pthread", src, "-o", out, "-lm"])
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building if needed) the oracle library; ``path`` selects another build of it."""
+    lib = ctypes.CDLL(path or build())
+    vp, ci = ctypes.c_void_p, ctypes.c_int
+    lib.oracle_router_logits.argtypes = [vp, vp, vp, ci, ci, ci, vp]
+    lib.oracle_router_logits.restype = None
+    lib.oracle_topk.argtypes = [vp, ci, ci, ci, ci, vp, vp]
+    lib.oracle_topk.restype = ci
+    lib.oracle_topk_margin.argtypes = [vp, ci, ci, ci, vp]
+    lib.oracle_topk_margin.restype = ci
+    lib.oracle_permute.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp]
+    lib.oracle_permute.restype = ci
+    lib.oracle_moe_tokens.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, ci, vp, ci, vp, ci]
+    lib.oracle_moe_tokens.restype = ci
+    return lib
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        _lib = load()
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def router_logits(x_bits: np.ndarray, w_router: np.ndarray, bias: np.ndarray | None = None, lib=None) -> np.ndarray:
+    """fp64 logits x . W_r^T (+bias): the router scores every expert from the token's hidden state
+    (section "From Dense to Sparse"). x_bits: [T,d] bf16 bits; w_router: [E,d] fp32."""
+    lib = lib or _L()
+    x = _c(x_bits, np.uint16)
+    wr = _c(w_router, np.float32)
+    T, d = x.shape
+    E = wr.shape[0]
+    b = _c(bias, np.float32) if bias is not None else None
+    out = np.empty((T, E), dtype=np.float64)
+    lib.oracle_router_logits(x.ctypes.data, wr.ctypes.data, b.ctypes.data if b is not None else None, T, d, E,
+                             out.ctypes.data)
+    return out
+
+
+def topk(logits_f32: np.ndarray, k: int, mode: str, lib=None):
+    """Top-k experts per token on fp32 logits (descending, lower id first on ties) and their weights (fp64)."""
+    lib = lib or _L()
+    l = _c(logits_f32, np.float32)
+    T, E = l.shape
+    idx = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    rc = lib.oracle_topk(l.ctypes.data, T, E, k, ROUTE_MODES[mode], idx.ctypes.data, w.ctypes.data)
+    if rc:
+        raise ValueError("oracle_topk: bad arguments")
+    return idx, w
+
+
+def topk_margin(logits64: np.ndarray, k: int, lib=None) -> np.ndarray:
+    lib = lib or _L()
+    l = _c(logits64, np.float64)
+    T, E = l.shape
+    m = np.empty(T, dtype=np.float64)
+    if lib.oracle_topk_margin(l.ctypes.data, T, E, k, m.ctypes.data):
+        raise ValueError("oracle_topk_margin: bad arguments")
+    return m
+
+
+def permute(idx: np.ndarray, E: int, lib=None):
+    """Stable grouping of the T*k assignments by expert id ("sort tokens by expert ID, group them",
+    section "Expert Backend"). Returns counts[E], offsets[E+1], perm_src[R], inv_perm[R]."""
+    lib = lib or _L()
+    ix = _c(idx, np.int32)
+    T, k = ix.shape
+    counts = np.empty(E, dtype=np.int32)
+    offsets = np.empty(E + 1, dtype=np.int32)
+    perm_src = np.empty(T * k, dtype=np.int32)
+    inv_perm = np.empty(T * k, dtype=np.int32)
+    if lib.oracle_permute(ix.ctypes.data, T, E, k, counts.ctypes.data, offsets.ctypes.data, perm_src.ctypes.data,
+                          inv_perm.ctypes.data):
+        raise ValueError("oracle_permute: expert index out of range")
+    return counts, offsets, perm_src, inv_perm
+
+
+def moe_tokens(x_bits, expert_gateup, expert_down, idx, w, tokens, shared_gateup=None, shared_down=None,
+               nthreads: int | None = None, lib=None) -> np.ndarray:
+    """Per-token loop over the selected experts (the eager backend of section "Expert Backend"):
+    out[q] = sum_j w[t,j] * down_e(silu(gate_e x_t) * up_e x_t) (+ shared expert), fp64.
+
+    expert_gateup / expert_down: sequences of length E holding [2f,d] / [d,f] bf16-bit arrays, or None
+    for experts that no listed token selects.
+    """
+    lib = lib or _L()
+    x = _c(x_bits, np.uint16)
+    T, d = x.shape
+    E = len(expert_gateup)
+    ix = _c(idx, np.int32)
+    k = ix.shape[1]
+    ww = _c(w, np.float64)
+    toks = _c(tokens, np.int32)
+    f = None
+    keep = []
+    gu_ptrs = (ctypes.c_void_p * E)()
+    dn_ptrs = (ctypes.c_void_p * E)()
+    for e in range(E):
+        gu, dn = expert_gateup[e], expert_down[e]
+        if gu is None or dn is None:
+            continue
+        gu = _c(gu, np.uint16)
+        dn = _c(dn, np.uint16)
+        f = gu.shape[0] // 2
+        keep += [gu, dn]
+        gu_ptrs[e] = gu.ctypes.data
+        dn_ptrs[e] = dn.ctypes.data
+    if f is None:
+        raise ValueError("no expert weights given")
+    sgu = _c(shared_gateup, np.uint16) if shared_gateup is not None else None
+    sdn = _c(shared_down, np.uint16) if shared_down is not None else None
+    fs = sgu.shape[0] // 2 if sgu is not None else 0
+    out = np.empty((len(toks), d), dtype=np.float64)
+    n = nthreads or max(1, len(os.sched_getaffinity(0)))
+    rc = lib.oracle_moe_tokens(x.ctypes.data, T, d, f, E, k, gu_ptrs, dn_ptrs, ix.ctypes.data, ww.ctypes.data,
+                               sgu.ctypes.data if sgu is not None else None,
+                               sdn.ctypes.data if sdn is not None else None, fs, toks.ctypes.data, len(toks),
+                               out.ctypes.data, n)
+    if rc:
+        raise ValueError(f"oracle_moe_tokens failed ({rc})")
+    return out
+
+
+class LayerReference:
+    """The whole layer for one synthetic workload, computed by the oracle.
+
+    Routing and grouping are computed for all tokens; expert outputs only for the tokens asked for,
+    generating only the experts those tokens select (so multi-gigabyte layers stay cheap on the host).
+    """
+
+    def __init__(self, wl, lib=None):
+        import synth
+
+        self.wl = wl
+        self.lib = lib or _L()
+        self.x = synth.x_host(wl)
+        self.w_router = synth.w_router_host(wl)
+        self.bias = synth.zipf_bias(wl)
+        self.logits64 = router_logits(self.x, self.w_router, self.bias, lib=self.lib)
+        self.logits32 = self.logits64.astype(np.float32)
+        self.idx, self.w = topk(self.logits32, wl.k, wl.route, lib=self.lib)
+        self.margin = topk_margin(self.logits64, wl.k, lib=self.lib)
+        self.counts, self.offsets, self.perm_src, self.inv_perm = permute(self.idx, wl.E, lib=self.lib)
+        self._gu = [None] * wl.E
+        self._dn = [None] * wl.E
+        self._shared = None
+
+    def near_ties(self, eps: float = 1e-5) -> np.ndarray:
+        return np.nonzero(self.margin < eps)[0]
+
+    def outputs(self, tokens, nthreads: int | None = None) -> np.ndarray:
+        import synth
+
+        wl = self.wl
+        tokens = np.asarray(tokens, dtype=np.int32)
+        need = np.unique(self.idx[tokens].ravel()) if len(tokens) else np.zeros(0, np.int32)
+        for e in need:
+            if self._gu[e] is None:
+                self._gu[e] = synth.w_gateup_expert_host(wl, int(e))
+                self._dn[e] = synth.w_down_expert_host(wl, int(e))
+        if wl.shared_f and self._shared is None:
+            self._shared = synth.shared_host(wl)
+        sgu, sdn = self._shared if self._shared else (None, None)
+        if len(tokens) == 0:
+            return np.zeros((0, wl.d))
+        return moe_tokens(self.x, self._gu, self._dn, self.idx, self.w, tokens, sgu, sdn, nthreads=nthreads,
+                          lib=self.lib)

@@ -1,0 +1,272 @@
+/*
+ * CPU oracle for the sparse MoE feed-forward layer.
+ *
+ * TEST INFRASTRUCTURE ONLY. This code proves the CUDA path correct; it is not
+ * part of the product. Only the tests, the smoke check and the benchmark's CPU
+ * baseline leg may load it. It shares no code, header, table or helper with
+ * the CUDA path.
+ *
+ * What it computes follows the blog post "Mixture of Experts (MoEs) in
+ * Transformers":
+ *   - section "From Dense to Sparse": a router picks a small subset of experts
+ *     per token; each expert is a learnable sub-network that replaces the
+ *     dense feed-forward block;
+ *   - section "Expert Backend": the runtime dispatches tokens to their
+ *     selected experts, runs the projections, applies the routing weights and
+ *     collects the results back in token order; the "eager" backend, a plain
+ *     loop over the selected experts, is the correctness reference. This file
+ *     is that loop, written per token;
+ *   - section "Dynamic Weight Loading with WeightConverter": the packed
+ *     gate_up_proj tensor stacks experts on dim 0 and concatenates w1 (gate)
+ *     then w3 (up) on dim 1, so expert e's rows [0,f) are gate and [f,2f) are
+ *     up, each row of length d; down_proj stacks the experts' w2 on dim 0,
+ *     each [d, f] (output row c, input column n).
+ *   - "sort tokens by expert ID, group them" (grouped_mm, section "Expert
+ *     Backend"): the grouping is a stable counting sort by expert id.
+ * The pages do not state the router formula or the expert activation; the
+ * layer descriptions this library serves fix them: fp32 logits x.W_r^T (+bias),
+ * top-k on the logits (descending, lower expert id first on ties), weights by
+ * one of three modes, and a SwiGLU expert silu(gate)*up followed by down.
+ *
+ * Precision: every sum is accumulated in fp64 from the bf16/fp32 inputs, and
+ * the SwiGLU intermediate is kept in fp64. The only rounding to fp32 is of
+ * the router logits, because top-k selection (an integer decision) is taken
+ * in fp32 on both sides.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORACLE_TOPK_SOFTMAX = 0, ORACLE_SOFTMAX_TOPK_RENORM = 1, ORACLE_SIGMOID_TOPK_NORM = 2 };
+
+static double bf16_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float v;
+    memcpy(&v, &u, 4);
+    return (double)v;
+}
+
+/* Router logits: l[t][e] = sum_i x[t][i] * W_r[e][i] (+ bias[e]), in fp64. */
+void oracle_router_logits(const uint16_t* x, const float* w_router, const float* bias, int T, int d, int E,
+                          double* logits) {
+    for (int t = 0; t < T; ++t) {
+        for (int e = 0; e < E; ++e) {
+            double s = 0.0;
+            for (int i = 0; i < d; ++i) s += bf16_to_double(x[(size_t)t * d + i]) * (double)w_router[(size_t)e * d + i];
+            if (bias) s += (double)bias[e];
+            logits[(size_t)t * E + e] = s;
+        }
+    }
+}
+
+/* Top-k selection and routing weights from fp32 logits [T][E].
+ * idx[t][j]: the j-th largest logit's expert (ties: lower expert id first).
+ * w[t][j]:   routing weight of that expert, by mode, in fp64.
+ * Returns 0, or -1 on bad arguments. */
+int oracle_topk(const float* logits, int T, int E, int k, int mode, int32_t* idx, double* w) {
+    if (T < 0 || E <= 0 || k <= 0 || k > E) return -1;
+    if (mode < 0 || mode > 2) return -1;
+    char* taken = (char*)malloc((size_t)E);
+    if (!taken) return -1;
+    for (int t = 0; t < T; ++t) {
+        const float* l = logits + (size_t)t * E;
+        memset(taken, 0, (size_t)E);
+        /* k passes of "largest not yet taken"; strict '>' keeps the lower id on ties. */
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e;
+            }
+            taken[best] = 1;
+            idx[(size_t)t * k + j] = best;
+        }
+        double* wt = w + (size_t)t * k;
+        const int32_t* it = idx + (size_t)t * k;
+        if (mode == ORACLE_TOPK_SOFTMAX) {
+            /* softmax over the k selected logits (max-subtracted) */
+            double m = (double)l[it[0]];
+            double z = 0.0;
+            for (int j = 0; j < k; ++j) { wt[j] = exp((double)l[it[j]] - m); z += wt[j]; }
+            for (int j = 0; j < k; ++j) wt[j] /= z;
+        } else if (mode == ORACLE_SOFTMAX_TOPK_RENORM) {
+            /* softmax over all E logits, keep the selected probabilities, divide by their sum */
+            double m = (double)l[it[0]];
+            double zall = 0.0;
+            for (int e = 0; e < E; ++e) zall += exp((double)l[e] - m);
+            double zsel = 0.0;
+            for (int j = 0; j < k; ++j) { wt[j] = exp((double)l[it[j]] - m) / zall; zsel += wt[j]; }
+            for (int j = 0; j < k; ++j) wt[j] /= zsel;
+        } else {
+            /* sigmoid scores of the selected experts, divided by their sum */
+            double z = 0.0;
+            for (int j = 0; j < k; ++j) { wt[j] = 1.0 / (1.0 + exp(-(double)l[it[j]])); z += wt[j]; }
+            for (int j = 0; j < k; ++j) wt[j] /= z;
+        }
+    }
+    free(taken);
+    return 0;
+}
+
+/* Margin between the k-th and (k+1)-th largest fp64 logits of each token
+ * (INFINITY when k == E). Tokens with a tiny margin are near-ties whose
+ * selection depends on summation order. */
+int oracle_topk_margin(const double* logits, int T, int E, int k, double* margin) {
+    if (k <= 0 || k > E) return -1;
+    double* v = (double*)malloc(sizeof(double) * (size_t)(k + 1));
+    if (!v) return -1;
+    for (int t = 0; t < T; ++t) {
+        if (k == E) { margin[t] = INFINITY; continue; }
+        const double* l = logits + (size_t)t * E;
+        /* keep the k+1 largest values in descending order (insertion) */
+        int n = 0;
+        for (int e = 0; e < E; ++e) {
+            double x = l[e];
+            if (n == k + 1 && x <= v[k]) continue;
+            int p = n < k + 1 ? n++ : k;
+            while (p > 0 && v[p - 1] < x) { v[p] = v[p - 1]; --p; }
+            v[p] = x;
+        }
+        margin[t] = v[k - 1] - v[k];
+    }
+    free(v);
+    return 0;
+}
+
+/* Grouping by expert id: a stable counting sort of the T*k assignments.
+ * Assignment a = t*k + j goes to expert idx[a].
+ * counts[e]    number of assignments to expert e
+ * offsets[e]   exclusive prefix sum of counts; offsets[E] = T*k
+ * perm_src[r]  token of the assignment placed at row r (rows sorted by expert,
+ *              then by a)
+ * inv_perm[a]  row at which assignment a is placed
+ * Returns 0, or -1 if an index is out of range. */
+int oracle_permute(const int32_t* idx, int T, int E, int k, int32_t* counts, int32_t* offsets, int32_t* perm_src,
+                   int32_t* inv_perm) {
+    long R = (long)T * k;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (long a = 0; a < R; ++a) {
+        if (idx[a] < 0 || idx[a] >= E) return -1;
+        counts[idx[a]]++;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+    if (!cursor) return -1;
+    for (int e = 0; e < E; ++e) cursor[e] = offsets[e];
+    for (long a = 0; a < R; ++a) {
+        int32_t r = cursor[idx[a]]++;
+        perm_src[r] = (int32_t)(a / k);
+        inv_perm[a] = r;
+    }
+    free(cursor);
+    return 0;
+}
+
+/* ---- expert MLP + weighted combine, per token -------------------------------------------------- */
+
+typedef struct {
+    const uint16_t* x;
+    int T, d, f, E, k, fs;
+    const uint16_t* const* wgu; /* E pointers to [2f][d] (NULL where not needed) */
+    const uint16_t* const* wd;  /* E pointers to [d][f] */
+    const int32_t* idx;
+    const double* w;
+    const uint16_t* wgu_s; /* shared expert [2fs][d] or NULL */
+    const uint16_t* wd_s;  /* shared expert [d][fs] or NULL */
+    const int32_t* tokens;
+    int n_tokens;
+    double* out;
+    int first, last;
+    int status;
+} tok_job_t;
+
+/* acc[c] += scale * sum_n h[n] * Wd[c][n], h[n] = silu(g[n]) * u[n],
+ * g[n] = sum_i x[i] Wgu[n][i], u[n] = sum_i x[i] Wgu[f+n][i]. */
+static void swiglu_expert(const uint16_t* xt, int d, int f, const uint16_t* wgu, const uint16_t* wd, double scale,
+                          double* h, double* acc) {
+    for (int n = 0; n < f; ++n) {
+        const uint16_t* gr = wgu + (size_t)n * d;
+        const uint16_t* ur = wgu + (size_t)(f + n) * d;
+        double g = 0.0, u = 0.0;
+        for (int i = 0; i < d; ++i) {
+            double xi = bf16_to_double(xt[i]);
+            g += xi * bf16_to_double(gr[i]);
+            u += xi * bf16_to_double(ur[i]);
+        }
+        h[n] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int c = 0; c < d; ++c) {
+        const uint16_t* dr = wd + (size_t)c * f;
+        double s = 0.0;
+        for (int n = 0; n < f; ++n) s += h[n] * bf16_to_double(dr[n]);
+        acc[c] += scale * s;
+    }
+}
+
+static void* tok_worker(void* p) {
+    tok_job_t* J = (tok_job_t*)p;
+    int hf = J->f > J->fs ? J->f : J->fs;
+    double* h = (double*)malloc(sizeof(double) * (size_t)(hf > 0 ? hf : 1));
+    if (!h) { J->status = -1; return NULL; }
+    for (int q = J->first; q < J->last; ++q) {
+        int t = J->tokens[q];
+        const uint16_t* xt = J->x + (size_t)t * J->d;
+        double* acc = J->out + (size_t)q * J->d;
+        for (int c = 0; c < J->d; ++c) acc[c] = 0.0;
+        for (int j = 0; j < J->k; ++j) {
+            int e = J->idx[(size_t)t * J->k + j];
+            if (e < 0 || e >= J->E || !J->wgu[e] || !J->wd[e]) { J->status = -2; free(h); return NULL; }
+            swiglu_expert(xt, J->d, J->f, J->wgu[e], J->wd[e], J->w[(size_t)t * J->k + j], h, acc);
+        }
+        if (J->wgu_s && J->wd_s) swiglu_expert(xt, J->d, J->fs, J->wgu_s, J->wd_s, 1.0, h, acc);
+    }
+    free(h);
+    return NULL;
+}
+
+/* out[q][c] for the listed tokens q: sum over the token's selected experts of
+ * w * down(silu(gate) * up), plus the shared expert (weight 1) when given.
+ * wgu/wd are arrays of E per-expert pointers; only the experts the listed
+ * tokens select must be non-NULL. Runs on nthreads threads (tokens split into
+ * contiguous chunks). Returns 0, -1 on allocation failure, -2 on a missing
+ * expert or bad index. */
+int oracle_moe_tokens(const uint16_t* x, int T, int d, int f, int E, int k, const uint16_t* const* wgu,
+                      const uint16_t* const* wd, const int32_t* idx, const double* w, const uint16_t* wgu_shared,
+                      const uint16_t* wd_shared, int f_shared, const int32_t* tokens, int n_tokens, double* out,
+                      int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > n_tokens) nthreads = n_tokens > 0 ? n_tokens : 1;
+    if (nthreads > 512) nthreads = 512;
+    for (int q = 0; q < n_tokens; ++q)
+        if (tokens[q] < 0 || tokens[q] >= T) return -2;
+    tok_job_t* jobs = (tok_job_t*)calloc((size_t)nthreads, sizeof(tok_job_t));
+    pthread_t* th = (pthread_t*)calloc((size_t)nthreads, sizeof(pthread_t));
+    char* started = (char*)calloc((size_t)nthreads, 1);
+    if (!jobs || !th || !started) { free(jobs); free(th); free(started); return -1; }
+    int per = (n_tokens + nthreads - 1) / nthreads;
+    for (int i = 0; i < nthreads; ++i) {
+        tok_job_t* J = &jobs[i];
+        J->x = x; J->T = T; J->d = d; J->f = f; J->E = E; J->k = k;
+        J->fs = (wgu_shared && wd_shared) ? f_shared : 0;
+        J->wgu = wgu; J->wd = wd; J->idx = idx; J->w = w;
+        J->wgu_s = wgu_shared; J->wd_s = wd_shared;
+        J->tokens = tokens; J->n_tokens = n_tokens; J->out = out;
+        J->first = i * per;
+        J->last = (i + 1) * per < n_tokens ? (i + 1) * per : n_tokens;
+        if (J->first >= J->last) continue;
+        if (nthreads == 1 || pthread_create(&th[i], NULL, tok_worker, J) != 0)
+            tok_worker(J);
+        else
+            started[i] = 1;
+    }
+    int status = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        if (started[i]) pthread_join(th[i], NULL);
+        if (jobs[i].status) status = jobs[i].status;
+    }
+    free(jobs); free(th); free(started);
+    return status;
+}
