@@ -1,0 +1,177 @@
+/*
+ * moe.h — C-ABI of the B200 (sm_100a) sparse mixture-of-experts feed-forward layer.
+ *
+ * The layer replaces a dense feed-forward block by E expert networks and a
+ * router that sends each token to a small subset of them (blog post "Mixture
+ * of Experts (MoEs) in Transformers", section "From Dense to Sparse"). At run
+ * time it must dispatch tokens to their selected experts, run the expert
+ * projections, apply the routing weights and collect the results back in
+ * token order (same post, section "Expert Backend"). This library does it the
+ * grouped_mm way described there: sort tokens by expert id, group them, and
+ * run one grouped GEMM over all experts. One layer call is:
+ *
+ *   moe_route_topk          logits, top-k expert ids and routing weights
+ *   moe_permute             expert histogram, exclusive scan, stable scatter,
+ *                           gather of x rows into expert-contiguous order
+ *   moe_grouped_gemm_gateup h = silu(x_perm Wg^T) * (x_perm Wu^T), per expert
+ *   moe_grouped_gemm_down   y_perm = h Wd^T, per expert
+ *   moe_unpermute_combine   y[t] = sum_j w[t,j] * y_perm[row of (t,j)] (+ shared[t])
+ *
+ * Conventions (all entry points):
+ *  - Every pointer argument is a DEVICE pointer to memory the caller allocated
+ *    and owns, unless stated otherwise. The library allocates no device memory
+ *    and frees nothing; it holds no state besides per-device attributes it
+ *    caches (SM count, kernel attributes) and a device-side error word.
+ *  - bf16 tensors are passed as moe_bf16_t (the raw 16-bit pattern of a
+ *    bfloat16). All tensors are dense and row-major (last index fastest).
+ *  - Pointers must be 16-byte aligned. d and f must be multiples of 8 (rows of
+ *    bf16 then start on 16-byte boundaries, as the TMA engine requires).
+ *  - Calls are asynchronous on `stream`. They never synchronise and never
+ *    read device memory from the host, except moe_get_device_error().
+ *  - Argument errors are reported before anything is launched (outputs are
+ *    left untouched): MOE_ERR_INVALID_ARG. A launch failure returns
+ *    MOE_ERR_CUDA; moe_last_error_string() describes it.
+ *  - Anomalies found on the device (an expert id or a group offset out of
+ *    range, a pipeline wait that timed out) never fault: the kernel skips the
+ *    offending access, sets a bit in a device error word and returns. Read and
+ *    clear it with moe_get_device_error().
+ *  - Integer sizes are int; T*k, T*d and T*E must fit in int32, group row
+ *    counts M in int32.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, k > E, unsupported mode */
+    MOE_ERR_UNSUPPORTED = 2, /* current device is not sm_100 */
+    MOE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_workspace_size() figure */
+    MOE_ERR_CUDA = 4,        /* a CUDA call or launch failed; see moe_last_error_string() */
+    MOE_ERR_DEVICE = 5       /* returned by moe_get_device_error() when the error word was set */
+} moe_status_t;
+
+/* Bits of the device error word. */
+#define MOE_DEVERR_WAIT_TIMEOUT 0x1u  /* a pipeline wait in a GEMM gave up after its time limit */
+#define MOE_DEVERR_EXPERT_RANGE 0x2u  /* an expert id outside [0, E) reached moe_permute */
+#define MOE_DEVERR_GROUP_RANGE 0x4u   /* group offsets not non-decreasing within [0, M] */
+#define MOE_DEVERR_ROW_RANGE 0x8u     /* a permutation entry outside its range */
+
+/* Routing weight modes. Selection is always the k largest logits in
+ * descending order, the lower expert id first on ties. Weights of the k
+ * selected experts of a token:
+ *   MOE_ROUTE_TOPK_SOFTMAX         softmax over the k selected logits
+ *   MOE_ROUTE_SOFTMAX_TOPK_RENORM  softmax over all E logits, keep the k
+ *                                  selected probabilities, divide by their sum
+ *   MOE_ROUTE_SIGMOID_TOPK_NORM    sigmoid of each selected logit, divided by
+ *                                  the sum of the k sigmoids
+ * The blog post names the router but not its formula ("From Dense to Sparse");
+ * these are the three variants used by the model families it lists. */
+typedef enum {
+    MOE_ROUTE_TOPK_SOFTMAX = 0,
+    MOE_ROUTE_SOFTMAX_TOPK_RENORM = 1,
+    MOE_ROUTE_SIGMOID_TOPK_NORM = 2
+} moe_route_mode_t;
+
+/* Router: logits[t][e] = sum_i x[t][i] * w_router[e][i] + bias[e] in fp32,
+ * then top-k selection and routing weights (section "From Dense to Sparse":
+ * "a router selects a small subset of experts" per token).
+ *   x          [T][d] bf16
+ *   w_router   [E][d] fp32
+ *   bias       [E] fp32, or NULL for none (added before selection and weights)
+ *   logits_out [T][E] fp32, written (required: the selection reads it back)
+ *   topk_idx   [T][k] int32, expert ids, descending logit order
+ *   topk_w     [T][k] fp32, routing weights per `mode`
+ * Limits: 1 <= k <= E <= 1024, T >= 0 (T == 0 launches nothing). */
+moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const float* bias, int T, int d, int E,
+                            int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx, float* topk_w,
+                            cudaStream_t stream);
+
+/* Top-k selection and routing weights from given fp32 logits [T][E] (bias, if
+ * any, already included). Same outputs and limits as moe_route_topk. */
+moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_route_mode_t mode,
+                                  int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
+/* Bytes of device workspace moe_permute needs for these sizes (a multiple of
+ * 256; 0 when T*k == 0). */
+size_t moe_permute_workspace_size(int T, int E, int k);
+
+/* Group the T*k (token, slot) assignments by expert: "sort tokens by expert
+ * ID, group them" (section "Expert Backend", grouped_mm). Assignment a = t*k+j
+ * goes to expert topk_idx[a]. The sort is stable: rows of one expert keep
+ * increasing a, so the result is unique and deterministic.
+ *   expert_counts  [E]   assignments per expert
+ *   expert_offsets [E+1] exclusive prefix sum of counts; [E] = T*k
+ *   perm_src       [T*k] token whose row sits at each grouped row
+ *   inv_perm       [T*k] grouped row of assignment a
+ *   x, x_perm      [T][d] and [T*k][d] bf16: x_perm[r] = x[perm_src[r]];
+ *                  pass both NULL to skip the gather (then d is ignored)
+ *   ws, ws_bytes   workspace of at least moe_permute_workspace_size(T,E,k)
+ *                  bytes, 256-byte aligned; its contents need not be
+ *                  initialised and are scratch after the call.
+ * Expert ids outside [0,E) are skipped and flagged (MOE_DEVERR_EXPERT_RANGE);
+ * the outputs are then incomplete. Limits: 1 <= k <= E <= 1024. */
+moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                         moe_bf16_t* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Grouped gate|up projection with fused SwiGLU, one expert per group:
+ * for every group g and row r in [group_offsets[g], group_offsets[g+1]):
+ *   h[r][n] = silu(sum_i a[r][i] * w[g][n][i]) * (sum_i a[r][i] * w[g][f+n][i]),  n < f,
+ * with silu(v) = v / (1 + exp(-v)), fp32 accumulation, h rounded to bf16.
+ * w is the packed gate_up_proj tensor [G][2f][d]: per expert, the gate rows
+ * (w1) then the up rows (w3), concatenated on dim 1 (section "Dynamic Weight
+ * Loading with WeightConverter").
+ *   a              [M][d] bf16 (rows grouped by expert, e.g. x_perm)
+ *   group_offsets  [G+1] int32, DEVICE memory, non-decreasing, [G] <= M;
+ *                  rows at or past group_offsets[G] are not written
+ *   h              [M][f] bf16
+ * M is the number of rows the caller allocated (T*k after moe_permute, T for
+ * a shared expert with G = 1 and offsets {0, T}). Limits: G >= 1, d, f >= 8,
+ * multiples of 8. */
+moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_gateup, const int32_t* group_offsets,
+                                     int G, int M, int d, int f, moe_bf16_t* h, cudaStream_t stream);
+
+/* Grouped down projection: y[r][c] = sum_n h[r][n] * w[g][c][n] (fp32
+ * accumulation, rounded to bf16) for r in group g. w is the packed down_proj
+ * tensor [G][d][f] (experts' w2 stacked on dim 0, same section).
+ *   h [M][f] bf16, y [M][d] bf16, group_offsets as above. */
+moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down, const int32_t* group_offsets,
+                                   int G, int M, int d, int f, moe_bf16_t* y, cudaStream_t stream);
+
+/* Apply the routing weights and return to token order ("apply the routing
+ * weights and then collect and reorder the results", section "Expert
+ * Backend"): y[t][c] = sum_{j<k} topk_w[t][j] * y_perm[inv_perm[t*k+j]][c]
+ * (+ shared[t][c]), summed in fp32 in slot order j, rounded to bf16. No
+ * atomics: the result is deterministic.
+ *   y_perm [T*k][d] bf16, inv_perm [T*k] int32, topk_w [T][k] fp32,
+ *   shared [T][d] bf16 or NULL (an always-on expert added with weight 1),
+ *   y [T][d] bf16 (must not alias the inputs). */
+moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w,
+                                   const moe_bf16_t* shared, int T, int d, int k, moe_bf16_t* y,
+                                   cudaStream_t stream);
+
+/* Synchronise `stream`, copy the device error word of the current device to
+ * *out (0 = no anomaly) and clear it. Returns MOE_OK when the word was 0,
+ * MOE_ERR_DEVICE when a bit was set, MOE_ERR_CUDA when the copy failed. */
+moe_status_t moe_get_device_error(unsigned int* out, cudaStream_t stream);
+
+/* Text of the last MOE_ERR_CUDA / MOE_ERR_INVALID_ARG on the calling thread
+ * ("" if none). The string is owned by the library, valid until the next call
+ * on that thread. */
+const char* moe_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

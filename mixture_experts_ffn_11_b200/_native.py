@@ -1,0 +1,179 @@
+"""ctypes binding of libmoe.so, the C-ABI declared in include/moe.h.
+
+Argument marshalling only: every function here checks dtypes/devices/shapes of torch tensors, passes
+their device pointers and the current CUDA stream to the library, and turns a non-zero status into an
+exception. All computation happens in the library's CUDA kernels. There is no fallback: if the library
+is missing or fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_WORKSPACE",
+          4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE"}
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
+DEVERR = {0x1: "wait timeout", 0x2: "expert id out of range", 0x4: "group offsets out of range",
+          0x8: "permutation entry out of range"}
+ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm": 2}
+
+# every entry point of include/moe.h
+EXPORTS = ("moe_route_topk", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
+           "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_unpermute_combine", "moe_get_device_error",
+           "moe_last_error_string")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m mixture_experts_ffn_11_b200.build` "
+                          "(there is no non-CUDA fallback)")
+    lib = ctypes.CDLL(path)
+    vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "moe_route_topk": [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp],
+        "moe_topk_from_logits": [vp, ci, ci, ci, ci, vp, vp, vp],
+        "moe_permute_workspace_size": [ci, ci, ci],
+        "moe_permute": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, sz, vp],
+        "moe_grouped_gemm_gateup": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_grouped_gemm_down": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_unpermute_combine": [vp, vp, vp, vp, ci, ci, ci, vp, vp],
+        "moe_get_device_error": [ctypes.POINTER(ctypes.c_uint), vp],
+        "moe_last_error_string": [],
+    }
+    for name, args in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ci
+    lib.moe_permute_workspace_size.restype = sz
+    lib.moe_last_error_string.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = load_library()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoEError(status, what, (_lib.moe_last_error_string() or b"").decode())
+
+
+def _stream(stream):
+    return (stream if stream is not None else torch.cuda.current_stream()).cuda_stream
+
+
+def _p(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t, dtype, shape=None, name="tensor"):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name}: want a contiguous CUDA {dtype} tensor, got {t.dtype} on {t.device}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: want shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def route_topk(x, w_router, bias, k, mode, logits, topk_idx, topk_w, stream=None):
+    T, d = x.shape
+    E = w_router.shape[0]
+    _need(x, torch.bfloat16, (T, d), "x")
+    _need(w_router, torch.float32, (E, d), "w_router")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    _need(logits, torch.float32, (T, E), "logits")
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    _check(_lib.moe_route_topk(_p(x), _p(w_router), _p(bias), T, d, E, k, ROUTE_MODES[mode], _p(logits),
+                               _p(topk_idx), _p(topk_w), _stream(stream)), "moe_route_topk")
+
+
+def topk_from_logits(logits, k, mode, topk_idx, topk_w, stream=None):
+    T, E = logits.shape
+    _need(logits, torch.float32, (T, E), "logits")
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    _check(_lib.moe_topk_from_logits(_p(logits), T, E, k, ROUTE_MODES[mode], _p(topk_idx), _p(topk_w),
+                                     _stream(stream)), "moe_topk_from_logits")
+
+
+def permute_workspace_size(T: int, E: int, k: int) -> int:
+    return int(_lib.moe_permute_workspace_size(T, E, k))
+
+
+def permute(x, topk_idx, E, counts, offsets, perm_src, inv_perm, x_perm, ws, stream=None):
+    T, k = topk_idx.shape
+    R = T * k
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(counts, torch.int32, (E,), "counts")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(perm_src, torch.int32, (R,), "perm_src")
+    _need(inv_perm, torch.int32, (R,), "inv_perm")
+    d = 0
+    if x is not None:
+        d = x.shape[1]
+        _need(x, torch.bfloat16, (T, d), "x")
+        _need(x_perm, torch.bfloat16, (R, d), "x_perm")
+    ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.moe_permute(_p(x), _p(topk_idx), T, d, E, k, _p(counts), _p(offsets), _p(perm_src),
+                            _p(inv_perm), _p(x_perm), _p(ws), ws_bytes, _stream(stream)), "moe_permute")
+
+
+def grouped_gemm_gateup(a, w_gateup, group_offsets, h, stream=None):
+    M, d = a.shape
+    G, two_f, d2 = w_gateup.shape
+    f = two_f // 2
+    _need(a, torch.bfloat16, (M, d), "a")
+    _need(w_gateup, torch.bfloat16, (G, 2 * f, d), "w_gateup")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(h, torch.bfloat16, (M, f), "h")
+    _check(_lib.moe_grouped_gemm_gateup(_p(a), _p(w_gateup), _p(group_offsets), G, M, d, f, _p(h),
+                                        _stream(stream)), "moe_grouped_gemm_gateup")
+
+
+def grouped_gemm_down(h, w_down, group_offsets, y, stream=None):
+    M, f = h.shape
+    G, d, f2 = w_down.shape
+    _need(h, torch.bfloat16, (M, f), "h")
+    _need(w_down, torch.bfloat16, (G, d, f), "w_down")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(y, torch.bfloat16, (M, d), "y")
+    _check(_lib.moe_grouped_gemm_down(_p(h), _p(w_down), _p(group_offsets), G, M, d, f, _p(y), _stream(stream)),
+           "moe_grouped_gemm_down")
+
+
+def unpermute_combine(y_perm, inv_perm, topk_w, shared, y, stream=None):
+    T, k = topk_w.shape
+    d = y.shape[1]
+    _need(y_perm, torch.bfloat16, (T * k, d), "y_perm")
+    _need(inv_perm, torch.int32, (T * k,), "inv_perm")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    if shared is not None:
+        _need(shared, torch.bfloat16, (T, d), "shared")
+    _need(y, torch.bfloat16, (T, d), "y")
+    _check(_lib.moe_unpermute_combine(_p(y_perm), _p(inv_perm), _p(topk_w), _p(shared), T, d, k, _p(y),
+                                      _stream(stream)), "moe_unpermute_combine")
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronise the stream and read-and-clear the device error word (0 = no anomaly)."""
+    v = ctypes.c_uint(0)
+    st = _lib.moe_get_device_error(ctypes.byref(v), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        _check(st, "moe_get_device_error")
+    return int(v.value)

@@ -1,0 +1,69 @@
+// Shared definitions of the CUDA path: the device error word, bf16 packing, warp helpers.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "moe.h"
+#include "sm100.cuh"
+
+namespace moe {
+
+// Device error word: kernels set MOE_DEVERR_* bits here instead of faulting. One per device (this
+// translation unit holds every kernel of the library, so there is exactly one definition).
+__device__ unsigned int g_device_error = 0;
+
+__device__ __forceinline__ void flag_error(unsigned int bit) { atomicOr(&g_device_error, bit); }
+
+// A pipeline wait gives up after this long and reports MOE_DEVERR_WAIT_TIMEOUT. No legitimate wait in
+// these kernels lasts more than a few hundred microseconds.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Bounded wait on an mbarrier phase. Returns false if `abort_flag` was raised by another role, or if
+// the time limit passed (then it raises the flag and the error bit itself).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    const uint32_t addr = smem_u32(bar);
+    if (mbar_try_wait(addr, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(addr, parity)) return true;
+        if ((spin & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                flag_error(MOE_DEVERR_WAIT_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait without an abort flag (used while draining on the way out).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+    const uint32_t addr = smem_u32(bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(addr, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            flag_error(MOE_DEVERR_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+    __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162*>(&u);
+    return __bfloat1622float2(v);
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+}  // namespace moe

@@ -1,0 +1,325 @@
+// C-ABI entry points of the MoE feed-forward layer library (declared in include/moe.h).
+// Every kernel of the library is in this one translation unit (the headers below), so the device
+// error word has a single definition.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "moe.h"
+#include "common.cuh"
+#include "route.cuh"
+#include "permute.cuh"
+#include "gemm.cuh"
+#include "combine.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+moe_status_t fail(moe_status_t st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return st;
+}
+
+moe_status_t check_launch(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Grouped-GEMM configurations compiled into the library.
+constexpr int kStages = 4;
+constexpr int kBN = 256;
+using GateUpShape = GemmShape<kBN, kStages, true>;
+using DownShape = GemmShape<kBN, kStages, false>;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool sm100 = false;
+    int sms = 0;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+
+moe_status_t device_info(DeviceInfo& out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& di = g_dev[dev];
+    if (!di.ready) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return fail(MOE_ERR_CUDA, "cudaDeviceGetAttribute failed on device %d", dev);
+        di.sm100 = (major == 10 && minor == 0);
+        di.sms = sms;
+        if (di.sm100) {
+            e = cudaFuncSetAttribute(grouped_gemm_kernel<kBN, kStages, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, GateUpShape::SMEM_BYTES);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(grouped_gemm_kernel<kBN, kStages, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, DownShape::SMEM_BYTES);
+            if (e != cudaSuccess)
+                return fail(MOE_ERR_CUDA, "cudaFuncSetAttribute(grouped GEMM): %s", cudaGetErrorString(e));
+        }
+        di.ready = true;
+    }
+    out = di;
+    if (!di.sm100) return fail(MOE_ERR_UNSUPPORTED, "device %d is not sm_100 (this library is built for sm_100a)", dev);
+    return MOE_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes for dims >= 1.
+moe_status_t make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint32_t elem_strides[3] = {1, 1, 1};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
+                           strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return MOE_OK;
+}
+
+template <int BN, int STAGES, bool GATEUP>
+moe_status_t launch_grouped_gemm(const void* a, const void* w, const int32_t* offsets, int G, int M, int K,
+                                 int n_out, int f, void* out, int sms, cudaStream_t stream) {
+    using S = GemmShape<BN, STAGES, GATEUP>;
+    CUtensorMap ta, tb;
+    const cuuint64_t adims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t astr[1] = {(cuuint64_t)K * 2};
+    const cuuint32_t abox[2] = {GG_BK, GG_BM};
+    moe_status_t st = make_tmap(&ta, a, 2, adims, astr, abox);
+    if (st != MOE_OK) return st;
+    // B slabs [G][rows][K]: rows = 2f for gate|up, n_out (= d) for down
+    const cuuint64_t rows = GATEUP ? (cuuint64_t)2 * f : (cuuint64_t)n_out;
+    const cuuint64_t bdims[3] = {(cuuint64_t)K, rows, (cuuint64_t)G};
+    const cuuint64_t bstr[2] = {(cuuint64_t)K * 2, rows * (cuuint64_t)K * 2};
+    const cuuint32_t bbox[3] = {GG_BK, (cuuint32_t)(GATEUP ? BN / 2 : BN), 1};
+    st = make_tmap(&tb, w, 3, bdims, bstr, bbox);
+    if (st != MOE_OK) return st;
+    GemmArgs args;
+    args.group_offsets = offsets;
+    args.G = G;
+    args.M = M;
+    args.K = K;
+    args.n_out = n_out;
+    args.f = f;
+    args.n_tiles = (n_out + S::OUT_COLS - 1) / S::OUT_COLS;
+    args.out = reinterpret_cast<__nv_bfloat16*>(out);
+    const long upper = ((long)M / GG_BM + G) * (long)args.n_tiles;  // >= the real tile count
+    const int grid = (int)(upper < sms ? upper : sms);
+    grouped_gemm_kernel<BN, STAGES, GATEUP><<<grid, GG_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args);
+    return check_launch(GATEUP ? "grouped_gemm_gateup" : "grouped_gemm_down");
+}
+
+moe_status_t check_gemm_args(const void* a, const void* w, const int32_t* offsets, int G, int M, int d, int f,
+                             const void* out) {
+    if (!a || !w || !offsets || !out) return fail(MOE_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(a) || !aligned16(w) || !aligned16(out))
+        return fail(MOE_ERR_INVALID_ARG, "activation, weight and output pointers must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return fail(MOE_ERR_INVALID_ARG, "offsets misaligned");
+    if (G < 1 || G > GG_MAX_GROUPS) return fail(MOE_ERR_INVALID_ARG, "G=%d outside [1, %d]", G, GG_MAX_GROUPS);
+    if (M < 0) return fail(MOE_ERR_INVALID_ARG, "M=%d < 0", M);
+    if (d < 8 || f < 8 || d % 8 || f % 8)
+        return fail(MOE_ERR_INVALID_ARG, "d=%d and f=%d must be positive multiples of 8", d, f);
+    return MOE_OK;
+}
+
+moe_status_t check_route_sizes(int T, int E, int k) {
+    if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d < 0", T);
+    if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", E);
+    if (k < 1 || k > E || k > 32) return fail(MOE_ERR_INVALID_ARG, "k=%d outside [1, min(E, 32)]", k);
+    if ((long)T * E > 0x7fffffffL || (long)T * k > 0x7fffffffL)
+        return fail(MOE_ERR_INVALID_ARG, "T*E or T*k exceeds int32");
+    return MOE_OK;
+}
+
+int grid_cap(long want, int sms, int per_sm) {
+    const long cap = (long)sms * per_sm;
+    if (want < 1) want = 1;
+    return (int)(want < cap ? want : cap);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const float* bias, int T, int d, int E,
+                            int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx, float* topk_w,
+                            cudaStream_t stream) {
+    moe_status_t st = check_route_sizes(T, E, k);
+    if (st != MOE_OK) return st;
+    if (mode < MOE_ROUTE_TOPK_SOFTMAX || mode > MOE_ROUTE_SIGMOID_TOPK_NORM)
+        return fail(MOE_ERR_INVALID_ARG, "unknown routing mode %d", (int)mode);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (!x || !w_router || !logits_out || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(w_router)) return fail(MOE_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    dim3 grid((T + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
+    router_logits_kernel<<<grid, RT_THREADS, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias,
+                                                         T, d, E, logits_out);
+    if ((st = check_launch("router_logits")) != MOE_OK) return st;
+    topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, stream>>>(logits_out, T, E, k, (int)mode,
+                                                                                  topk_idx, topk_w);
+    return check_launch("topk");
+}
+
+moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_route_mode_t mode,
+                                  int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+    moe_status_t st = check_route_sizes(T, E, k);
+    if (st != MOE_OK) return st;
+    if (mode < MOE_ROUTE_TOPK_SOFTMAX || mode > MOE_ROUTE_SIGMOID_TOPK_NORM)
+        return fail(MOE_ERR_INVALID_ARG, "unknown routing mode %d", (int)mode);
+    if (!logits || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, stream>>>(logits, T, E, k, (int)mode,
+                                                                                  topk_idx, topk_w);
+    return check_launch("topk");
+}
+
+size_t moe_permute_workspace_size(int T, int E, int k) {
+    if (T <= 0 || E <= 0 || k <= 0) return 0;
+    const size_t bytes = (size_t)perm_num_segments((long)T * k) * (size_t)E * sizeof(int32_t);
+    return (bytes + 255) / 256 * 256;
+}
+
+moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                         int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                         moe_bf16_t* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_route_sizes(T, E, k);
+    if (st != MOE_OK) return st;
+    if (!topk_idx || !expert_counts || !expert_offsets || !perm_src || !inv_perm)
+        return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if ((x == nullptr) != (x_perm == nullptr)) return fail(MOE_ERR_INVALID_ARG, "x and x_perm: give both or neither");
+    if (x) {
+        if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+        if (!aligned16(x) || !aligned16(x_perm)) return fail(MOE_ERR_INVALID_ARG, "x / x_perm not 16-byte aligned");
+        if ((long)T * k * (long)d > 0x7fffffffffffL) return fail(MOE_ERR_INVALID_ARG, "x_perm too large");
+    }
+    const size_t need = moe_permute_workspace_size(T, E, k);
+    if (need && (!ws || ws_bytes < need))
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : (size_t)0);
+    if (ws && (reinterpret_cast<uintptr_t>(ws) & 255u)) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    const int R = T * k;
+    if (R == 0) {  // no assignments: counts are zero, offsets all zero
+        cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), stream);
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+        return MOE_OK;
+    }
+    int32_t* seg = reinterpret_cast<int32_t*>(ws);
+    const int nseg = perm_num_segments(R);
+    permute_hist_kernel<<<nseg, PERM_THREADS, E * sizeof(int32_t), stream>>>(topk_idx, R, E, seg);
+    if ((st = check_launch("permute_hist")) != MOE_OK) return st;
+    permute_scan_kernel<<<1, 1024, 0, stream>>>(seg, nseg, E, expert_counts, expert_offsets);
+    if ((st = check_launch("permute_scan")) != MOE_OK) return st;
+    permute_scatter_kernel<<<nseg, PERM_THREADS, PERM_WARPS * E * sizeof(int32_t), stream>>>(topk_idx, R, E, k, seg,
+                                                                                            perm_src, inv_perm);
+    if ((st = check_launch("permute_scatter")) != MOE_OK) return st;
+    if (x) {
+        const int grid = grid_cap((R + 7) / 8, di.sms, 16);
+        gather_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), perm_src, R, T, d,
+                                                     reinterpret_cast<__nv_bfloat16*>(x_perm));
+        if ((st = check_launch("gather_rows")) != MOE_OK) return st;
+    }
+    return MOE_OK;
+}
+
+moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_gateup, const int32_t* group_offsets,
+                                     int G, int M, int d, int f, moe_bf16_t* h, cudaStream_t stream) {
+    moe_status_t st = check_gemm_args(a, w_gateup, group_offsets, G, M, d, f, h);
+    if (st != MOE_OK) return st;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    return launch_grouped_gemm<kBN, kStages, true>(a, w_gateup, group_offsets, G, M, d, f, f, h, di.sms, stream);
+}
+
+moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down, const int32_t* group_offsets,
+                                   int G, int M, int d, int f, moe_bf16_t* y, cudaStream_t stream) {
+    moe_status_t st = check_gemm_args(h, w_down, group_offsets, G, M, d, f, y);
+    if (st != MOE_OK) return st;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    return launch_grouped_gemm<kBN, kStages, false>(h, w_down, group_offsets, G, M, f, d, f, y, di.sms, stream);
+}
+
+moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w,
+                                   const moe_bf16_t* shared, int T, int d, int k, moe_bf16_t* y,
+                                   cudaStream_t stream) {
+    if (T < 0 || k < 1 || k > 32) return fail(MOE_ERR_INVALID_ARG, "T=%d, k=%d (need T >= 0, 1 <= k <= 32)", T, k);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (!y_perm || !inv_perm || !topk_w || !y) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(y_perm) || !aligned16(y) || (shared && !aligned16(shared)))
+        return fail(MOE_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    if ((long)T * k > 0x7fffffffL) return fail(MOE_ERR_INVALID_ARG, "T*k exceeds int32");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    if (T == 0) return MOE_OK;
+    const int grid = grid_cap((T + 7) / 8, di.sms, 16);
+    combine_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(y_perm), inv_perm, topk_w,
+                                             reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
+                                             reinterpret_cast<__nv_bfloat16*>(y));
+    return check_launch("unpermute_combine");
+}
+
+moe_status_t moe_get_device_error(unsigned int* out, cudaStream_t stream) {
+    if (!out) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    cudaError_t e = cudaStreamSynchronize(stream);
+    unsigned int v = 0;
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof v);
+    const unsigned int zero = 0;
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    *out = v;
+    return v ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+const char* moe_last_error_string(void) { return t_last_error.c_str(); }
+
+}  // extern "C"

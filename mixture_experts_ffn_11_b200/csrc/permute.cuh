@@ -1,0 +1,166 @@
+// Grouping of the T*k (token, slot) assignments by expert: "sort tokens by expert ID, group them"
+// (blog post "Mixture of Experts (MoEs) in Transformers", section "Expert Backend", grouped_mm),
+// as a stable counting sort: expert histogram -> exclusive scan -> stable scatter, then a gather of
+// x rows into expert-contiguous order ("dispatch tokens to their selected expert weights").
+//
+// Stability without atomics on positions: the assignments are cut into segments of
+// PERM_SEG = 8 warps x 512; segment histograms are scanned in segment order, and inside a segment
+// each warp walks its 512 assignments in order, ranking equal experts within 32 lanes with
+// __match_any_sync. Positions therefore depend only on the input, never on timing.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int PERM_WARPS = 8;
+constexpr int PERM_PER_WARP = 512;
+constexpr int PERM_SEG = PERM_WARPS * PERM_PER_WARP;  // assignments per segment (block)
+constexpr int PERM_THREADS = PERM_WARPS * 32;
+
+__host__ __device__ inline int perm_num_segments(long R) { return (int)((R + PERM_SEG - 1) / PERM_SEG); }
+
+// Per-segment expert histogram: seg_hist[s][e].
+__global__ void __launch_bounds__(PERM_THREADS) permute_hist_kernel(const int32_t* __restrict__ idx, int R, int E,
+                                                                    int32_t* __restrict__ seg_hist) {
+    extern __shared__ int32_t sh[];  // [E]
+    for (int e = threadIdx.x; e < E; e += PERM_THREADS) sh[e] = 0;
+    __syncthreads();
+    const long base = (long)blockIdx.x * PERM_SEG;
+    for (int i = threadIdx.x; i < PERM_SEG; i += PERM_THREADS) {
+        const long a = base + i;
+        if (a >= R) break;
+        const int e = idx[a];
+        if (e >= 0 && e < E)
+            atomicAdd(&sh[e], 1);
+        else
+            flag_error(MOE_DEVERR_EXPERT_RANGE);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += PERM_THREADS) seg_hist[(size_t)blockIdx.x * E + e] = sh[e];
+}
+
+// One block of 1024 threads, thread e handles expert e (E <= 1024):
+//   counts[e] = sum over segments; offsets = exclusive scan of counts (block-wide);
+//   seg_hist[s][e] <- offsets[e] + sum_{s' < s} seg_hist[s'][e]   (the segment's first row for e)
+__global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict__ seg_hist, int nseg, int E,
+                                                            int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+    __shared__ int32_t warp_tot[32];
+    const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    int total = 0;
+    if (e < E)
+        for (int s = 0; s < nseg; ++s) total += seg_hist[(size_t)s * E + e];
+    // inclusive warp scan
+    int incl = total;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int v = warp_tot[lane];
+        int vi = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, vi, o);
+            if (lane >= o) vi += u;
+        }
+        warp_tot[lane] = vi - v;  // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    const int excl = warp_tot[w] + incl - total;
+    if (e < E) {
+        counts[e] = total;
+        offsets[e] = excl;
+        if (e == E - 1) offsets[E] = excl + total;
+        int run = excl;
+        constexpr int B = 8;  // batch the loads so the running sum does not serialise on memory latency
+        for (int s0 = 0; s0 < nseg; s0 += B) {
+            int v[B];
+#pragma unroll
+            for (int b = 0; b < B; ++b) v[b] = (s0 + b < nseg) ? seg_hist[(size_t)(s0 + b) * E + e] : 0;
+#pragma unroll
+            for (int b = 0; b < B; ++b)
+                if (s0 + b < nseg) {
+                    seg_hist[(size_t)(s0 + b) * E + e] = run;
+                    run += v[b];
+                }
+        }
+    }
+}
+
+// Stable scatter: perm_src[row] = token, inv_perm[a] = row.
+__global__ void __launch_bounds__(PERM_THREADS) permute_scatter_kernel(const int32_t* __restrict__ idx, int R,
+                                                                       int E, int k,
+                                                                       const int32_t* __restrict__ seg_base,
+                                                                       int32_t* __restrict__ perm_src,
+                                                                       int32_t* __restrict__ inv_perm) {
+    extern __shared__ int32_t wh[];  // [PERM_WARPS][E]: warp histograms, then warp running row cursors
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < PERM_WARPS * E; i += PERM_THREADS) wh[i] = 0;
+    __syncthreads();
+    const long wbase = (long)blockIdx.x * PERM_SEG + (long)warp * PERM_PER_WARP;
+    int32_t* my = wh + warp * E;
+    for (int s = 0; s < PERM_PER_WARP / 32; ++s) {
+        const long a = wbase + s * 32 + lane;
+        if (a < R) {
+            const int e = idx[a];
+            if (e >= 0 && e < E) atomicAdd(&my[e], 1);
+        }
+    }
+    __syncthreads();
+    // cursor of warp w for expert e = segment base + rows taken by warps before w
+    for (int e = threadIdx.x; e < E; e += PERM_THREADS) {
+        int run = seg_base[(size_t)blockIdx.x * E + e];
+        for (int w = 0; w < PERM_WARPS; ++w) {
+            const int c = wh[w * E + e];
+            wh[w * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+    const unsigned lt = lanemask_lt();
+    for (int s = 0; s < PERM_PER_WARP / 32; ++s) {
+        const long a = wbase + s * 32 + lane;
+        int e = -1;
+        if (a < R) e = idx[a];
+        const bool valid = a < R && e >= 0 && e < E;
+        const int key = valid ? e : -1 - lane;  // invalid lanes never match anybody
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
+        int pos = 0;
+        if (valid) {
+            pos = my[e] + __popc(peers & lt);
+            perm_src[pos] = (int32_t)(a / k);
+            inv_perm[a] = pos;
+        } else if (a < R) {
+            inv_perm[a] = -1;
+        }
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) my[e] += __popc(peers);
+        __syncwarp();
+    }
+}
+
+// x_perm[r] = x[perm_src[r]]: one warp per row, 16-byte vectors (d is a multiple of 8).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const int32_t* __restrict__ perm_src, int R, int T,
+                                                          int d, __nv_bfloat16* __restrict__ x_perm) {
+    const int lane = threadIdx.x & 31;
+    const int nvec = d / 8;
+    const long nwarps = (long)gridDim.x * (blockDim.x / 32);
+    for (long r = (long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < R; r += nwarps) {
+        const int src = perm_src[r];
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)r * d);
+        if (src < 0 || src >= T) {
+            if (lane == 0) flag_error(MOE_DEVERR_ROW_RANGE);
+            for (int v = lane; v < nvec; v += 32) dst[v] = make_uint4(0, 0, 0, 0);
+            continue;
+        }
+        const uint4* s = reinterpret_cast<const uint4*>(x + (size_t)src * d);
+        for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(s + v);
+    }
+}
+
+}  // namespace moe

@@ -1,0 +1,92 @@
+"""The sparse MoE feed-forward layer as a sequence of C-ABI calls.
+
+Blog post "Mixture of Experts (MoEs) in Transformers": the layer keeps the transformer backbone and
+replaces the dense feed-forward block with experts and a router (section "From Dense to Sparse"); at
+run time it dispatches tokens to their selected experts, runs the projections, applies the routing
+weights and collects the results in token order (section "Expert Backend"), here the grouped_mm way:
+sort by expert id, group, one grouped GEMM over all experts.
+
+This module owns device buffers (allocated with torch; the library never allocates) and calls the five
+library entry points in order on one stream. It does no arithmetic of its own.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _native as N
+
+
+class MoEFFN:
+    """One MoE feed-forward layer with packed expert weights.
+
+    w_router [E, d] fp32; w_gateup [E, 2f, d] bf16 (gate rows, then up rows); w_down [E, d, f] bf16;
+    bias [E] fp32 or None; optional shared expert w_gateup_shared [2fs, d], w_down_shared [d, fs].
+    """
+
+    def __init__(self, w_router, w_gateup, w_down, k: int, route: str = "topk_softmax", bias=None,
+                 w_gateup_shared=None, w_down_shared=None):
+        self.E, self.d = w_router.shape
+        self.f = w_gateup.shape[1] // 2
+        self.k = k
+        self.route = route
+        if route not in N.ROUTE_MODES:
+            raise ValueError(f"unknown routing mode {route!r}")
+        self.w_router, self.w_gateup, self.w_down, self.bias = w_router, w_gateup, w_down, bias
+        self.w_gateup_shared, self.w_down_shared = w_gateup_shared, w_down_shared
+        self.shared_f = w_gateup_shared.shape[0] // 2 if w_gateup_shared is not None else 0
+        self.device = w_gateup.device
+        self._T = None
+        self.buf = {}
+
+    def buffers(self, T: int) -> dict:
+        """Allocate (once per T) every intermediate the layer writes."""
+        if self._T == T:
+            return self.buf
+        dev, E, d, f, k = self.device, self.E, self.d, self.f, self.k
+        R = T * k
+        i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
+        b = {
+            "logits": torch.empty(T, E, dtype=f32, device=dev),
+            "topk_idx": torch.empty(T, k, dtype=i32, device=dev),
+            "topk_w": torch.empty(T, k, dtype=f32, device=dev),
+            "counts": torch.empty(E, dtype=i32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=i32, device=dev),
+            "perm_src": torch.empty(R, dtype=i32, device=dev),
+            "inv_perm": torch.empty(R, dtype=i32, device=dev),
+            "x_perm": torch.empty(R, d, dtype=bf, device=dev),
+            "h": torch.empty(R, f, dtype=bf, device=dev),
+            "y_perm": torch.empty(R, d, dtype=bf, device=dev),
+            "ws": torch.empty(max(N.permute_workspace_size(T, E, k), 256), dtype=torch.uint8, device=dev),
+            "y": torch.empty(T, d, dtype=bf, device=dev),
+        }
+        if self.shared_f:
+            b["shared_offsets"] = torch.tensor([0, T], dtype=i32, device=dev)
+            b["h_shared"] = torch.empty(T, self.shared_f, dtype=bf, device=dev)
+            b["shared"] = torch.empty(T, d, dtype=bf, device=dev)
+        self.buf, self._T = b, T
+        return b
+
+    def forward(self, x, stream=None):
+        """y = MoE(x) for x [T, d] bf16 on the GPU. Returns the layer's output buffer [T, d] (bf16)."""
+        T = x.shape[0]
+        b = self.buffers(T)
+        N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"],
+                     stream)
+        N.permute(x, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], b["x_perm"],
+                  b["ws"], stream)
+        N.grouped_gemm_gateup(b["x_perm"], self.w_gateup, b["offsets"], b["h"], stream)
+        N.grouped_gemm_down(b["h"], self.w_down, b["offsets"], b["y_perm"], stream)
+        shared = None
+        if self.shared_f:
+            N.grouped_gemm_gateup(x, self.w_gateup_shared.unsqueeze(0), b["shared_offsets"], b["h_shared"], stream)
+            N.grouped_gemm_down(b["h_shared"], self.w_down_shared.unsqueeze(0), b["shared_offsets"], b["shared"],
+                                stream)
+            shared = b["shared"]
+        N.unpermute_combine(b["y_perm"], b["inv_perm"], b["topk_w"], shared, b["y"], stream)
+        return b["y"]
+
+    __call__ = forward
+
+    def kernel_launches(self, T: int) -> int:
+        """Kernels one forward() launches: route (2), permute (4), gate|up, down, combine (+2 shared)."""
+        return 9 + (2 if self.shared_f else 0) if T > 0 else 0

@@ -1,0 +1,331 @@
+"""Parity of the CUDA path (through the C-ABI) with the CPU oracle, on a B200.
+
+Inputs come from the seeded generator; expected values come only from the oracle. Integer results
+(routing indices, counts, offsets, permutation, gathered rows) must match bit for bit; the layer output
+must meet the bar in gpu_util (per element and relative Frobenius).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_util import bf16_bits_of, bf16_to_host_f32, check_close, to_dev_bf16
+
+pytestmark = pytest.mark.gpu
+
+N = pytest.importorskip("mixture_experts_ffn_11_b200._native")
+from mixture_experts_ffn_11_b200 import MoEFFN  # noqa: E402
+
+NEAR_TIE = 1e-5
+CONFIGS = ["tiny", "gpt-oss-20b-prefill", "mixtral-8x7b-prefill", "zipf-128e", "decode-256e-shared"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    synth.build_cuda()
+    torch.cuda.set_device(0)
+    N.get_device_error()  # clear
+    yield
+    torch.cuda.synchronize()
+
+
+_refs = {}
+
+
+def layer_ref(name):
+    if name not in _refs:
+        _refs[name] = oracle.LayerReference(synth.workload(name))
+    return _refs[name]
+
+
+# ---- generator -------------------------------------------------------------------------------------
+
+def test_device_generator_matches_host_bitwise():
+    for tid, first, count, sigma in ((0, 0, 100_003, 1.0), (2, 77_777, 50_000, 0.02), (3, 1 << 33, 4096, 0.02)):
+        t = torch.empty(count, dtype=torch.bfloat16, device="cuda")
+        synth.fill_device(t, 0, tid, first, sigma)
+        assert (bf16_bits_of(t) == synth.normal_bf16(0, tid, first, count, sigma)).all()
+    t = torch.empty(10_000, dtype=torch.float32, device="cuda")
+    synth.fill_device(t, 5, 1, 123, 0.02)
+    assert (t.cpu().numpy() == synth.normal_f32(5, 1, 123, 10_000, 0.02)).all()
+
+
+# ---- routing ---------------------------------------------------------------------------------------
+
+def _gpu_route(wl, x, w_router, bias):
+    T, E, k = wl.T, wl.E, wl.k
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    N.route_topk(x, w_router, bias, k, wl.route, logits, idx, w)
+    return logits, idx, w
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+def test_router_matches_oracle(name):
+    wl = synth.workload(name)
+    ref = layer_ref(name)
+    x = to_dev_bf16(ref.x)
+    wr = torch.from_numpy(ref.w_router).cuda()
+    bias = torch.from_numpy(ref.bias).cuda() if ref.bias is not None else None
+    logits, idx, w = _gpu_route(wl, x, wr, bias)
+    assert N.get_device_error() == 0
+    lg = logits.cpu().numpy().astype(np.float64)
+    scale = np.abs(ref.logits64).max()
+    assert np.abs(lg - ref.logits64).max() <= 1e-5 * max(scale, 1.0)
+    ties = set(ref.near_ties(NEAR_TIE).tolist())
+    keep = np.array([t for t in range(wl.T) if t not in ties], dtype=np.int64)
+    gi = idx.cpu().numpy()
+    assert (gi[keep] == ref.idx[keep]).all(), "routing indices differ outside near-ties"
+    np.testing.assert_allclose(w.cpu().numpy()[keep], ref.w[keep], rtol=2e-5, atol=2e-6)
+    print(f"{name}: {len(ties)} near-tie tokens excluded: {sorted(ties)[:16]}")
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+def test_topk_bit_exact_given_fp32_logits(name):
+    """Given the same fp32 logits (the oracle's), selection is identical for every token, no exclusions."""
+    wl = synth.workload(name)
+    ref = layer_ref(name)
+    logits = torch.from_numpy(ref.logits32).cuda()
+    idx = torch.empty(wl.T, wl.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(wl.T, wl.k, dtype=torch.float32, device="cuda")
+    N.topk_from_logits(logits, wl.k, wl.route, idx, w)
+    assert (idx.cpu().numpy() == ref.idx).all()
+    np.testing.assert_allclose(w.cpu().numpy(), ref.w, rtol=2e-6, atol=1e-7)
+
+
+def test_topk_ties_and_modes_small():
+    rng = np.random.default_rng(0)
+    for E, k in ((8, 2), (33, 5), (256, 8), (1024, 32), (3, 3)):
+        l = rng.integers(-2, 3, size=(97, E)).astype(np.float32)  # many exact ties
+        for mode in ("topk_softmax", "softmax_topk_renorm", "sigmoid_topk_norm"):
+            ri, rw = oracle.topk(l, k, mode)
+            idx = torch.empty(97, k, dtype=torch.int32, device="cuda")
+            w = torch.empty(97, k, dtype=torch.float32, device="cuda")
+            N.topk_from_logits(torch.from_numpy(l).cuda(), k, mode, idx, w)
+            assert (idx.cpu().numpy() == ri).all(), (E, k, mode)
+            np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
+
+
+# ---- permutation -----------------------------------------------------------------------------------
+
+def _gpu_permute(x_bits, idx_np, E):
+    T, k = idx_np.shape
+    R = T * k
+    d = x_bits.shape[1]
+    dev = "cuda"
+    out = dict(counts=torch.empty(E, dtype=torch.int32, device=dev),
+               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+               perm_src=torch.empty(R, dtype=torch.int32, device=dev),
+               inv_perm=torch.empty(R, dtype=torch.int32, device=dev),
+               x_perm=torch.empty(R, d, dtype=torch.bfloat16, device=dev),
+               ws=torch.empty(max(N.permute_workspace_size(T, E, k), 256), dtype=torch.uint8, device=dev))
+    x = to_dev_bf16(x_bits)
+    N.permute(x, torch.from_numpy(np.ascontiguousarray(idx_np, dtype=np.int32)).cuda(), E, out["counts"],
+              out["offsets"], out["perm_src"], out["inv_perm"], out["x_perm"], out["ws"])
+    return x, out
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+def test_permute_bit_exact(name):
+    wl = synth.workload(name)
+    ref = layer_ref(name)
+    _, out = _gpu_permute(ref.x, ref.idx, wl.E)
+    assert N.get_device_error() == 0
+    np.testing.assert_array_equal(out["counts"].cpu().numpy(), ref.counts)
+    np.testing.assert_array_equal(out["offsets"].cpu().numpy(), ref.offsets)
+    np.testing.assert_array_equal(out["perm_src"].cpu().numpy(), ref.perm_src)
+    np.testing.assert_array_equal(out["inv_perm"].cpu().numpy(), ref.inv_perm)
+    assert (bf16_bits_of(out["x_perm"]) == ref.x[ref.perm_src]).all()
+
+
+def test_permute_edge_sizes():
+    rng = np.random.default_rng(1)
+    for T, E, k in ((1, 1, 1), (1, 7, 7), (5000, 3, 2), (4097, 1024, 1), (2048, 16, 16), (9000, 64, 4)):
+        idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+        x_bits = synth.normal_bf16(9, 0, 0, T * 8, 1.0).reshape(T, 8)
+        _, out = _gpu_permute(x_bits, idx, E)
+        c, o, ps, ip = oracle.permute(idx, E)
+        np.testing.assert_array_equal(out["counts"].cpu().numpy(), c)
+        np.testing.assert_array_equal(out["offsets"].cpu().numpy(), o)
+        np.testing.assert_array_equal(out["perm_src"].cpu().numpy(), ps)
+        np.testing.assert_array_equal(out["inv_perm"].cpu().numpy(), ip)
+        assert (bf16_bits_of(out["x_perm"]) == x_bits[ps]).all()
+    assert N.get_device_error() == 0
+
+
+# ---- expert GEMMs + combine on ragged groups ---------------------------------------------------------
+
+def _gpu_experts(x_bits, gu_bits, dn_bits, idx, w32, shared=None):
+    """permute -> gate|up -> down -> combine on the GPU for a given routing."""
+    T, d = x_bits.shape
+    E, two_f, _ = gu_bits.shape
+    f = two_f // 2
+    k = idx.shape[1]
+    R = T * k
+    x, p = _gpu_permute(x_bits, idx, E)
+    wgu, wdn = to_dev_bf16(gu_bits), to_dev_bf16(dn_bits)
+    h = torch.empty(R, f, dtype=torch.bfloat16, device="cuda")
+    y_perm = torch.empty(R, d, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    N.grouped_gemm_gateup(p["x_perm"], wgu, p["offsets"], h)
+    N.grouped_gemm_down(h, wdn, p["offsets"], y_perm)
+    sh = None
+    if shared is not None:
+        sgu, sdn = to_dev_bf16(shared[0]), to_dev_bf16(shared[1])
+        fs = shared[0].shape[0] // 2
+        so = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+        hs = torch.empty(T, fs, dtype=torch.bfloat16, device="cuda")
+        sh = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        N.grouped_gemm_gateup(x, sgu.unsqueeze(0), so, hs)
+        N.grouped_gemm_down(hs, sdn.unsqueeze(0), so, sh)
+    N.unpermute_combine(y_perm, p["inv_perm"], torch.from_numpy(w32).cuda(), sh, y)
+    assert N.get_device_error() == 0
+    return bf16_to_host_f32(y), p
+
+
+def _routing_with_counts(counts, k, rng):
+    """Assignments (T = sum(counts)/k tokens, k distinct experts each) realising the given expert counts."""
+    E = len(counts)
+    if k == 1:
+        idx = np.concatenate([np.full(c, e) for e, c in enumerate(counts)]).astype(np.int32)
+        rng.shuffle(idx)
+        return idx.reshape(-1, 1)
+    raise ValueError("k == 1 only")
+
+
+RAGGED = [
+    # (name, counts per expert, d, f)
+    ("empty_single_tail_full", [0, 1, 127, 128, 129, 257, 0], 200, 72),
+    ("one_expert_takes_all", [0, 0, 300, 0], 256, 512),
+    ("many_small", [3] * 40 + [0] * 24, 64, 96),
+    ("wide_k_tail", [130, 5], 1000, 264),
+]
+
+
+@pytest.mark.parametrize("name,counts,d,f", RAGGED, ids=[r[0] for r in RAGGED])
+def test_ragged_groups_match_oracle(name, counts, d, f):
+    rng = np.random.default_rng(2)
+    E = len(counts)
+    idx = _routing_with_counts(counts, 1, rng)
+    T = idx.shape[0]
+    x = synth.normal_bf16(3, 0, 0, T * d, 1.0).reshape(T, d)
+    gu = synth.normal_bf16(3, 2, 0, E * 2 * f * d, 0.05).reshape(E, 2 * f, d)
+    dn = synth.normal_bf16(3, 3, 0, E * d * f, 0.05).reshape(E, d, f)
+    w = np.ones((T, 1), dtype=np.float32)
+    y, p = _gpu_experts(x, gu, dn, idx, w)
+    np.testing.assert_array_equal(p["counts"].cpu().numpy(), counts)
+    ref = oracle.moe_tokens(x, list(gu), list(dn), idx, w.astype(np.float64), np.arange(T))
+    check_close(y, ref, name)
+
+
+def test_k2_random_routing_with_shared_expert():
+    rng = np.random.default_rng(3)
+    T, d, f, E, k, fs = 333, 128, 384, 5, 2, 136
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    x = synth.normal_bf16(4, 0, 0, T * d, 1.0).reshape(T, d)
+    gu = synth.normal_bf16(4, 2, 0, E * 2 * f * d, 0.05).reshape(E, 2 * f, d)
+    dn = synth.normal_bf16(4, 3, 0, E * d * f, 0.05).reshape(E, d, f)
+    sgu = synth.normal_bf16(4, 5, 0, 2 * fs * d, 0.05).reshape(2 * fs, d)
+    sdn = synth.normal_bf16(4, 6, 0, d * fs, 0.05).reshape(d, fs)
+    y, _ = _gpu_experts(x, gu, dn, idx, w, shared=(sgu, sdn))
+    ref = oracle.moe_tokens(x, list(gu), list(dn), idx, w.astype(np.float64), np.arange(T), sgu, sdn)
+    check_close(y, ref, "k2+shared")
+
+
+def test_identical_experts_equal_dense_swiglu():
+    """All experts equal: the layer is one dense SwiGLU whatever the routing (weights sum to 1)."""
+    rng = np.random.default_rng(5)
+    T, d, f, E, k = 256, 256, 256, 8, 2
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    w = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    x = synth.normal_bf16(5, 0, 0, T * d, 1.0).reshape(T, d)
+    gu1 = synth.normal_bf16(5, 2, 0, 2 * f * d, 0.05).reshape(2 * f, d)
+    dn1 = synth.normal_bf16(5, 3, 0, d * f, 0.05).reshape(d, f)
+    y, _ = _gpu_experts(x, np.stack([gu1] * E), np.stack([dn1] * E), idx, w)
+    ref = oracle.moe_tokens(x, [gu1], [dn1], np.zeros((T, 1), np.int32), np.ones((T, 1)), np.arange(T))
+    check_close(y, ref, "identical experts")
+
+
+# ---- full layer at the benchmark's sizes -------------------------------------------------------------
+
+SAMPLE = {"tiny": None, "gpt-oss-20b-prefill": 48, "mixtral-8x7b-prefill": 24, "zipf-128e": 48,
+          "decode-256e-shared": 8}
+
+
+def _sample_tokens(ref, n, rng):
+    wl = ref.wl
+    if n is None:
+        return np.arange(wl.T)
+    toks = set(rng.choice(wl.T, size=n, replace=False).tolist())
+    nonempty = np.nonzero(ref.counts)[0]
+    for e in (nonempty[np.argmin(ref.counts[nonempty])], int(np.argmax(ref.counts))):
+        rows = np.nonzero((ref.idx == e).any(axis=1))[0]
+        toks.update(rng.choice(rows, size=min(8, len(rows)), replace=False).tolist())
+    return np.array(sorted(toks), dtype=np.int32)
+
+
+@pytest.mark.parametrize("name", CONFIGS)
+def test_full_layer_matches_oracle(name):
+    wl = synth.workload(name)
+    ref = layer_ref(name)
+    inp = synth.device_inputs(wl)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
+                   inp["w_gateup_shared"], inp["w_down_shared"])
+    y = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
+    # the device inputs are the oracle's inputs
+    assert (bf16_bits_of(inp["x"]) == ref.x).all()
+    gi = layer.buf["topk_idx"].cpu().numpy()
+    ties = set(ref.near_ties(NEAR_TIE).tolist())
+    toks = [t for t in _sample_tokens(ref, SAMPLE[name], np.random.default_rng(0)) if t not in ties]
+    toks = np.array(toks, dtype=np.int32)
+    assert (gi[toks] == ref.idx[toks]).all()
+    yh = bf16_to_host_f32(y)[toks]
+    want = ref.outputs(toks)
+    fro = check_close(yh, want, name)
+    print(f"{name}: {len(toks)} tokens compared, relative Frobenius error {fro:.2e}")
+    # run again: bitwise identical (deterministic path)
+    y2 = layer(inp["x"])
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+
+
+def test_layer_is_deterministic():
+    wl = synth.workload("gpt-oss-20b-prefill", T=1024)
+    inp = synth.device_inputs(wl)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route)
+    a = layer(inp["x"]).clone()
+    b = layer(inp["x"]).clone()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    # permuting the tokens permutes the output rows exactly (rows never interact)
+    perm = torch.randperm(wl.T, generator=torch.Generator().manual_seed(0)).cuda()
+    c = layer(inp["x"][perm].contiguous()).clone()
+    assert torch.equal(c.view(torch.int16), a[perm].view(torch.int16))
+
+
+# ---- device-side anomalies are reported, not faulted -------------------------------------------------
+
+def test_expert_id_out_of_range_is_flagged():
+    T, E, k, d = 100, 4, 2, 16
+    idx = np.tile(np.array([[0, 1]], np.int32), (T, 1))
+    idx[7, 1] = E  # out of range
+    x_bits = synth.normal_bf16(1, 0, 0, T * d, 1.0).reshape(T, d)
+    _gpu_permute(x_bits, idx, E)
+    err = N.get_device_error()
+    assert err & 0x2
+    assert N.get_device_error() == 0  # read clears
+
+
+def test_bad_group_offsets_are_flagged():
+    M, d, f = 200, 64, 64
+    a = torch.zeros(M, d, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(3, 2 * f, d, dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros(M, f, dtype=torch.bfloat16, device="cuda")
+    offs = torch.tensor([0, 100, 50, 500], dtype=torch.int32, device="cuda")  # decreasing, and past M
+    N.grouped_gemm_gateup(a, w, offs, h)
+    assert N.get_device_error() & 0x4
