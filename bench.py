@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MoE feed-forward layer on B200.
+
+One step = one pass of the whole layer (route -> permute -> gate|up grouped GEMM + SwiGLU -> down grouped
+GEMM -> weighted combine) over one batch of seeded synthetic tokens, through the library's public API.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line (rank 0). Device timing: CUDA events on the launching stream around each step, L2
+flushed (256 MiB write) before every step outside the events, max over ranks. `e2e` repeats the step with
+the input copied from pinned host memory and the output copied back inside the timed region. Multi-GPU
+runs are independent replicas (the layer has no cross-GPU exchange): weak scaling, value = all tokens / time.
+`--impl reference` times the CPU oracle (plain fp64 C, all host cores) on a bounded token sample.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s and achieved TFLOP/s or HBM GB/s vs roofline, 1×B200"
+DEFAULT_WORKLOAD = "gpt-oss-20b-prefill"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu capture, keyed by the
+# kernel, the workload and a hash of the kernel's source files at capture time. A stale hash -> null.
+TRAFFIC = {}
+KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/gemm.cuh", "mixture_experts_ffn_11_b200/csrc/sm100.cuh",
+                  "mixture_experts_ffn_11_b200/csrc/common.cuh"]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--settle-seconds", type=float, default=2.0,
+                    help="extra untimed load after the warm-up so clocks and power settle")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    return args
+
+
+# ---- distributed plumbing (replicas) ----------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+
+    rank, local, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, local, world
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---- clocks ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock, power and throttle reasons for one GPU while the benchmark runs."""
+
+    FIELDS = ["timestamp", "uuid", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS),
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.out.flush()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        rows = []
+        self.out.seek(0)
+        for line in self.out.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            if self.uuid and self.uuid not in parts[1]:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[4], parts[6:]))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if len(inside) < 3:  # short timed region: include the preceding second of the same load (warm-up)
+            inside = [r for r in rows if t0 - 1.0 <= r[0] <= t1]
+            window = "timed region + preceding 1 s of identical warm-up load"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[4]) if v.lower().startswith("active")})
+        powers = [float(r[3]) for r in inside if r[3].replace(".", "", 1).isdigit()]
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window": window,
+                "power_w_max": max(powers) if powers else None}
+
+
+# ---- roofline arithmetic -------------------------------------------------------------------------------
+
+def gemm_figures(wl, counts):
+    """Algorithmic FLOPs and DRAM bytes per launch of the two grouped GEMMs, from the realised routing."""
+    R, d, f = wl.R, wl.d, wl.f
+    active = int((counts > 0).sum())
+    gateup = {"flop": 4.0 * R * d * f, "bytes": active * 2 * f * d * 2 + R * d * 2 + R * f * 2}
+    down = {"flop": 2.0 * R * f * d, "bytes": active * d * f * 2 + R * f * 2 + R * d * 2}
+    return active, gateup, down
+
+
+def layer_figures(wl, active):
+    flop = wl.flops()
+    bytes_ = (active * 3 * wl.d * wl.f * 2 + 3 * wl.d * wl.shared_f * 2 + wl.T * wl.d * 2 * 2 + wl.E * wl.d * 4)
+    return flop, bytes_
+
+
+def roofline_entry(name, fig, t_ms, peaks, peak_kind, traffic_bytes):
+    t_flop = fig["flop"] / (peaks[peak_kind] * 1e12)
+    t_byte = fig["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if t_flop >= t_byte:
+        achieved = fig["flop"] / (t_ms * 1e-3) / 1e12
+        return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 2), "peak": peaks[peak_kind],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks[peak_kind], 4), "traffic": traffic_bytes,
+                "algorithmic_flop": fig["flop"], "algorithmic_bytes": fig["bytes"], "launch_ms": round(t_ms, 5)}
+    achieved = fig["bytes"] / (t_ms * 1e-3) / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic_bytes,
+            "algorithmic_flop": fig["flop"], "algorithmic_bytes": fig["bytes"], "launch_ms": round(t_ms, 5)}
+
+
+# ---- CPU oracle (baseline and reference arm) ------------------------------------------------------------
+
+class OracleStep:
+    """One pass of the oracle over a token sample: router logits, top-k, grouping, per-token expert loop."""
+
+    def __init__(self, wl):
+        import numpy as np
+
+        import oracle
+        import synth
+
+        self.np, self.oracle, self.wl = np, oracle, wl
+        self.x = synth.x_host(wl)
+        self.wr = synth.w_router_host(wl)
+        self.bias = synth.zipf_bias(wl)
+        self.order = np.random.default_rng(1234).permutation(wl.T).astype(np.int32)
+        self.gu = [None] * wl.E
+        self.dn = [None] * wl.E
+        self.shared = synth.shared_host(wl) if wl.shared_f else (None, None)
+        self.threads = max(1, len(os.sched_getaffinity(0)))
+
+    def prepare(self, n):
+        """Generate the experts the first n sampled tokens select (outside any timing)."""
+        import synth
+
+        toks = self.order[:n]
+        l = self.oracle.router_logits(self.x[toks], self.wr, self.bias).astype(self.np.float32)
+        idx, _ = self.oracle.topk(l, self.wl.k, self.wl.route)
+        for e in self.np.unique(idx):
+            if self.gu[e] is None:
+                self.gu[e] = synth.w_gateup_expert_host(self.wl, int(e))
+                self.dn[e] = synth.w_down_expert_host(self.wl, int(e))
+
+    def run(self, n):
+        o, np = self.oracle, self.np
+        xs = self.x[self.order[:n]]
+        l64 = o.router_logits(xs, self.wr, self.bias)
+        idx, w = o.topk(l64.astype(np.float32), self.wl.k, self.wl.route)
+        o.permute(idx, self.wl.E)
+        return o.moe_tokens(xs, self.gu, self.dn, idx, w, np.arange(n, dtype=np.int32), self.shared[0],
+                            self.shared[1], nthreads=self.threads)
+
+
+def calibrate_sample(step: OracleStep, seconds: float, cap: int) -> int:
+    n0 = min(8, cap)
+    step.prepare(n0)
+    t = time.perf_counter()
+    step.run(n0)
+    per_tok = max((time.perf_counter() - t) / n0, 1e-6)
+    return int(max(1, min(cap, seconds / per_tok)))
+
+
+def cpu_baseline(wl, seconds: float) -> dict:
+    step = OracleStep(wl)
+    n = calibrate_sample(step, seconds, wl.T)
+    step.prepare(n)
+    t = time.perf_counter()
+    step.run(n)
+    dt = time.perf_counter() - t
+    return {"value": round(n / dt, 3), "unit": "tokens/s", "cores": step.threads, "kind": "oracle",
+            "sample": f"{n} of the {wl.T} tokens (seeded sample), whole layer per token in fp64 "
+                      f"(router, top-k, grouping, per-token expert loop), {dt:.1f} s wall"}
+
+
+def workload_config(wl) -> dict:
+    return {"workload": wl.name, "T": wl.T, "d": wl.d, "f": wl.f, "E": wl.E, "k": wl.k, "route": wl.route,
+            "shared_f": wl.shared_f, "zipf_s": wl.zipf_s, "seed": wl.seed,
+            "l2": "flushed (256 MiB write) before every timed step, outside the events"}
+
+
+DATA = "synthetic: seeded generator, x ~N(0,1) bf16, weights ~N(0,0.02) (random init, no checkpoint)"
+
+
+def run_reference(args):
+    import synth
+
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    wl = synth.workload(args.workload)
+    step = OracleStep(wl)
+    budget = 150.0 / max(1, args.steps + args.warmup)  # whole run within a few minutes
+    n = calibrate_sample(step, budget, wl.T)
+    step.prepare(n)
+    for _ in range(args.warmup):
+        step.run(n)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        step.run(n)
+        times.append(time.perf_counter() - t)
+    ms = 1e3 * sum(times) / len(times)
+    value = n / (ms * 1e-3)
+    sample = f"{n} of the {wl.T} tokens per step (seeded sample); oracle in fp64 on {step.threads} host threads"
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": DATA, "config": workload_config(wl),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": step.threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- our arm --------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import synth
+    from mixture_experts_ffn_11_b200 import MoEFFN, get_device_error
+
+    rank, local, world = dist_init("nccl")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = synth.workload(args.workload)
+    synth.build_cuda()
+    inp = synth.device_inputs(wl, dev)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
+                   inp["w_gateup_shared"], inp["w_down_shared"])
+    x = inp["x"]
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    launches_per_step = layer.kernel_launches(wl.T)
+    sampler = ClockSampler(torch.cuda.get_device_properties(dev).uuid.__str__() if rank >= 0 else None)
+    sampler.start()
+
+    def step(timing=None):
+        return layer.forward(x, timing=timing)
+
+    # warm-up: W steps, then keep the same load going for ~2 s so clocks and power settle
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    t_end = time.perf_counter() + args.settle_seconds
+    while time.perf_counter() < t_end:
+        flush.zero_()
+        step()
+        torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(dev)
+    if get_device_error():
+        raise SystemExit("device error word set during warm-up")
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    stage_ev = [dict() for _ in range(K)]
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(timing=stage_ev[i])
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    t1 = time.time()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), dev)
+    ms_per_step = total_ms / K
+    stages = {}
+    for name in stage_ev[0]:
+        stages[name] = statistics.mean(a.elapsed_time(b) for a, b in (s[name] for s in stage_ev))
+    err = get_device_error()
+    if err:
+        raise SystemExit(f"device error word {err:#x} set during the timed region")
+
+    # end to end: pinned host input -> device, layer, device -> pinned host output, every step
+    e2e = None
+    if not args.no_e2e:
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory()
+        x_dev = torch.empty_like(x)
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            y = layer.forward(x_dev)
+            y_host.copy_(y, non_blocking=True)
+
+        for _ in range(args.warmup):
+            flush.zero_()
+            e2e_step()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        for i in range(K):
+            flush.zero_()
+            ev2[i][0].record(stream)
+            e2e_step()
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), dev) / K
+        nbytes = wl.T * wl.d * 2
+        e2e = {"value": round(world * wl.T / (e2e_ms * 1e-3), 1), "unit": "tokens/s", "ms_per_step": round(e2e_ms, 4),
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "path": "pinned host x -> device (copy on the layer stream), MoEFFN.forward, device y -> pinned host"}
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    counts = layer.buf["counts"].cpu().numpy()
+    active, fig_gu, fig_dn = gemm_figures(wl, counts)
+    peaks, peak_src = load_peaks()
+    peak_kind = "bf16_tflops_sustained" if total_ms > 1000.0 else "bf16_tflops"
+    src_hash = kernel_source_hash()
+    tr = TRAFFIC.get(("grouped_gemm_gateup", wl.name, src_hash))
+    roof = roofline_entry("grouped_gemm_gateup", fig_gu, stages["gateup"], peaks, peak_kind, tr)
+    roof["peak_source"] = f"{peak_src} {'hbm_gbs' if roof['bound'] == 'hbm' else peak_kind}"
+    roof_dn = roofline_entry("grouped_gemm_down", fig_dn, stages["down"], peaks, peak_kind,
+                             TRAFFIC.get(("grouped_gemm_down", wl.name, src_hash)))
+    lflop, lbytes = layer_figures(wl, active)
+    t_roof = max(lflop / (peaks[peak_kind] * 1e12), lbytes / (peaks["hbm_gbs"] * 1e9))
+    line = {"metric": METRIC, "value": round(world * wl.T / (ms_per_step * 1e-3), 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": DATA,
+            "config": workload_config(wl), "roofline": roof, "roofline_down": roof_dn,
+            "layer_roofline": {"flop": lflop, "bytes": lbytes, "active_experts": active,
+                               "t_roofline_ms": round(t_roof * 1e3, 5),
+                               "frac": round(t_roof * 1e3 / ms_per_step, 4),
+                               "achieved_tflops": round(lflop / (ms_per_step * 1e-3) / 1e12, 2)},
+            "breakdown_ms": {k: round(v, 5) for k, v in stages.items()},
+            "gpu_launches": K * launches_per_step, "clocks": clocks, "e2e": e2e,
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

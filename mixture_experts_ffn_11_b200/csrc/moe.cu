@@ -12,6 +12,7 @@
 #include "moe.h"
 #include "common.cuh"
 #include "route.cuh"
+#include "route_tc.cuh"
 #include "permute.cuh"
 #include "gemm.cuh"
 #include "combine.cuh"
@@ -46,6 +47,27 @@ constexpr int kBN = 256;
 using GateUpShape = GemmShape<kBN, kStages, true>;
 using DownShape = GemmShape<kBN, kStages, false>;
 
+constexpr int kRouterSmallMaxSmem = 200 * 1024;  // W_r rows staged by the small-T router kernel
+constexpr int kRouterTcMinT = 2048;               // token count from which the tensor-core router pays off
+
+template <int BNR>
+cudaError_t set_router_tc_attr() {
+    return cudaFuncSetAttribute(router_tc_kernel<BNR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                RouterTcShape<BNR>::SMEM_BYTES);
+}
+
+cudaError_t set_router_attributes() {
+    cudaError_t e = set_router_tc_attr<16>();
+    if (e == cudaSuccess) e = set_router_tc_attr<32>();
+    if (e == cudaSuccess) e = set_router_tc_attr<64>();
+    if (e == cudaSuccess) e = set_router_tc_attr<128>();
+    if (e == cudaSuccess) e = set_router_tc_attr<256>();
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(router_logits_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kRouterSmallMaxSmem);
+    return e;
+}
+
 struct DeviceInfo {
     bool ready = false;
     bool sm100 = false;
@@ -76,8 +98,9 @@ moe_status_t device_info(DeviceInfo& out) {
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(grouped_gemm_kernel<kBN, kStages, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, DownShape::SMEM_BYTES);
+            if (e == cudaSuccess) e = set_router_attributes();
             if (e != cudaSuccess)
-                return fail(MOE_ERR_CUDA, "cudaFuncSetAttribute(grouped GEMM): %s", cudaGetErrorString(e));
+                return fail(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         }
         di.ready = true;
     }
@@ -194,10 +217,46 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
     if (T == 0) return MOE_OK;
-    dim3 grid((T + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
-    router_logits_kernel<<<grid, RT_THREADS, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), w_router, bias,
-                                                         T, d, E, logits_out);
-    if ((st = check_launch("router_logits")) != MOE_OK) return st;
+    const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    if (E <= 256 && T >= kRouterTcMinT) {
+        // tensor cores, W_r split into three bf16 pieces; top-k fused when k <= 8
+        CUtensorMap tm;
+        const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
+        const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+        const cuuint32_t box[2] = {RTC_BK, RTC_BM};
+        if ((st = make_tmap(&tm, x, 2, dims, strides, box)) != MOE_OK) return st;
+        const int fuse = k <= RTC_KMAX ? 1 : 0;
+        const int grid = (T + RTC_BM - 1) / RTC_BM;
+        if (E <= 16)
+            router_tc_kernel<16><<<grid, RTC_THREADS, RouterTcShape<16>::SMEM_BYTES, stream>>>(
+                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+        else if (E <= 32)
+            router_tc_kernel<32><<<grid, RTC_THREADS, RouterTcShape<32>::SMEM_BYTES, stream>>>(
+                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+        else if (E <= 64)
+            router_tc_kernel<64><<<grid, RTC_THREADS, RouterTcShape<64>::SMEM_BYTES, stream>>>(
+                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+        else if (E <= 128)
+            router_tc_kernel<128><<<grid, RTC_THREADS, RouterTcShape<128>::SMEM_BYTES, stream>>>(
+                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+        else
+            router_tc_kernel<256><<<grid, RTC_THREADS, RouterTcShape<256>::SMEM_BYTES, stream>>>(
+                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+        if ((st = check_launch("router_tc")) != MOE_OK) return st;
+        if (fuse) return MOE_OK;
+    } else if ((size_t)d * sizeof(float) <= (size_t)kRouterSmallMaxSmem) {
+        // few tokens: CUDA cores, parallel over experts so every SM streams part of W_r
+        int epb = E >= 2 * di.sms ? 4 : (E >= di.sms ? 2 : 1);
+        while (epb > 1 && (size_t)epb * d * sizeof(float) > (size_t)kRouterSmallMaxSmem) --epb;
+        const int grid = (E + epb - 1) / epb;
+        router_logits_small_kernel<<<grid, RS_THREADS, (size_t)epb * d * sizeof(float), stream>>>(
+            xb, w_router, bias, T, d, E, epb, logits_out);
+        if ((st = check_launch("router_logits_small")) != MOE_OK) return st;
+    } else {
+        dim3 grid((T + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
+        router_logits_kernel<<<grid, RT_THREADS, 0, stream>>>(xb, w_router, bias, T, d, E, logits_out);
+        if ((st = check_launch("router_logits")) != MOE_OK) return st;
+    }
     topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, stream>>>(logits_out, T, E, k, (int)mode,
                                                                                   topk_idx, topk_w);
     return check_launch("topk");

@@ -1,0 +1,341 @@
+// Router on the tensor cores, for large token counts, with top-k fused into the epilogue.
+//
+// logits[t][e] = sum_i x[t][i] * W_r[e][i] + bias[e] with x bf16 and W_r fp32. The fp32 weights are split
+// on the fly into three bf16 pieces, W_r = hi + mid + lo (hi = bf16(w), mid = bf16(w - hi),
+// lo = bf16(w - hi - mid); both differences are exact in fp32), so the product is three bf16 MMAs into one
+// fp32 accumulator: x*hi + x*mid + x*lo, which carries ~24 bits of W_r (relative error ~2^-27 per
+// weight). bf16*bf16 products are exact in fp32, so the logits keep fp32 accuracy.
+//
+// One CTA per 128-token tile (192 threads):
+//   warp 0     TMA of the x tile [128 x 64] per K step into a STAGES-deep ring
+//   warp 1     TMEM allocation; one lane issues 3 x 4 tcgen05.mma (M=128, N=BNR, K=16) per K step
+//   warps 2-5  convert the W_r block [BNR x 64] to the three swizzled bf16 pieces in shared memory (the
+//              same 128-byte-swizzled K-major layout the TMA engine writes), then, as the epilogue, read
+//              their 32 accumulator lanes: + bias, store the logits row, select the top-k (k <= 8) by
+//              insertion in descending order (equal logits keep the lower expert id first) and write the
+//              routing weights.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 192, RTC_KMAX = 8;
+
+template <int BNR>
+struct RouterTcShape {
+    static_assert(BNR % 16 == 0 && BNR >= 16 && BNR <= 256, "UMMA N");
+    static constexpr int STAGES = BNR >= 256 ? 2 : (BNR >= 128 ? 3 : 4);
+    static constexpr int A_BYTES = RTC_BM * RTC_BK * 2;
+    static constexpr int P_BYTES = BNR * RTC_BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
+    static constexpr int TMEM_COLS = BNR <= 32 ? 32 : (BNR <= 64 ? 64 : (BNR <= 128 ? 128 : 256));
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void split3_bf16(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+    hi = *reinterpret_cast<const uint16_t*>(&h);
+    mid = *reinterpret_cast<const uint16_t*>(&m);
+    lo = *reinterpret_cast<const uint16_t*>(&l);
+}
+
+template <int BNR>
+__global__ void __launch_bounds__(RTC_THREADS, 1)
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const float* __restrict__ w_router,
+                     const float* __restrict__ bias, int T, int d, int E, int k, int mode, int fuse_topk,
+                     float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    using S = RouterTcShape<BNR>;
+    constexpr int STAGES = S::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
+    uint64_t* empty_bar = full_bar + STAGES;
+    uint64_t* tfull_bar = empty_bar + STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * RTC_BM;
+    const int KB = (d + RTC_BK - 1) / RTC_BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1 + 128);  // TMA expect_tx arrival + 128 converter threads
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(tfull_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmX);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, S::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        bool ok = true;
+        const uint64_t pol = l2_policy_evict_first();
+        for (int kb = 0; kb < KB; ++kb) {
+            if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES);
+                tma_load_2d(smem + stage * S::STAGE_BYTES, &tmX, &full_bar[stage], kb * RTC_BK, m0, pol);
+            }
+            ++issued;
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (lane == 0)
+            for (int n = issued > STAGES ? issued - STAGES : 0; n < issued; ++n)
+                mbar_wait_drain(&full_bar[n % STAGES], (uint32_t)((n / STAGES) & 1));
+        __syncwarp();
+    } else if (warp == 1) {
+        constexpr uint32_t IDESC = idesc_bf16_f32(RTC_BM, BNR);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (lane == 0) {
+                const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
+                const uint64_t adesc = smem_desc_sw128(sa);
+#pragma unroll
+                for (int p = 0; p < 3; ++p) {
+                    const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + p * S::P_BYTES);
+#pragma unroll
+                    for (int kk = 0; kk < RTC_BK / 16; ++kk)
+                        umma_bf16_ss(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | p | kk) != 0 ? 1u : 0u);
+                }
+                umma_commit(&empty_bar[stage]);
+            }
+            __syncwarp();
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        if (lane == 0) umma_commit(tfull_bar);  // also the last MMA's completion before TMEM is freed
+        __syncwarp();
+    } else {
+        // ---- converters: W_r [E][d] fp32 -> hi/mid/lo bf16 pieces, swizzled K-major ----
+        const int ct = threadIdx.x - 64;  // 0..127
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        constexpr int ITEMS = BNR * (RTC_BK / 8) / 128;  // 16-byte output chunks per thread per piece
+        for (int kb = 0; kb < KB && ok; ++kb) {
+            if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            uint8_t* pbase = smem + stage * S::STAGE_BYTES + S::A_BYTES;
+            const int k0 = kb * RTC_BK;
+#pragma unroll 4
+            for (int it = 0; it < ITEMS; ++it) {
+                const int item = ct + 128 * it;
+                const int r = item >> 3, c = item & 7;
+                float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+                if (r < E && k0 + c * 8 < d) {
+                    const float4* src = reinterpret_cast<const float4*>(w_router + (size_t)r * d + k0 + c * 8);
+                    v0 = __ldg(src);
+                    v1 = __ldg(src + 1);
+                }
+                const float w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                uint32_t hi[4], mi[4], lo[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint16_t h0, m0_, l0, h1, m1, l1;
+                    split3_bf16(w8[2 * j], h0, m0_, l0);
+                    split3_bf16(w8[2 * j + 1], h1, m1, l1);
+                    hi[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+                    mi[j] = (uint32_t)m0_ | ((uint32_t)m1 << 16);
+                    lo[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
+                }
+                const int off = r * 128 + ((c ^ (r & 7)) << 4);
+                *reinterpret_cast<uint4*>(pbase + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(pbase + S::P_BYTES + off) = make_uint4(mi[0], mi[1], mi[2], mi[3]);
+                *reinterpret_cast<uint4*>(pbase + 2 * S::P_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor core
+            mbar_arrive(&full_bar[stage]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
+        // ---- epilogue ----
+        if (ok) {
+            if (lane == 0) ok = mbar_wait_bounded(tfull_bar, 0, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        if (ok) {
+            tc_fence_after_sync();
+            const int q = warp & 3;
+            const int row = m0 + q * 32 + lane;
+            const bool valid = row < T;
+            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+            float tv[RTC_KMAX];
+            int te[RTC_KMAX];
+#pragma unroll
+            for (int i = 0; i < RTC_KMAX; ++i) {
+                tv[i] = 0.f;
+                te[i] = INT_MAX;
+            }
+            float* lrow = logits + (size_t)(valid ? row : 0) * E;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BNR; c0 += 32) {
+                if (c0 >= E) break;
+                uint32_t v[32];
+                tmem_load_32cols(t_row + c0, v);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int e = c0 + j;
+                    if (e < E) {
+                        float cv = __uint_as_float(v[j]) + (bias ? __ldg(bias + e) : 0.f);
+                        if (valid) lrow[e] = cv;
+                        if (fuse_topk) {
+                            int ce = e;
+#pragma unroll
+                            for (int i = 0; i < RTC_KMAX; ++i) {
+                                if (te[i] == INT_MAX || cv > tv[i]) {
+                                    const float tf = tv[i];
+                                    const int ti = te[i];
+                                    tv[i] = cv;
+                                    te[i] = ce;
+                                    cv = tf;
+                                    ce = ti;
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            if (fuse_topk && valid) {
+                float wv[RTC_KMAX];
+                float z = 0.f;
+                if (mode == MOE_ROUTE_SIGMOID_TOPK_NORM) {
+#pragma unroll
+                    for (int j = 0; j < RTC_KMAX; ++j)
+                        if (j < k) {
+                            wv[j] = 1.f / (1.f + expf(-tv[j]));
+                            z += wv[j];
+                        }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < RTC_KMAX; ++j)
+                        if (j < k) {
+                            wv[j] = expf(tv[j] - tv[0]);
+                            z += wv[j];
+                        }
+                    if (mode == MOE_ROUTE_SOFTMAX_TOPK_RENORM) {
+                        // probabilities under the softmax over all E logits, renormalised over the selection
+                        float zall = 0.f;
+                        for (int e = 0; e < E; ++e) zall += expf(lrow[e] - tv[0]);
+                        float zp = 0.f;
+#pragma unroll
+                        for (int j = 0; j < RTC_KMAX; ++j)
+                            if (j < k) {
+                                wv[j] = wv[j] / zall;
+                                zp += wv[j];
+                            }
+                        z = zp;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < RTC_KMAX; ++j)
+                    if (j < k) {
+                        topk_idx[(size_t)row * k + j] = te[j];
+                        topk_w[(size_t)row * k + j] = wv[j] / z;
+                    }
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    if (warp == 1) {
+        if (lane == 0) mbar_wait_drain(tfull_bar, 0);
+        __syncwarp();
+        tmem_dealloc(tmem_base, S::TMEM_COLS);
+    }
+}
+
+// ---- small token counts: logits on CUDA cores, parallel over experts -----------------------------------
+// Block b handles experts [b*EPB, b*EPB + EPB) for every token; each warp takes tokens warp, warp+8, ...
+// and reduces its dot products across lanes with shuffles (fixed order: deterministic). x rows are
+// read in 16-byte vectors; W_r rows of the block's experts are staged in shared memory.
+constexpr int RS_THREADS = 256;
+
+__global__ void __launch_bounds__(RS_THREADS) router_logits_small_kernel(const __nv_bfloat16* __restrict__ x,
+                                                                         const float* __restrict__ w_router,
+                                                                         const float* __restrict__ bias, int T,
+                                                                         int d, int E, int epb,
+                                                                         float* __restrict__ logits) {
+    extern __shared__ float wsm[];  // [epb][d]
+    const int e0 = blockIdx.x * epb;
+    const int ne = min(epb, E - e0);
+    for (int i = threadIdx.x; i < ne * d / 4; i += RS_THREADS)
+        reinterpret_cast<float4*>(wsm)[i] = __ldg(reinterpret_cast<const float4*>(w_router + (size_t)e0 * d) + i);
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvec = d / 8;
+    for (int t = warp; t < T; t += RS_THREADS / 32) {
+        const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // epb <= 4
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 q = __ldg(xr + v);
+            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+            float xf[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = unpack_bf16x2(u[j]);
+                xf[2 * j] = f.x;
+                xf[2 * j + 1] = f.y;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (e < ne) {
+                    const float4* wr = reinterpret_cast<const float4*>(wsm + (size_t)e * d + v * 8);
+                    const float4 a = wr[0], b = wr[1];
+                    acc[e] = fmaf(xf[0], a.x, acc[e]);
+                    acc[e] = fmaf(xf[1], a.y, acc[e]);
+                    acc[e] = fmaf(xf[2], a.z, acc[e]);
+                    acc[e] = fmaf(xf[3], a.w, acc[e]);
+                    acc[e] = fmaf(xf[4], b.x, acc[e]);
+                    acc[e] = fmaf(xf[5], b.y, acc[e]);
+                    acc[e] = fmaf(xf[6], b.z, acc[e]);
+                    acc[e] = fmaf(xf[7], b.w, acc[e]);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            float s = acc[e];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (lane == 0 && e < ne) logits[(size_t)t * E + e0 + e] = s + (bias ? bias[e0 + e] : 0.f);
+        }
+    }
+}
+
+}  // namespace moe

@@ -66,27 +66,56 @@ class MoEFFN:
         self.buf, self._T = b, T
         return b
 
-    def forward(self, x, stream=None):
-        """y = MoE(x) for x [T, d] bf16 on the GPU. Returns the layer's output buffer [T, d] (bf16)."""
+    def forward(self, x, stream=None, timing=None):
+        """y = MoE(x) for x [T, d] bf16 on the GPU. Returns the layer's output buffer [T, d] (bf16).
+
+        timing: optional dict; if given, a (start, end) pair of CUDA events is recorded on the stream
+        around each stage ("route", "permute", "gateup", "down", "shared", "combine").
+        """
         T = x.shape[0]
         b = self.buffers(T)
-        N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"],
-                     stream)
+        s = stream if stream is not None else torch.cuda.current_stream(x.device)
+
+        def mark(name, first):
+            if timing is None:
+                return
+            if first:
+                timing[name] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            timing[name][0 if first else 1].record(s)
+
+        mark("route", True)
+        N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"], s)
+        mark("route", False)
+        mark("permute", True)
         N.permute(x, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], b["x_perm"],
-                  b["ws"], stream)
-        N.grouped_gemm_gateup(b["x_perm"], self.w_gateup, b["offsets"], b["h"], stream)
-        N.grouped_gemm_down(b["h"], self.w_down, b["offsets"], b["y_perm"], stream)
+                  b["ws"], s)
+        mark("permute", False)
+        mark("gateup", True)
+        N.grouped_gemm_gateup(b["x_perm"], self.w_gateup, b["offsets"], b["h"], s)
+        mark("gateup", False)
+        mark("down", True)
+        N.grouped_gemm_down(b["h"], self.w_down, b["offsets"], b["y_perm"], s)
+        mark("down", False)
         shared = None
         if self.shared_f:
-            N.grouped_gemm_gateup(x, self.w_gateup_shared.unsqueeze(0), b["shared_offsets"], b["h_shared"], stream)
+            mark("shared", True)
+            N.grouped_gemm_gateup(x, self.w_gateup_shared.unsqueeze(0), b["shared_offsets"], b["h_shared"], s)
             N.grouped_gemm_down(b["h_shared"], self.w_down_shared.unsqueeze(0), b["shared_offsets"], b["shared"],
-                                stream)
+                                s)
+            mark("shared", False)
             shared = b["shared"]
-        N.unpermute_combine(b["y_perm"], b["inv_perm"], b["topk_w"], shared, b["y"], stream)
+        mark("combine", True)
+        N.unpermute_combine(b["y_perm"], b["inv_perm"], b["topk_w"], shared, b["y"], s)
+        mark("combine", False)
         return b["y"]
 
     __call__ = forward
 
     def kernel_launches(self, T: int) -> int:
-        """Kernels one forward() launches: route (2), permute (4), gate|up, down, combine (+2 shared)."""
-        return 9 + (2 if self.shared_f else 0) if T > 0 else 0
+        """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the
+        tensor-core path with fused top-k is taken (E <= 256, T >= 2048, k <= 8), else logits + top-k;
+        permute 4; gate|up, down, combine 1 each; the shared expert 2 more."""
+        if T <= 0:
+            return 0
+        route = 1 if (self.E <= 256 and T >= 2048 and self.k <= 8) else 2
+        return route + 4 + 3 + (2 if self.shared_f else 0)

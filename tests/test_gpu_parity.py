@@ -110,6 +110,40 @@ def test_topk_ties_and_modes_small():
             np.testing.assert_allclose(w.cpu().numpy(), rw, rtol=2e-6, atol=1e-7)
 
 
+ROUTER_CASES = [
+    # T, d, E, k, mode, with bias: both sides of the tensor-core threshold (T >= 2048), fused (k <= 8) and
+    # unfused top-k, padded expert counts, every mode
+    (2047, 256, 8, 2, "softmax_topk_renorm", False),
+    (2048, 256, 8, 2, "softmax_topk_renorm", True),
+    (2100, 520, 100, 8, "topk_softmax", True),
+    (3000, 1024, 256, 8, "sigmoid_topk_norm", False),
+    (2176, 264, 40, 12, "topk_softmax", True),
+    (300, 7168, 256, 8, "sigmoid_topk_norm", True),
+    (64, 2880, 32, 4, "topk_softmax", False),
+    (1500, 2048, 384, 6, "topk_softmax", False),
+]
+
+
+@pytest.mark.parametrize("T,d,E,k,mode,with_bias", ROUTER_CASES)
+def test_router_paths_match_oracle(T, d, E, k, mode, with_bias):
+    x = synth.normal_bf16(7, 0, 0, T * d, 1.0).reshape(T, d)
+    wr = synth.normal_f32(7, 1, 0, E * d, 0.02).reshape(E, d)
+    bias = (synth.normal_f32(7, 4, 0, E, 1.0)) if with_bias else None
+    l64 = oracle.router_logits(x, wr, bias)
+    idx_ref, w_ref = oracle.topk(l64.astype(np.float32), k, mode)
+    margin = oracle.topk_margin(l64, k)
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    N.route_topk(to_dev_bf16(x), torch.from_numpy(wr).cuda(), torch.from_numpy(bias).cuda() if with_bias else None,
+                 k, mode, logits, idx, w)
+    assert N.get_device_error() == 0
+    assert np.abs(logits.cpu().numpy() - l64).max() <= 1e-5 * max(np.abs(l64).max(), 1.0)
+    keep = margin >= NEAR_TIE
+    assert (idx.cpu().numpy()[keep] == idx_ref[keep]).all()
+    np.testing.assert_allclose(w.cpu().numpy()[keep], w_ref[keep], rtol=2e-5, atol=2e-6)
+
+
 # ---- permutation -----------------------------------------------------------------------------------
 
 def _gpu_permute(x_bits, idx_np, E):
