@@ -66,7 +66,7 @@ struct GemmShape {
 template <int BN, int STAGES, bool GATEUP>
 __global__ void __launch_bounds__(GG_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const GemmArgs args) {
+                        const GemmArgs args, int weights_streamed_once) {
     using S = GemmShape<BN, STAGES, GATEUP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -160,8 +160,10 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
-        const uint64_t pol_a = l2_policy_evict_last();   // activations: re-read by every N-block
-        const uint64_t pol_b = l2_policy_evict_first();  // weights: streamed once per M-block wave
+        // activations are re-read by every N-block; weights are re-read by the M-blocks of their group unless
+        // each group fits one M-block, in which case they are streamed once and should not displace anything
+        const uint64_t pol_a = l2_policy_evict_last();
+        const uint64_t pol_b = weights_streamed_once ? l2_policy_evict_first() : l2_policy_evict_normal();
         int stage = 0;
         uint32_t phase = 0;
         long issued = 0;
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                 if (valid) {
 #pragma unroll
                     for (int v8 = 0; v8 < 4; ++v8)
-                        if (col0 + v8 * 8 < args.n_out)
+                        if (c0 + v8 * 8 < S::OUT_COLS && col0 + v8 * 8 < args.n_out)
                             *reinterpret_cast<uint4*>(dst_row + col0 + v8 * 8) =
                                 make_uint4(pk[4 * v8], pk[4 * v8 + 1], pk[4 * v8 + 2], pk[4 * v8 + 3]);
                 }

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -15,6 +16,7 @@
 #include "route_tc.cuh"
 #include "permute.cuh"
 #include "gemm.cuh"
+#include "gemm_pair.cuh"
 #include "combine.cuh"
 
 using namespace moe;
@@ -41,11 +43,28 @@ moe_status_t check_launch(const char* what) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Grouped-GEMM configurations compiled into the library.
-constexpr int kStages = 4;
-constexpr int kBN = 256;
-using GateUpShape = GemmShape<kBN, kStages, true>;
-using DownShape = GemmShape<kBN, kStages, false>;
+// Grouped-GEMM configurations compiled into the library:
+//   single CTA, BN 256 (4 stages) or 64 (8 stages): few rows per group (decode) or few tiles
+//   CTA pair, BN 256 (6 stages), and BN 240 for the down projection when d is a multiple of 240
+using Single256GU = GemmShape<256, 4, true>;
+using Single256DN = GemmShape<256, 4, false>;
+using Single64GU = GemmShape<64, 8, true>;
+using Single64DN = GemmShape<64, 8, false>;
+using Pair256GU = GemmPairShape<256, 6, true>;
+using Pair256DN = GemmPairShape<256, 6, false>;
+using Pair240DN = GemmPairShape<240, 6, false>;
+
+cudaError_t set_gemm_attributes() {
+    const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<256, 4, true>, a, Single256GU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_kernel<256, 4, false>, a, Single256DN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_kernel<64, 8, true>, a, Single64GU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_kernel<64, 8, false>, a, Single64DN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<256, 6, true>, a, Pair256GU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<256, 6, false>, a, Pair256DN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<240, 6, false>, a, Pair240DN::SMEM_BYTES);
+    return e;
+}
 
 constexpr int kRouterSmallMaxSmem = 200 * 1024;  // W_r rows staged by the small-T router kernel
 constexpr int kRouterTcMinT = 2048;               // token count from which the tensor-core router pays off
@@ -61,7 +80,6 @@ cudaError_t set_router_attributes() {
     if (e == cudaSuccess) e = set_router_tc_attr<32>();
     if (e == cudaSuccess) e = set_router_tc_attr<64>();
     if (e == cudaSuccess) e = set_router_tc_attr<128>();
-    if (e == cudaSuccess) e = set_router_tc_attr<256>();
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(router_logits_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  kRouterSmallMaxSmem);
@@ -93,11 +111,7 @@ moe_status_t device_info(DeviceInfo& out) {
         di.sm100 = (major == 10 && minor == 0);
         di.sms = sms;
         if (di.sm100) {
-            e = cudaFuncSetAttribute(grouped_gemm_kernel<kBN, kStages, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, GateUpShape::SMEM_BYTES);
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(grouped_gemm_kernel<kBN, kStages, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, DownShape::SMEM_BYTES);
+            e = set_gemm_attributes();
             if (e == cudaSuccess) e = set_router_attributes();
             if (e != cudaSuccess)
                 return fail(MOE_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -140,36 +154,85 @@ moe_status_t make_tmap(CUtensorMap* map, const void* base, int rank, const cuuin
     return MOE_OK;
 }
 
+struct GemmProblem {
+    const void* a;
+    const void* w;
+    const int32_t* offsets;
+    int G, M, K, n_out, f;
+    void* out;
+};
+
+// Tensor maps: A [M][K] in 128-row x 64 boxes; B slabs [G][rows][K] (rows = 2f for gate|up, n_out for
+// down) in b_rows x 64 boxes.
+moe_status_t make_gemm_maps(const GemmProblem& p, bool gateup, int b_rows, CUtensorMap* ta, CUtensorMap* tb) {
+    const cuuint64_t adims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
+    const cuuint64_t astr[1] = {(cuuint64_t)p.K * 2};
+    const cuuint32_t abox[2] = {GG_BK, GG_BM};
+    moe_status_t st = make_tmap(ta, p.a, 2, adims, astr, abox);
+    if (st != MOE_OK) return st;
+    const cuuint64_t rows = gateup ? (cuuint64_t)2 * p.f : (cuuint64_t)p.n_out;
+    const cuuint64_t bdims[3] = {(cuuint64_t)p.K, rows, (cuuint64_t)p.G};
+    const cuuint64_t bstr[2] = {(cuuint64_t)p.K * 2, rows * (cuuint64_t)p.K * 2};
+    const cuuint32_t bbox[3] = {GG_BK, (cuuint32_t)b_rows, 1};
+    return make_tmap(tb, p.w, 3, bdims, bstr, bbox);
+}
+
+GemmArgs gemm_args(const GemmProblem& p, int out_cols) {
+    GemmArgs args;
+    args.group_offsets = p.offsets;
+    args.G = p.G;
+    args.M = p.M;
+    args.K = p.K;
+    args.n_out = p.n_out;
+    args.f = p.f;
+    args.n_tiles = (p.n_out + out_cols - 1) / out_cols;
+    args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    return args;
+}
+
 template <int BN, int STAGES, bool GATEUP>
-moe_status_t launch_grouped_gemm(const void* a, const void* w, const int32_t* offsets, int G, int M, int K,
-                                 int n_out, int f, void* out, int sms, cudaStream_t stream) {
+moe_status_t launch_single(const GemmProblem& p, int sms, cudaStream_t stream) {
     using S = GemmShape<BN, STAGES, GATEUP>;
     CUtensorMap ta, tb;
-    const cuuint64_t adims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t astr[1] = {(cuuint64_t)K * 2};
-    const cuuint32_t abox[2] = {GG_BK, GG_BM};
-    moe_status_t st = make_tmap(&ta, a, 2, adims, astr, abox);
+    moe_status_t st = make_gemm_maps(p, GATEUP, GATEUP ? BN / 2 : BN, &ta, &tb);
     if (st != MOE_OK) return st;
-    // B slabs [G][rows][K]: rows = 2f for gate|up, n_out (= d) for down
-    const cuuint64_t rows = GATEUP ? (cuuint64_t)2 * f : (cuuint64_t)n_out;
-    const cuuint64_t bdims[3] = {(cuuint64_t)K, rows, (cuuint64_t)G};
-    const cuuint64_t bstr[2] = {(cuuint64_t)K * 2, rows * (cuuint64_t)K * 2};
-    const cuuint32_t bbox[3] = {GG_BK, (cuuint32_t)(GATEUP ? BN / 2 : BN), 1};
-    st = make_tmap(&tb, w, 3, bdims, bstr, bbox);
-    if (st != MOE_OK) return st;
-    GemmArgs args;
-    args.group_offsets = offsets;
-    args.G = G;
-    args.M = M;
-    args.K = K;
-    args.n_out = n_out;
-    args.f = f;
-    args.n_tiles = (n_out + S::OUT_COLS - 1) / S::OUT_COLS;
-    args.out = reinterpret_cast<__nv_bfloat16*>(out);
-    const long upper = ((long)M / GG_BM + G) * (long)args.n_tiles;  // >= the real tile count
+    const GemmArgs args = gemm_args(p, S::OUT_COLS);
+    const long upper = ((long)p.M / GG_BM + p.G) * (long)args.n_tiles;  // >= the real tile count
     const int grid = (int)(upper < sms ? upper : sms);
-    grouped_gemm_kernel<BN, STAGES, GATEUP><<<grid, GG_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args);
+    const int streamed_once = (long)p.M <= (long)p.G * GG_BM ? 1 : 0;
+    grouped_gemm_kernel<BN, STAGES, GATEUP><<<grid, GG_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args, streamed_once);
     return check_launch(GATEUP ? "grouped_gemm_gateup" : "grouped_gemm_down");
+}
+
+template <int BN, int STAGES, bool GATEUP>
+moe_status_t launch_pair(const GemmProblem& p, int sms, cudaStream_t stream) {
+    using S = GemmPairShape<BN, STAGES, GATEUP>;
+    CUtensorMap ta, tb;
+    moe_status_t st = make_gemm_maps(p, GATEUP, BN / 2, &ta, &tb);
+    if (st != MOE_OK) return st;
+    const GemmArgs args = gemm_args(p, S::OUT_COLS);
+    const long upper = ((long)p.M / GP_BM + p.G) * (long)args.n_tiles;
+    const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
+    const int streamed_once = (long)p.M <= (long)p.G * GP_BM ? 1 : 0;
+    grouped_gemm_pair_kernel<BN, STAGES, GATEUP><<<2 * clusters, GG_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args,
+                                                                                                      streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup (pair)" : "grouped_gemm_down (pair)");
+}
+
+// Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs. Otherwise a single CTA
+// per tile, 256 wide unless that leaves SMs idle (e.g. one small group), then 64 wide.
+moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cudaStream_t stream) {
+    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2) {
+        if (gateup) return launch_pair<256, 6, true>(p, sms, stream);
+        const long w256 = (long)(p.n_out + 255) / 256 * 256, w240 = (long)(p.n_out + 239) / 240 * 240;
+        if (w240 < w256) return launch_pair<240, 6, false>(p, sms, stream);
+        return launch_pair<256, 6, false>(p, sms, stream);
+    }
+    const long row_tiles = std::max<long>((p.M + GG_BM - 1) / GG_BM, std::min<long>(p.G, p.M));
+    const long wide_tiles = row_tiles * ((p.n_out + (gateup ? 127 : 255)) / (gateup ? 128 : 256));
+    if (wide_tiles >= sms)
+        return gateup ? launch_single<256, 4, true>(p, sms, stream) : launch_single<256, 4, false>(p, sms, stream);
+    return gateup ? launch_single<64, 8, true>(p, sms, stream) : launch_single<64, 8, false>(p, sms, stream);
 }
 
 moe_status_t check_gemm_args(const void* a, const void* w, const int32_t* offsets, int G, int M, int d, int f,
@@ -218,7 +281,7 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     if ((st = device_info(di)) != MOE_OK) return st;
     if (T == 0) return MOE_OK;
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-    if (E <= 256 && T >= kRouterTcMinT) {
+    if (E <= 128 && T >= kRouterTcMinT) {
         // tensor cores, W_r split into three bf16 pieces; top-k fused when k <= 8
         CUtensorMap tm;
         const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
@@ -236,11 +299,8 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
         else if (E <= 64)
             router_tc_kernel<64><<<grid, RTC_THREADS, RouterTcShape<64>::SMEM_BYTES, stream>>>(
                 tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
-        else if (E <= 128)
-            router_tc_kernel<128><<<grid, RTC_THREADS, RouterTcShape<128>::SMEM_BYTES, stream>>>(
-                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
         else
-            router_tc_kernel<256><<<grid, RTC_THREADS, RouterTcShape<256>::SMEM_BYTES, stream>>>(
+            router_tc_kernel<128><<<grid, RTC_THREADS, RouterTcShape<128>::SMEM_BYTES, stream>>>(
                 tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
         if ((st = check_launch("router_tc")) != MOE_OK) return st;
         if (fuse) return MOE_OK;
@@ -334,7 +394,8 @@ moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_ga
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
     if (M == 0) return MOE_OK;
-    return launch_grouped_gemm<kBN, kStages, true>(a, w_gateup, group_offsets, G, M, d, f, f, h, di.sms, stream);
+    const GemmProblem p{a, w_gateup, group_offsets, G, M, d, f, f, h};
+    return launch_grouped_gemm(p, true, di.sms, stream);
 }
 
 moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down, const int32_t* group_offsets,
@@ -344,7 +405,8 @@ moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
     if (M == 0) return MOE_OK;
-    return launch_grouped_gemm<kBN, kStages, false>(h, w_down, group_offsets, G, M, f, d, f, y, di.sms, stream);
+    const GemmProblem p{h, w_down, group_offsets, G, M, f, d, f, y};
+    return launch_grouped_gemm(p, false, di.sms, stream);
 }
 
 moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w,

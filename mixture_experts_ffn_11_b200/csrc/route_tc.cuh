@@ -2,35 +2,42 @@
 //
 // logits[t][e] = sum_i x[t][i] * W_r[e][i] + bias[e] with x bf16 and W_r fp32. The fp32 weights are split
 // on the fly into three bf16 pieces, W_r = hi + mid + lo (hi = bf16(w), mid = bf16(w - hi),
-// lo = bf16(w - hi - mid); both differences are exact in fp32), so the product is three bf16 MMAs into one
-// fp32 accumulator: x*hi + x*mid + x*lo, which carries ~24 bits of W_r (relative error ~2^-27 per
-// weight). bf16*bf16 products are exact in fp32, so the logits keep fp32 accuracy.
+// lo = bf16(w - hi - mid); both differences are exact in fp32), so the product is three bf16 MMAs:
+// x*hi + x*mid + x*lo, which carries ~24 bits of W_r (relative error ~2^-27 per weight). bf16*bf16
+// products are exact in fp32.
 //
-// One CTA per 128-token tile (192 threads):
-//   warp 0     TMA of the x tile [128 x 64] per K step into a STAGES-deep ring
-//   warp 1     TMEM allocation; one lane issues 3 x 4 tcgen05.mma (M=128, N=BNR, K=16) per K step
-//   warps 2-5  convert the W_r block [BNR x 64] to the three swizzled bf16 pieces in shared memory (the
-//              same 128-byte-swizzled K-major layout the TMA engine writes), then, as the epilogue, read
-//              their 32 accumulator lanes: + bias, store the logits row, select the top-k (k <= 8) by
-//              insertion in descending order (equal logits keep the lower expert id first) and write the
-//              routing weights.
+// The tensor core's fp32 accumulator drops low-order bits when it adds (a bias toward zero that grows
+// with the number of accumulation steps and the size of the running sum; on a 3 x 4096-long reduction it
+// reaches ~1e-5 of the logit). So each 64-wide K block is accumulated on its own, in one of two TMEM
+// buffers, and CUDA-core threads add the block partials into fp32 registers with IEEE round-to-nearest.
+//
+// One CTA per 128-token tile (320 threads):
+//   warp 0     TMA of the x tile [128 x 64] per K block into a STAGES-deep ring
+//   warp 1     TMEM allocation; one lane issues 3 x 4 tcgen05.mma (M=128, N=BNR, K=16) per K block into
+//              accumulator buffer (kb & 1), starting it afresh
+//   warps 2-5  convert the W_r block [BNR x 64] into the three bf16 pieces, stored in the 128-byte-swizzled
+//              K-major layout the TMA engine writes
+//   warps 6-9  drain: add each finished block partial of their 32 TMEM lanes into registers; at the end
+//              + bias, store the logits row, select the top-k (k <= 8) by insertion in descending order
+//              (equal logits keep the lower expert id first) and write the routing weights.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 192, RTC_KMAX = 8;
+constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 320, RTC_KMAX = 8;
 
 template <int BNR>
 struct RouterTcShape {
-    static_assert(BNR % 16 == 0 && BNR >= 16 && BNR <= 256, "UMMA N");
-    static constexpr int STAGES = BNR >= 256 ? 2 : (BNR >= 128 ? 3 : 4);
+    static_assert(BNR % 16 == 0 && BNR >= 16 && BNR <= 128, "UMMA N (and the drain's register budget)");
+    static constexpr int STAGES = BNR >= 128 ? 3 : 4;
     static constexpr int A_BYTES = RTC_BM * RTC_BK * 2;
     static constexpr int P_BYTES = BNR * RTC_BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
-    static constexpr int TMEM_COLS = BNR <= 32 ? 32 : (BNR <= 64 ? 64 : (BNR <= 128 ? 128 : 256));
+    static constexpr int TMEM_COLS = 2 * BNR <= 32 ? 32 : (2 * BNR <= 64 ? 64 : (2 * BNR <= 128 ? 128 : 256));
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert((2 * STAGES + 5) * 8 + 8 <= 256, "barrier area");
 };
 
 __device__ __forceinline__ void split3_bf16(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
@@ -55,8 +62,10 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
     uint64_t* empty_bar = full_bar + STAGES;
-    uint64_t* tfull_bar = empty_bar + STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tfull_bar + 1);
+    uint64_t* tfull_bar = empty_bar + STAGES;  // [2]
+    uint64_t* tempty_bar = tfull_bar + 2;      // [2]
+    uint64_t* final_bar = tempty_bar + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -68,7 +77,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             mbar_init(&full_bar[s], 1 + 128);  // TMA expect_tx arrival + 128 converter threads
             mbar_init(&empty_bar[s], 1);
         }
-        mbar_init(tfull_bar, 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull_bar[a], 1);
+            mbar_init(&tempty_bar[a], 4);  // lane 0 of each drain warp
+        }
+        mbar_init(final_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
@@ -83,6 +96,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
+        // ---------------- TMA: x tile ----------------
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
@@ -107,11 +121,16 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 mbar_wait_drain(&full_bar[n % STAGES], (uint32_t)((n / STAGES) & 1));
         __syncwarp();
     } else if (warp == 1) {
+        // ---------------- MMA: one fresh accumulation per K block ----------------
         constexpr uint32_t IDESC = idesc_bf16_f32(RTC_BM, BNR);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
+            const int acc = kb & 1;
+            if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], ((kb >> 1) & 1) ^ 1u, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
             if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
@@ -119,14 +138,16 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             if (lane == 0) {
                 const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
                 const uint64_t adesc = smem_desc_sw128(sa);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BNR);
 #pragma unroll
                 for (int p = 0; p < 3; ++p) {
                     const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + p * S::P_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < RTC_BK / 16; ++kk)
-                        umma_bf16_ss(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | p | kk) != 0 ? 1u : 0u);
+                        umma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (p | kk) != 0 ? 1u : 0u);
                 }
                 umma_commit(&empty_bar[stage]);
+                umma_commit(&tfull_bar[acc]);
             }
             __syncwarp();
             if (++stage == STAGES) {
@@ -134,22 +155,22 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 phase ^= 1u;
             }
         }
-        if (lane == 0) umma_commit(tfull_bar);  // also the last MMA's completion before TMEM is freed
+        if (lane == 0) umma_commit(final_bar);
         __syncwarp();
-    } else {
-        // ---- converters: W_r [E][d] fp32 -> hi/mid/lo bf16 pieces, swizzled K-major ----
+    } else if (warp < 6) {
+        // ---------------- converters: W_r [E][d] fp32 -> hi/mid/lo bf16 pieces ----------------
         const int ct = threadIdx.x - 64;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         constexpr int ITEMS = BNR * (RTC_BK / 8) / 128;  // 16-byte output chunks per thread per piece
-        for (int kb = 0; kb < KB && ok; ++kb) {
+        for (int kb = 0; kb < KB; ++kb) {
             if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             uint8_t* pbase = smem + stage * S::STAGE_BYTES + S::A_BYTES;
             const int k0 = kb * RTC_BK;
-#pragma unroll 4
+#pragma unroll
             for (int it = 0; it < ITEMS; ++it) {
                 const int item = ct + 128 * it;
                 const int r = item >> 3, c = item & 7;
@@ -163,11 +184,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 uint32_t hi[4], mi[4], lo[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint16_t h0, m0_, l0, h1, m1, l1;
-                    split3_bf16(w8[2 * j], h0, m0_, l0);
-                    split3_bf16(w8[2 * j + 1], h1, m1, l1);
+                    uint16_t h0, md0, l0, h1, md1, l1;
+                    split3_bf16(w8[2 * j], h0, md0, l0);
+                    split3_bf16(w8[2 * j + 1], h1, md1, l1);
                     hi[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                    mi[j] = (uint32_t)m0_ | ((uint32_t)m1 << 16);
+                    mi[j] = (uint32_t)md0 | ((uint32_t)md1 << 16);
                     lo[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
                 }
                 const int off = r * 128 + ((c ^ (r & 7)) << 4);
@@ -182,17 +203,44 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 phase ^= 1u;
             }
         }
-        // ---- epilogue ----
-        if (ok) {
-            if (lane == 0) ok = mbar_wait_bounded(tfull_bar, 0, abort_flag);
+    } else {
+        // ---------------- drain + epilogue (warps 6-9) ----------------
+        const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+        const int row = m0 + q * 32 + lane;
+        const bool valid = row < T;
+        const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+        float sum[BNR];
+#pragma unroll
+        for (int j = 0; j < BNR; ++j) sum[j] = 0.f;
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int acc = kb & 1;
+            if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], (kb >> 1) & 1, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after_sync();
+            if constexpr (BNR == 16) {  // a 32-column load would leave the 32-column allocation
+                uint32_t v[16];
+                tmem_load_16cols(t_row + (uint32_t)(acc * BNR), v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sum[j] += __uint_as_float(v[j]);
+            } else {
+#pragma unroll
+                for (int c0 = 0; c0 < BNR; c0 += 32) {
+                    if (c0 < E) {
+                        uint32_t v[32];
+                        tmem_load_32cols(t_row + (uint32_t)(acc * BNR + c0), v);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) sum[c0 + j] += __uint_as_float(v[j]);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
         }
         if (ok) {
-            tc_fence_after_sync();
-            const int q = warp & 3;
-            const int row = m0 + q * 32 + lane;
-            const bool valid = row < T;
-            const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+            float* lrow = logits + (size_t)(valid ? row : 0) * E;
             float tv[RTC_KMAX];
             int te[RTC_KMAX];
 #pragma unroll
@@ -200,30 +248,23 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 tv[i] = 0.f;
                 te[i] = INT_MAX;
             }
-            float* lrow = logits + (size_t)(valid ? row : 0) * E;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BNR; c0 += 32) {
-                if (c0 >= E) break;
-                uint32_t v[32];
-                tmem_load_32cols(t_row + c0, v);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int e = c0 + j;
-                    if (e < E) {
-                        float cv = __uint_as_float(v[j]) + (bias ? __ldg(bias + e) : 0.f);
-                        if (valid) lrow[e] = cv;
-                        if (fuse_topk) {
-                            int ce = e;
+            for (int e = 0; e < BNR; ++e) {
+                if (e < E) {
+                    sum[e] += bias ? __ldg(bias + e) : 0.f;
+                    if (valid) lrow[e] = sum[e];
+                    if (fuse_topk) {
+                        float cv = sum[e];
+                        int ce = e;
 #pragma unroll
-                            for (int i = 0; i < RTC_KMAX; ++i) {
-                                if (te[i] == INT_MAX || cv > tv[i]) {
-                                    const float tf = tv[i];
-                                    const int ti = te[i];
-                                    tv[i] = cv;
-                                    te[i] = ce;
-                                    cv = tf;
-                                    ce = ti;
-                                }
+                        for (int i = 0; i < RTC_KMAX; ++i) {
+                            if (te[i] == INT_MAX || cv > tv[i]) {
+                                const float tf = tv[i];
+                                const int ti = te[i];
+                                tv[i] = cv;
+                                te[i] = ce;
+                                cv = tf;
+                                ce = ti;
                             }
                         }
                     }
@@ -249,7 +290,9 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                     if (mode == MOE_ROUTE_SOFTMAX_TOPK_RENORM) {
                         // probabilities under the softmax over all E logits, renormalised over the selection
                         float zall = 0.f;
-                        for (int e = 0; e < E; ++e) zall += expf(lrow[e] - tv[0]);
+#pragma unroll
+                        for (int e = 0; e < BNR; ++e)
+                            if (e < E) zall += expf(sum[e] - tv[0]);
                         float zp = 0.f;
 #pragma unroll
                         for (int j = 0; j < RTC_KMAX; ++j)
@@ -274,7 +317,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     if (warp == 1) {
-        if (lane == 0) mbar_wait_drain(tfull_bar, 0);
+        if (lane == 0) mbar_wait_drain(final_bar, 0);
         __syncwarp();
         tmem_dealloc(tmem_base, S::TMEM_COLS);
     }

@@ -237,6 +237,13 @@ RAGGED = [
     ("one_expert_takes_all", [0, 0, 300, 0], 256, 512),
     ("many_small", [3] * 40 + [0] * 24, 64, 96),
     ("wide_k_tail", [130, 5], 1000, 264),
+    # CTA-pair kernel (groups average >= 128 rows): 256-row tiles, ragged and empty groups
+    ("pair_ragged", [0, 1, 255, 256, 257, 600, 0, 129], 256, 200),
+    ("pair_down_240_wide", [300, 0, 700, 45], 480, 136),
+    ("pair_one_expert", [0, 0, 2000, 0], 256, 256),
+    # single-CTA kernel, 256 wide (many groups of a few rows) and 64 wide (one small group)
+    ("single_wide", [2] * 160, 64, 256),
+    ("single_group_narrow", [50], 512, 256),
 ]
 
 
