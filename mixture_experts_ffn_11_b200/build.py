@@ -1,6 +1,9 @@
 """Build the CUDA library (libmoe.so) in-tree for sm_100a.
 
-    python -m mixture_experts_ffn_11_b200.build [--force] [--verbose]
+    python mixture_experts_ffn_11_b200/build.py [--force] [--verbose]
+
+Run it by path (or load it with load_build_module below): importing the package itself loads libmoe.so,
+which is what this script produces.
 
 The library is one translation unit (csrc/moe.cu plus the kernel headers it includes) compiled by nvcc
 into a shared object next to this file, so it travels with the source tree.
@@ -30,6 +33,16 @@ def nvcc_command(out: str = LIB, verbose: bool = False, extra=()):
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     return cmd
+
+
+def load_build_module():
+    """This module, loaded by file path without importing the package (usable before libmoe.so exists)."""
+    import importlib.util
+
+    spec = importlib.util.spec_from_file_location("_moe_build", os.path.abspath(__file__))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

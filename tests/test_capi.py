@@ -17,9 +17,6 @@ def _header_functions():
 
 @pytest.fixture(scope="module")
 def native():
-    from mixture_experts_ffn_11_b200 import build
-
-    build.build()
     from mixture_experts_ffn_11_b200 import _native
 
     return _native
