@@ -124,6 +124,34 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
                          moe_bf16_t* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Allocation-free variant of moe_permute. The blog post has no counterpart to
+ * this call; it exists for callers that cannot supply device scratch memory.
+ * Some callers cannot hand this library a workspace: they reach it through a
+ * fixed interface with no workspace argument and have no device allocator of
+ * their own, or they must not call cudaMalloc at run time (it can block the
+ * whole device, and it fails once a memory pool has reserved the device).
+ * This call does exactly what moe_permute does, with the same arguments minus
+ * the workspace; its scratch is a file-scope array of
+ * MOE_PERMUTE_STATIC_WS_BYTES bytes inside the library, which every GPU that
+ * loads the library holds until the process exits. It allocates nothing.
+ *  - Sizes whose moe_permute_workspace_size(T, E, k) exceeds
+ *    MOE_PERMUTE_STATIC_WS_BYTES are rejected with MOE_ERR_WORKSPACE before
+ *    anything is launched (the scratch is 4 bytes per expert per block of
+ *    4096 assignments: E = 128 allows up to 8,388,608 assignments T*k,
+ *    E = 1024 up to 1,048,576).
+ *  - The first call on a device looks up the array's device address (a
+ *    one-time set-up per device); make that first call before capturing a
+ *    stream.
+ *  - All calls on a device share the one array. Its contents persist between
+ *    calls, and each call rewrites every byte it reads before reading it, so
+ *    nothing has to be cleared. Calls that can overlap on the GPU (different
+ *    streams without ordering between them) race on the array and must be
+ *    serialised by the caller. */
+#define MOE_PERMUTE_STATIC_WS_BYTES (1u << 20)
+moe_status_t moe_permute_static_ws(const moe_bf16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                                   int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src,
+                                   int32_t* inv_perm, moe_bf16_t* x_perm, cudaStream_t stream);
+
 /* Grouped gate|up projection with fused SwiGLU, one expert per group:
  * for every group g and row r in [group_offsets[g], group_offsets[g+1]):
  *   h[r][n] = silu(sum_i a[r][i] * w[g][n][i]) * (sum_i a[r][i] * w[g][f+n][i]),  n < f,

@@ -23,6 +23,7 @@ ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm":
 
 # every entry point of include/moe.h
 EXPORTS = ("moe_route_topk", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
+           "moe_permute_static_ws",
            "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_unpermute_combine", "moe_get_device_error",
            "moe_last_error_string")
 
@@ -35,7 +36,7 @@ class MoEError(RuntimeError):
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
-        raise ImportError(f"{path} is not built; run `python -m mixture_experts_ffn_11_b200.build` "
+        raise ImportError(f"{path} is not built; run `python mixture_experts_ffn_11_b200/build.py` "
                           "(there is no non-CUDA fallback)")
     lib = ctypes.CDLL(path)
     vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -44,6 +45,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_topk_from_logits": [vp, ci, ci, ci, ci, vp, vp, vp],
         "moe_permute_workspace_size": [ci, ci, ci],
         "moe_permute": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, sz, vp],
+        "moe_permute_static_ws": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp],
         "moe_grouped_gemm_gateup": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_down": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_unpermute_combine": [vp, vp, vp, vp, ci, ci, ci, vp, vp],
@@ -132,6 +134,28 @@ def permute(x, topk_idx, E, counts, offsets, perm_src, inv_perm, x_perm, ws, str
     ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
     _check(_lib.moe_permute(_p(x), _p(topk_idx), T, d, E, k, _p(counts), _p(offsets), _p(perm_src),
                             _p(inv_perm), _p(x_perm), _p(ws), ws_bytes, _stream(stream)), "moe_permute")
+
+
+PERMUTE_STATIC_WS_BYTES = 1 << 20  # MOE_PERMUTE_STATIC_WS_BYTES in include/moe.h
+
+
+def permute_static_ws(x, topk_idx, E, counts, offsets, perm_src, inv_perm, x_perm, stream=None):
+    """moe_permute without a workspace argument: the library uses its own static scratch array (for
+    callers that cannot supply device scratch memory; see include/moe.h for the limits)."""
+    T, k = topk_idx.shape
+    R = T * k
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(counts, torch.int32, (E,), "counts")
+    _need(offsets, torch.int32, (E + 1,), "offsets")
+    _need(perm_src, torch.int32, (R,), "perm_src")
+    _need(inv_perm, torch.int32, (R,), "inv_perm")
+    d = 0
+    if x is not None:
+        d = x.shape[1]
+        _need(x, torch.bfloat16, (T, d), "x")
+        _need(x_perm, torch.bfloat16, (R, d), "x_perm")
+    _check(_lib.moe_permute_static_ws(_p(x), _p(topk_idx), T, d, E, k, _p(counts), _p(offsets), _p(perm_src),
+                                      _p(inv_perm), _p(x_perm), _stream(stream)), "moe_permute_static_ws")
 
 
 def grouped_gemm_gateup(a, w_gateup, group_offsets, h, stream=None):

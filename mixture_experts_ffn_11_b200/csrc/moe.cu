@@ -265,6 +265,32 @@ int grid_cap(long want, int sms, int per_sm) {
 
 }  // namespace
 
+// Scratch of moe_permute_static_ws: one array per device, part of the loaded module (nothing is
+// allocated). Host code must not pass this symbol to a kernel (on the host it is only a stand-in); the
+// device address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_permute_static_ws[MOE_PERMUTE_STATIC_WS_BYTES];
+
+namespace {
+void* g_static_ws_addr[kMaxDevices] = {};
+
+moe_status_t static_ws_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_static_ws_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_permute_static_ws);
+        if (e != cudaSuccess || !p)
+            return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress(static permute scratch): %s", cudaGetErrorString(e));
+        g_static_ws_addr[dev] = p;
+    }
+    *out = g_static_ws_addr[dev];
+    return MOE_OK;
+}
+}  // namespace
+
 extern "C" {
 
 moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const float* bias, int T, int d, int E,
@@ -385,6 +411,23 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
         if ((st = check_launch("gather_rows")) != MOE_OK) return st;
     }
     return MOE_OK;
+}
+
+moe_status_t moe_permute_static_ws(const moe_bf16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
+                                   int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src,
+                                   int32_t* inv_perm, moe_bf16_t* x_perm, cudaStream_t stream) {
+    moe_status_t st = check_route_sizes(T, E, k);
+    if (st != MOE_OK) return st;
+    const size_t need = moe_permute_workspace_size(T, E, k);
+    if (need > MOE_PERMUTE_STATIC_WS_BYTES)
+        return fail(MOE_ERR_WORKSPACE,
+                    "T=%d, E=%d, k=%d need %zu bytes of scratch; the library's static array holds %u (use moe_permute "
+                    "with a workspace for larger sizes)",
+                    T, E, k, need, (unsigned)MOE_PERMUTE_STATIC_WS_BYTES);
+    void* ws = nullptr;
+    if ((st = static_ws_address(&ws)) != MOE_OK) return st;
+    return moe_permute(x, topk_idx, T, d, E, k, expert_counts, expert_offsets, perm_src, inv_perm, x_perm, ws,
+                       MOE_PERMUTE_STATIC_WS_BYTES, stream);
 }
 
 moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_gateup, const int32_t* group_offsets,
