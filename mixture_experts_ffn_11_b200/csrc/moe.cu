@@ -141,15 +141,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor map with 128-byte swizzle; dims/strides innermost first, strides in bytes for dims >= 1.
+// Tiled tensor map; dims/strides innermost first, strides in bytes for dims >= 1. bf16 maps use the
+// 128-byte swizzle the UMMA descriptors expect; the fp32 router-weight map is unswizzled.
 moe_status_t make_tmap(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-                       const cuuint64_t* strides, const cuuint32_t* box) {
+                       const cuuint64_t* strides, const cuuint32_t* box,
+                       CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
     const cuuint32_t elem_strides[3] = {1, 1, 1};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), dims,
-                           strides, box, elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = enc(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, elem_strides,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return MOE_OK;
 }
@@ -309,25 +312,32 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     if (E <= 128 && T >= kRouterTcMinT) {
         // tensor cores, W_r split into three bf16 pieces; top-k fused when k <= 8
-        CUtensorMap tm;
+        CUtensorMap tm, tw;
         const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
         const cuuint32_t box[2] = {RTC_BK, RTC_BM};
         if ((st = make_tmap(&tm, x, 2, dims, strides, box)) != MOE_OK) return st;
+        const int bnr = E <= 16 ? 16 : (E <= 32 ? 32 : (E <= 64 ? 64 : 128));
+        const cuuint64_t wdims[2] = {(cuuint64_t)d, (cuuint64_t)E};
+        const cuuint64_t wstrides[1] = {(cuuint64_t)d * 4};
+        const cuuint32_t wbox[2] = {RTC_BK, (cuuint32_t)bnr};
+        if ((st = make_tmap(&tw, w_router, 2, wdims, wstrides, wbox, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) != MOE_OK)
+            return st;
         const int fuse = k <= RTC_KMAX ? 1 : 0;
         const int grid = (T + RTC_BM - 1) / RTC_BM;
         if (E <= 16)
             router_tc_kernel<16><<<grid, RTC_THREADS, RouterTcShape<16>::SMEM_BYTES, stream>>>(
-                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
         else if (E <= 32)
             router_tc_kernel<32><<<grid, RTC_THREADS, RouterTcShape<32>::SMEM_BYTES, stream>>>(
-                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
         else if (E <= 64)
             router_tc_kernel<64><<<grid, RTC_THREADS, RouterTcShape<64>::SMEM_BYTES, stream>>>(
-                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
         else
             router_tc_kernel<128><<<grid, RTC_THREADS, RouterTcShape<128>::SMEM_BYTES, stream>>>(
-                tm, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
         if ((st = check_launch("router_tc")) != MOE_OK) return st;
         if (fuse) return MOE_OK;
     } else if ((size_t)d * sizeof(float) <= (size_t)kRouterSmallMaxSmem) {
@@ -465,7 +475,8 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
     moe_status_t st = device_info(di);
     if (st != MOE_OK) return st;
     if (T == 0) return MOE_OK;
-    const int grid = grid_cap((T + 7) / 8, di.sms, 16);
+    const long items = (long)T * ((d / 8 + CB_CHUNK_VEC - 1) / CB_CHUNK_VEC);
+    const int grid = grid_cap((items + 7) / 8, di.sms, 16);
     combine_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(y_perm), inv_perm, topk_w,
                                              reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
                                              reinterpret_cast<__nv_bfloat16*>(y));

@@ -109,16 +109,35 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
     if (t >= T) return;
     const float* l = logits + (size_t)t * E;
     const int per = (E + 31) / 32;
+    // E <= 256: the token's logits stay in registers (8 per lane) across the k rounds
+    constexpr int RPER = 8;
+    float rv[RPER];
+    if (per <= RPER) {
+#pragma unroll
+        for (int s = 0; s < RPER; ++s) {
+            const int e = s * 32 + lane;
+            rv[s] = (s < per && e < E) ? l[e] : 0.f;
+        }
+    }
     uint32_t taken = 0;
     float my_v = 0.f;
     int my_e = -1;
     for (int j = 0; j < k; ++j) {
         Cand c{0.f, INT_MAX};
-        for (int s = 0; s < per; ++s) {
-            const int e = s * 32 + lane;
-            if (e >= E || (taken >> s) & 1u) continue;
-            const float v = l[e];
-            if (c.e == INT_MAX || v > c.v) c = Cand{v, e};  // ascending e: strict '>' keeps the lower id
+        if (per <= RPER) {
+#pragma unroll
+            for (int s = 0; s < RPER; ++s) {
+                const int e = s * 32 + lane;
+                if (s >= per || e >= E || (taken >> s) & 1u) continue;
+                if (c.e == INT_MAX || rv[s] > c.v) c = Cand{rv[s], e};  // ascending e: strict '>' keeps the lower id
+            }
+        } else {
+            for (int s = 0; s < per; ++s) {
+                const int e = s * 32 + lane;
+                if (e >= E || (taken >> s) & 1u) continue;
+                const float v = l[e];
+                if (c.e == INT_MAX || v > c.v) c = Cand{v, e};
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {

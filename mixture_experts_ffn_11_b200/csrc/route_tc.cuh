@@ -8,15 +8,17 @@
 //
 // The tensor core's fp32 accumulator drops low-order bits when it adds (a bias toward zero that grows
 // with the number of accumulation steps and the size of the running sum; on a 3 x 4096-long reduction it
-// reaches ~1e-5 of the logit). So each 64-wide K block is accumulated on its own, in one of two TMEM
-// buffers, and CUDA-core threads add the block partials into fp32 registers with IEEE round-to-nearest.
+// reaches ~1e-5 of the logit). So each 64-wide K block is accumulated on its own, in one of NBUF TMEM
+// buffers (as many as fit, up to 8, so the round trip MMA -> drain -> reuse is not on the critical
+// path), and CUDA-core threads add the block partials into fp32 registers with IEEE round-to-nearest.
 //
 // One CTA per 128-token tile (320 threads):
-//   warp 0     TMA of the x tile [128 x 64] per K block into a STAGES-deep ring
+//   warp 0     TMA of the x tile [128 x 64] bf16 and of the W_r block [BNR x 64] fp32 per K block into a
+//              STAGES-deep ring (the W_r block lands unswizzled, 256 bytes per expert row)
 //   warp 1     TMEM allocation; one lane issues 3 x 4 tcgen05.mma (M=128, N=BNR, K=16) per K block into
-//              accumulator buffer (kb & 1), starting it afresh
-//   warps 2-5  convert the W_r block [BNR x 64] into the three bf16 pieces, stored in the 128-byte-swizzled
-//              K-major layout the TMA engine writes
+//              accumulator buffer (kb % NBUF), starting it afresh
+//   warps 2-5  convert the staged W_r block into the three bf16 pieces, stored in the 128-byte-swizzled
+//              K-major layout the TMA engine writes, then signal conv[stage]
 //   warps 6-9  drain: add each finished block partial of their 32 TMEM lanes into registers; at the end
 //              + bias, store the logits row, select the top-k (k <= 8) by insertion in descending order
 //              (equal logits keep the lower expert id first) and write the routing weights.
@@ -30,14 +32,19 @@ constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 320, RTC_KMAX = 8;
 template <int BNR>
 struct RouterTcShape {
     static_assert(BNR % 16 == 0 && BNR >= 16 && BNR <= 128, "UMMA N (and the drain's register budget)");
-    static constexpr int STAGES = BNR >= 128 ? 3 : 4;
-    static constexpr int A_BYTES = RTC_BM * RTC_BK * 2;
-    static constexpr int P_BYTES = BNR * RTC_BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
-    static constexpr int TMEM_COLS = 2 * BNR <= 32 ? 32 : (2 * BNR <= 64 ? 64 : (2 * BNR <= 128 ? 128 : 256));
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+    static constexpr int A_BYTES = RTC_BM * RTC_BK * 2;  // x tile, bf16
+    static constexpr int W_BYTES = BNR * RTC_BK * 4;     // W_r block, fp32 as loaded
+    static constexpr int P_BYTES = BNR * RTC_BK * 2;     // one bf16 piece
+    static constexpr int STAGE_BYTES = A_BYTES + W_BYTES + 3 * P_BYTES;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
+    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
+    static_assert(STAGES >= 2, "ring depth");
+    static constexpr int NBUF = 512 / BNR >= 8 ? 8 : 512 / BNR;  // partial-sum buffers in TMEM
+    static constexpr int TMEM_COLS = NBUF * BNR <= 32 ? 32 : (NBUF * BNR <= 64 ? 64 : (NBUF * BNR <= 128 ? 128 : (NBUF * BNR <= 256 ? 256 : 512)));
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
-    static_assert((2 * STAGES + 5) * 8 + 8 <= 256, "barrier area");
+    static_assert((3 * STAGES + 2 * NBUF + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
 };
 
 __device__ __forceinline__ void split3_bf16(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
@@ -53,18 +60,20 @@ __device__ __forceinline__ void split3_bf16(float w, uint16_t& hi, uint16_t& mid
 
 template <int BNR>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
-    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const float* __restrict__ w_router,
+    router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const float* __restrict__ bias, int T, int d, int E, int k, int mode, int fuse_topk,
                      float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     using S = RouterTcShape<BNR>;
     constexpr int STAGES = S::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);
-    uint64_t* empty_bar = full_bar + STAGES;
-    uint64_t* tfull_bar = empty_bar + STAGES;  // [2]
-    uint64_t* tempty_bar = tfull_bar + 2;      // [2]
-    uint64_t* final_bar = tempty_bar + 2;
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);  // TMA landed
+    uint64_t* conv_bar = full_bar + STAGES;                                            // pieces written
+    uint64_t* empty_bar = conv_bar + STAGES;                                           // MMA done
+    constexpr int NBUF = S::NBUF;
+    uint64_t* tfull_bar = empty_bar + STAGES;  // [NBUF]
+    uint64_t* tempty_bar = tfull_bar + NBUF;   // [NBUF]
+    uint64_t* final_bar = tempty_bar + NBUF;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -74,10 +83,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1 + 128);  // TMA expect_tx arrival + 128 converter threads
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&conv_bar[s], 128);  // every converter thread
             mbar_init(&empty_bar[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < NBUF; ++a) {
             mbar_init(&tfull_bar[a], 1);
             mbar_init(&tempty_bar[a], 4);  // lane 0 of each drain warp
         }
@@ -85,6 +95,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
+        tma_prefetch_desc(&tmW);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -101,14 +112,17 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         uint32_t phase = 0;
         int issued = 0;
         bool ok = true;
-        const uint64_t pol = l2_policy_evict_first();
+        const uint64_t pol = l2_policy_evict_first();      // x: read once per tile
+        const uint64_t pol_w = l2_policy_evict_last();     // W_r: read by every tile
         for (int kb = 0; kb < KB; ++kb) {
             if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             if (lane == 0) {
-                mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES);
-                tma_load_2d(smem + stage * S::STAGE_BYTES, &tmX, &full_bar[stage], kb * RTC_BK, m0, pol);
+                uint8_t* sa = smem + stage * S::STAGE_BYTES;
+                mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES + S::W_BYTES);
+                tma_load_2d(sa, &tmX, &full_bar[stage], kb * RTC_BK, m0, pol);
+                tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], kb * RTC_BK, 0, pol_w);
             }
             ++issued;
             if (++stage == STAGES) {
@@ -127,11 +141,12 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         uint32_t phase = 0;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
-            const int acc = kb & 1;
-            if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], ((kb >> 1) & 1) ^ 1u, abort_flag);
+            const int acc = kb % NBUF;
+            if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], ((kb / NBUF) & 1) ^ 1u, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
+            if (lane == 0) ok = mbar_wait_bounded(&conv_bar[stage], phase, abort_flag) &&
+                                mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
@@ -141,7 +156,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BNR);
 #pragma unroll
                 for (int p = 0; p < 3; ++p) {
-                    const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + p * S::P_BYTES);
+                    const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + S::W_BYTES + p * S::P_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < RTC_BK / 16; ++kk)
                         umma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (p | kk) != 0 ? 1u : 0u);
@@ -158,28 +173,24 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (lane == 0) umma_commit(final_bar);
         __syncwarp();
     } else if (warp < 6) {
-        // ---------------- converters: W_r [E][d] fp32 -> hi/mid/lo bf16 pieces ----------------
+        // ---------------- converters: staged W_r block (fp32) -> hi/mid/lo bf16 pieces ----------------
         const int ct = threadIdx.x - 64;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         constexpr int ITEMS = BNR * (RTC_BK / 8) / 128;  // 16-byte output chunks per thread per piece
         for (int kb = 0; kb < KB; ++kb) {
-            if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
+            if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            uint8_t* pbase = smem + stage * S::STAGE_BYTES + S::A_BYTES;
-            const int k0 = kb * RTC_BK;
+            const uint8_t* wbase = smem + stage * S::STAGE_BYTES + S::A_BYTES;
+            uint8_t* pbase = smem + stage * S::STAGE_BYTES + S::A_BYTES + S::W_BYTES;
 #pragma unroll
             for (int it = 0; it < ITEMS; ++it) {
                 const int item = ct + 128 * it;
-                const int r = item >> 3, c = item & 7;
-                float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-                if (r < E && k0 + c * 8 < d) {
-                    const float4* src = reinterpret_cast<const float4*>(w_router + (size_t)r * d + k0 + c * 8);
-                    v0 = __ldg(src);
-                    v1 = __ldg(src + 1);
-                }
+                const int r = item >> 3, c = item & 7;  // expert row, 8-element chunk of the 64-wide block
+                const float4* src = reinterpret_cast<const float4*>(wbase + r * (RTC_BK * 4) + c * 32);
+                const float4 v0 = src[0], v1 = src[1];  // rows past E and columns past d arrive as zeros
                 const float w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                 uint32_t hi[4], mi[4], lo[4];
 #pragma unroll
@@ -197,7 +208,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 *reinterpret_cast<uint4*>(pbase + 2 * S::P_BYTES + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes -> tensor core
-            mbar_arrive(&full_bar[stage]);
+            mbar_arrive(&conv_bar[stage]);
             if (++stage == STAGES) {
                 stage = 0;
                 phase ^= 1u;
@@ -214,8 +225,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         for (int j = 0; j < BNR; ++j) sum[j] = 0.f;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
-            const int acc = kb & 1;
-            if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], (kb >> 1) & 1, abort_flag);
+            const int acc = kb % NBUF;
+            if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], (kb / NBUF) & 1, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
@@ -324,10 +335,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
 }
 
 // ---- small token counts: logits on CUDA cores, parallel over experts -----------------------------------
-// Block b handles experts [b*EPB, b*EPB + EPB) for every token; each warp takes tokens warp, warp+8, ...
-// and reduces its dot products across lanes with shuffles (fixed order: deterministic). x rows are
-// read in 16-byte vectors; W_r rows of the block's experts are staged in shared memory.
-constexpr int RS_THREADS = 256;
+// Block b handles experts [b*EPB, b*EPB + EPB) (EPB <= 4) for every token. W_r rows of the block's experts are
+// staged in shared memory; each warp then takes RS_TPW tokens at a time and walks d in 16-byte vectors of x,
+// so RS_TPW independent loads per lane are in flight; dot products are reduced across lanes with shuffles
+// in a fixed order (deterministic).
+constexpr int RS_THREADS = 256, RS_TPW = 8;
 
 __global__ void __launch_bounds__(RS_THREADS) router_logits_small_kernel(const __nv_bfloat16* __restrict__ x,
                                                                          const float* __restrict__ w_router,
@@ -337,47 +349,62 @@ __global__ void __launch_bounds__(RS_THREADS) router_logits_small_kernel(const _
     extern __shared__ float wsm[];  // [epb][d]
     const int e0 = blockIdx.x * epb;
     const int ne = min(epb, E - e0);
-    for (int i = threadIdx.x; i < ne * d / 4; i += RS_THREADS)
-        reinterpret_cast<float4*>(wsm)[i] = __ldg(reinterpret_cast<const float4*>(w_router + (size_t)e0 * d) + i);
+    {
+        const float4* src = reinterpret_cast<const float4*>(w_router + (size_t)e0 * d);
+        float4* dst = reinterpret_cast<float4*>(wsm);
+        const int n4 = ne * d / 4;
+#pragma unroll 4
+        for (int i = threadIdx.x; i < n4; i += RS_THREADS) dst[i] = __ldg(src + i);
+    }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nvec = d / 8;
-    for (int t = warp; t < T; t += RS_THREADS / 32) {
-        const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};  // epb <= 4
-        for (int v = lane; v < nvec; v += 32) {
-            const uint4 q = __ldg(xr + v);
-            const uint32_t u[4] = {q.x, q.y, q.z, q.w};
-            float xf[8];
+    for (int t0 = warp * RS_TPW; t0 < T; t0 += (RS_THREADS / 32) * RS_TPW) {
+        float acc[RS_TPW][4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = unpack_bf16x2(u[j]);
-                xf[2 * j] = f.x;
-                xf[2 * j + 1] = f.y;
-            }
+        for (int i = 0; i < RS_TPW; ++i)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+#pragma unroll 2
+        for (int v = lane; v < nvec; v += 32) {
+            uint4 q[RS_TPW];
+#pragma unroll
+            for (int i = 0; i < RS_TPW; ++i)
+                q[i] = t0 + i < T ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + i) * d) + v)
+                                  : make_uint4(0, 0, 0, 0);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 if (e < ne) {
                     const float4* wr = reinterpret_cast<const float4*>(wsm + (size_t)e * d + v * 8);
                     const float4 a = wr[0], b = wr[1];
-                    acc[e] = fmaf(xf[0], a.x, acc[e]);
-                    acc[e] = fmaf(xf[1], a.y, acc[e]);
-                    acc[e] = fmaf(xf[2], a.z, acc[e]);
-                    acc[e] = fmaf(xf[3], a.w, acc[e]);
-                    acc[e] = fmaf(xf[4], b.x, acc[e]);
-                    acc[e] = fmaf(xf[5], b.y, acc[e]);
-                    acc[e] = fmaf(xf[6], b.z, acc[e]);
-                    acc[e] = fmaf(xf[7], b.w, acc[e]);
+#pragma unroll
+                    for (int i = 0; i < RS_TPW; ++i) {
+                        const float2 x01 = unpack_bf16x2(q[i].x), x23 = unpack_bf16x2(q[i].y);
+                        const float2 x45 = unpack_bf16x2(q[i].z), x67 = unpack_bf16x2(q[i].w);
+                        float s = acc[i][e];
+                        s = fmaf(x01.x, a.x, s);
+                        s = fmaf(x01.y, a.y, s);
+                        s = fmaf(x23.x, a.z, s);
+                        s = fmaf(x23.y, a.w, s);
+                        s = fmaf(x45.x, b.x, s);
+                        s = fmaf(x45.y, b.y, s);
+                        s = fmaf(x67.x, b.z, s);
+                        s = fmaf(x67.y, b.w, s);
+                        acc[i][e] = s;
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            float s = acc[e];
+        for (int i = 0; i < RS_TPW; ++i)
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0 && e < ne) logits[(size_t)t * E + e0 + e] = s + (bias ? bias[e0 + e] : 0.f);
-        }
+            for (int e = 0; e < 4; ++e) {
+                float s = acc[i][e];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (lane == 0 && e < ne && t0 + i < T)
+                    logits[(size_t)(t0 + i) * E + e0 + e] = s + (bias ? bias[e0 + e] : 0.f);
+            }
     }
 }
 
