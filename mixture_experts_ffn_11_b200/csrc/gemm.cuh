@@ -48,6 +48,32 @@ struct GemmArgs {
     __nv_bfloat16* out;  // [M][n_out]
 };
 
+// Epilogue store of one warp's 32 rows x 32 bf16 columns (thread = row, 16 packed words per thread).
+// A thread's own row is 64 contiguous bytes, but a warp-wide store of one 16-byte piece per row touches
+// 32 rows and only half of each 32-byte sector; L2 then has to fetch the rest of every sector from DRAM.
+// So the rows go through a 2 KB per-warp staging buffer (16-byte units XOR-swizzled by row, which keeps
+// both the write and the read at the minimum of four shared-memory wavefronts) and leave it as
+// 8 rows x 64 contiguous bytes per instruction: whole sectors, masked per row and column.
+__device__ __forceinline__ void store_warp_rows_32cols(uint8_t* stage, const uint32_t (&pk)[16], int lane,
+                                                       __nv_bfloat16* out, int ld_out, int row_base, int row_end,
+                                                       int col0, int n_out, int cols_in_tile) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+        *reinterpret_cast<uint4*>(stage + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    __syncwarp();
+    const int u = lane & 3;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int row = i * 8 + (lane >> 2);
+        const uint4 val = *reinterpret_cast<const uint4*>(stage + row * 64 + ((u ^ ((row >> 1) & 3)) << 4));
+        const int grow = row_base + row, col = col0 + u * 8;
+        if (grow < row_end && u * 8 < cols_in_tile && col < n_out)
+            *reinterpret_cast<uint4*>(out + (size_t)grow * ld_out + col) = val;
+    }
+    __syncwarp();
+}
+
 template <int BN, int STAGES, bool GATEUP>
 struct GemmShape {
     static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128 is a multiple of 16 up to 256");
@@ -58,9 +84,12 @@ struct GemmShape {
     static constexpr int OUT_COLS = GATEUP ? BN / 2 : BN;
     static constexpr int TMEM_COLS = 2 * BN <= 64 ? 64 : (2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512));
     static constexpr int BAR_BYTES = 256;
-    static constexpr int TABLE_BYTES = 2 * (GG_MAX_GROUPS + 1) * 4;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES;
+    static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;  // keeps what follows 128-B aligned
+    static constexpr int EPI_BYTES = 4 * 2048;  // per-epilogue-warp store staging
+    static_assert((STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES) % 128 == 0, "staging buffer alignment");
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES + EPI_BYTES;
     static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 template <int BN, int STAGES, bool GATEUP>
@@ -80,6 +109,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES);
     int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
+    uint8_t* epi_stage = smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES + S::TABLE_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = args.G;
@@ -252,15 +282,14 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
             int g, nb, mb;
             locate(tile, g, nb, mb);
             const int row_end = s_off[g + 1];
-            const int r = s_off[g] + mb * GG_BM + q * 32 + lane;
-            const bool valid = r < row_end;
+            const int row_base = s_off[g] + mb * GG_BM + q * 32;  // global row of this warp's lane 0
             if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const int col_base = nb * S::OUT_COLS;
-            __nv_bfloat16* dst_row = args.out + (size_t)(valid ? r : 0) * args.n_out;
+            uint8_t* my_stage = epi_stage + (warp - 2) * 2048;
 #pragma unroll 1
             for (int c0 = 0; c0 < S::OUT_COLS; c0 += 32) {
                 const int col0 = col_base + c0;
@@ -283,13 +312,8 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                     for (int i = 0; i < 16; ++i)
                         pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                 }
-                if (valid) {
-#pragma unroll
-                    for (int v8 = 0; v8 < 4; ++v8)
-                        if (c0 + v8 * 8 < S::OUT_COLS && col0 + v8 * 8 < args.n_out)
-                            *reinterpret_cast<uint4*>(dst_row + col0 + v8 * 8) =
-                                make_uint4(pk[4 * v8], pk[4 * v8 + 1], pk[4 * v8 + 2], pk[4 * v8 + 3]);
-                }
+                store_warp_rows_32cols(my_stage, pk, lane, args.out, args.n_out, row_base, row_end, col0, args.n_out,
+                                       S::OUT_COLS - c0);
             }
             tc_fence_before_sync();
             __syncwarp();

@@ -25,7 +25,9 @@ namespace moe {
 
 constexpr int GP_BM = 256;  // rows per pair tile (128 per CTA)
 
-template <int BN, int STAGES, bool GATEUP>
+// SUB: 64-wide K blocks per ring stage. Two halve the barrier round trips per FLOP (8 MMAs per stage); measured
+// faster on long reductions (gate|up with K >= 4096).
+template <int BN, int STAGES, bool GATEUP, int SUB = 1>
 struct GemmPairShape {
     static_assert(BN % 32 == 0 || (!GATEUP && BN % 16 == 0), "tile width");
     static_assert(BN >= 64 && BN <= 256, "UMMA N for M=256 (cta_group::2) is a multiple of 16 up to 256");
@@ -33,22 +35,25 @@ struct GemmPairShape {
     static_assert((BN / 2) % 8 == 0, "each CTA's B half must be whole 8-row swizzle atoms");
     static constexpr int A_BYTES = 128 * GG_BK * 2;
     static constexpr int B_BYTES = (BN / 2) * GG_BK * 2;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static_assert(STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
+    static constexpr int SUB_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGE_BYTES = SUB * SUB_BYTES;
+    static_assert(SUB_BYTES % 1024 == 0, "sub-block bases stay 1024-byte aligned");
     static constexpr int OUT_COLS = GATEUP ? BN / 2 : BN;
     static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
     static constexpr int BAR_BYTES = 256;
-    static constexpr int TABLE_BYTES = 2 * (GG_MAX_GROUPS + 1) * 4;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES;
+    static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;  // keeps what follows 128-B aligned
+    static constexpr int EPI_BYTES = 4 * 2048;  // per-epilogue-warp store staging
+    static_assert((STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES) % 128 == 0, "staging buffer alignment");
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES + EPI_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
 };
 
-template <int BN, int STAGES, bool GATEUP>
+template <int BN, int STAGES, bool GATEUP, int SUB = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const GemmArgs args, int weights_streamed_once) {
-    using S = GemmPairShape<BN, STAGES, GATEUP>;
+    using S = GemmPairShape<BN, STAGES, GATEUP, SUB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* stages = smem;
@@ -61,13 +66,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES);
     int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
+    uint8_t* epi_stage = smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES + S::TABLE_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
     const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
     const int G = args.G;
-    const int KB = (args.K + GG_BK - 1) / GG_BK;
+    const int KB = (args.K + GG_BK * SUB - 1) / (GG_BK * SUB);  // ring stages per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -167,8 +173,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
                     uint8_t* sa = stages + stage * S::STAGE_BYTES;
                     const uint32_t bar = mapa_shared(smem_u32(&full_bar[stage]), 0);
                     if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * S::STAGE_BYTES);
-                    tma_load_2d_pair(sa, &tmA, bar, kb * GG_BK, row0, pol_a);
-                    tma_load_3d_pair(sa + S::A_BYTES, &tmB, bar, kb * GG_BK, brow, g, pol_b);
+#pragma unroll
+                    for (int sb = 0; sb < SUB; ++sb) {  // K past the end arrives as zeros
+                        const int kc = (kb * SUB + sb) * GG_BK;
+                        tma_load_2d_pair(sa + sb * S::SUB_BYTES, &tmA, bar, kc, row0, pol_a);
+                        tma_load_3d_pair(sa + sb * S::SUB_BYTES + S::A_BYTES, &tmB, bar, kc, brow, g, pol_b);
+                    }
                 }
                 ++issued;
                 if (++stage == STAGES) {
@@ -202,12 +212,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
                     if (!ok) break;
                     tc_fence_after_sync();
                     if (lane == 0) {
-                        const uint32_t sa = smem_u32(stages + stage * S::STAGE_BYTES);
-                        const uint64_t adesc = smem_desc_sw128(sa);
-                        const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES);
 #pragma unroll
-                        for (int k = 0; k < GG_BK / 16; ++k)
-                            umma_bf16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC, (kb | k) != 0 ? 1u : 0u);
+                        for (int sb = 0; sb < SUB; ++sb) {
+                            const uint32_t sa = smem_u32(stages + stage * S::STAGE_BYTES + sb * S::SUB_BYTES);
+                            const uint64_t adesc = smem_desc_sw128(sa);
+                            const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES);
+#pragma unroll
+                            for (int k = 0; k < GG_BK / 16; ++k)
+                                umma_bf16_ss_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, IDESC,
+                                                  (kb | sb | k) != 0 ? 1u : 0u);
+                        }
                         umma_commit_pair_multicast(&empty_bar[stage], 0x3);
                     }
                     __syncwarp();
@@ -237,15 +251,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
             int g, nb, mb;
             locate(tile, g, nb, mb);
             const int row_end = s_off[g + 1];
-            const int r = s_off[g] + mb * GP_BM + (int)rank * 128 + q * 32 + lane;
-            const bool valid = r < row_end;
+            const int row_base = s_off[g] + mb * GP_BM + (int)rank * 128 + q * 32;  // row of lane 0
             if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const int col_base = nb * S::OUT_COLS;
-            __nv_bfloat16* dst_row = args.out + (size_t)(valid ? r : 0) * args.n_out;
+            uint8_t* my_stage = epi_stage + (warp - 2) * 2048;
 #pragma unroll 1
             for (int c0 = 0; c0 < S::OUT_COLS; c0 += 32) {
                 const int col0 = col_base + c0;
@@ -268,13 +281,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
                     for (int i = 0; i < 16; ++i)
                         pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                 }
-                if (valid) {
-#pragma unroll
-                    for (int v8 = 0; v8 < 4; ++v8)
-                        if (c0 + v8 * 8 < S::OUT_COLS && col0 + v8 * 8 < args.n_out)
-                            *reinterpret_cast<uint4*>(dst_row + col0 + v8 * 8) =
-                                make_uint4(pk[4 * v8], pk[4 * v8 + 1], pk[4 * v8 + 2], pk[4 * v8 + 3]);
-                }
+                store_warp_rows_32cols(my_stage, pk, lane, args.out, args.n_out, row_base, row_end, col0, args.n_out,
+                                       S::OUT_COLS - c0);
             }
             tc_fence_before_sync();
             __syncwarp();

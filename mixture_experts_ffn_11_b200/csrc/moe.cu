@@ -17,6 +17,7 @@
 #include "permute.cuh"
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
+#include "gemm_wide.cuh"
 #include "combine.cuh"
 
 using namespace moe;
@@ -53,6 +54,14 @@ using Single64DN = GemmShape<64, 8, false>;
 using Pair256GU = GemmPairShape<256, 6, true>;
 using Pair256DN = GemmPairShape<256, 6, false>;
 using Pair240DN = GemmPairShape<240, 6, false>;
+using Pair256GU2 = GemmPairShape<256, 3, true, 2>;  // two K blocks per stage, for K >= kSub2MinK
+constexpr int kSub2MinK = 4096;
+//   CTA pair with two accumulators (2*NH-wide tiles, NH 256 or 240) when K is long
+using Wide256GU = GemmWideShape<256, 4, true>;
+using Wide240GU = GemmWideShape<240, 4, true>;
+using Wide256DN = GemmWideShape<256, 4, false>;
+using Wide240DN = GemmWideShape<240, 4, false>;
+constexpr int kWideMinK = 8192;  // the wide tile's epilogue is not overlapped: it pays off on long K only
 
 cudaError_t set_gemm_attributes() {
     const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
@@ -63,6 +72,12 @@ cudaError_t set_gemm_attributes() {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<256, 6, true>, a, Pair256GU::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<256, 6, false>, a, Pair256DN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<240, 6, false>, a, Pair240DN::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_pair_kernel<256, 3, true, 2>, a, Pair256GU2::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<256, 4, true>, a, Wide256GU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, true>, a, Wide240GU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<256, 4, false>, a, Wide256DN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, false>, a, Wide240DN::SMEM_BYTES);
     return e;
 }
 
@@ -207,9 +222,9 @@ moe_status_t launch_single(const GemmProblem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup" : "grouped_gemm_down");
 }
 
-template <int BN, int STAGES, bool GATEUP>
+template <int BN, int STAGES, bool GATEUP, int SUB = 1>
 moe_status_t launch_pair(const GemmProblem& p, int sms, cudaStream_t stream) {
-    using S = GemmPairShape<BN, STAGES, GATEUP>;
+    using S = GemmPairShape<BN, STAGES, GATEUP, SUB>;
     CUtensorMap ta, tb;
     moe_status_t st = make_gemm_maps(p, GATEUP, BN / 2, &ta, &tb);
     if (st != MOE_OK) return st;
@@ -217,16 +232,41 @@ moe_status_t launch_pair(const GemmProblem& p, int sms, cudaStream_t stream) {
     const long upper = ((long)p.M / GP_BM + p.G) * (long)args.n_tiles;
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GP_BM ? 1 : 0;
-    grouped_gemm_pair_kernel<BN, STAGES, GATEUP><<<2 * clusters, GG_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args,
-                                                                                                      streamed_once);
+    grouped_gemm_pair_kernel<BN, STAGES, GATEUP, SUB><<<2 * clusters, GG_THREADS, S::SMEM_BYTES, stream>>>(
+        ta, tb, args, streamed_once);
     return check_launch(GATEUP ? "grouped_gemm_gateup (pair)" : "grouped_gemm_down (pair)");
+}
+
+template <int NH, int STAGES, bool GATEUP>
+moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
+    using S = GemmWideShape<NH, STAGES, GATEUP>;
+    CUtensorMap ta, tb;
+    moe_status_t st = make_gemm_maps(p, GATEUP, NH, &ta, &tb);
+    if (st != MOE_OK) return st;
+    const GemmArgs args = gemm_args(p, S::OUT_COLS);
+    const long upper = ((long)p.M / GP_BM + p.G) * (long)args.n_tiles;
+    const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
+    const int streamed_once = (long)p.M <= (long)p.G * GP_BM ? 1 : 0;
+    grouped_gemm_wide_kernel<NH, STAGES, GATEUP><<<2 * clusters, GW_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args,
+                                                                                                      streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)");
 }
 
 // Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs. Otherwise a single CTA
 // per tile, 256 wide unless that leaves SMs idle (e.g. one small group), then 64 wide.
 moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cudaStream_t stream) {
+    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2 && p.K >= kWideMinK) {
+        // columns padded per tile: gate|up NH per tile, down 2*NH per tile; pick the width that pads less
+        const long span = gateup ? 1 : 2;
+        const long w256 = (long)(p.n_out + 256 * span - 1) / (256 * span) * (256 * span);
+        const long w240 = (long)(p.n_out + 240 * span - 1) / (240 * span) * (240 * span);
+        if (gateup)
+            return w240 < w256 ? launch_wide<240, 4, true>(p, sms, stream) : launch_wide<256, 4, true>(p, sms, stream);
+        return w240 < w256 ? launch_wide<240, 4, false>(p, sms, stream) : launch_wide<256, 4, false>(p, sms, stream);
+    }
     if ((long)p.M >= (long)p.G * GG_BM && sms >= 2) {
-        if (gateup) return launch_pair<256, 6, true>(p, sms, stream);
+        if (gateup)
+            return p.K >= kSub2MinK ? launch_pair<256, 3, true, 2>(p, sms, stream) : launch_pair<256, 6, true>(p, sms, stream);
         const long w256 = (long)(p.n_out + 255) / 256 * 256, w240 = (long)(p.n_out + 239) / 240 * 240;
         if (w240 < w256) return launch_pair<240, 6, false>(p, sms, stream);
         return launch_pair<256, 6, false>(p, sms, stream);

@@ -37,6 +37,9 @@ class MoEFFN:
         self.device = w_gateup.device
         self._T = None
         self.buf = {}
+        # the shared expert depends only on x: it runs on a side stream, beside routing and grouping (which
+        # leave most SMs free), and the routed GEMMs wait for it
+        self._side = torch.cuda.Stream(self.device) if self.shared_f else None
 
     def buffers(self, T: int) -> dict:
         """Allocate (once per T) every intermediate the layer writes."""
@@ -69,8 +72,9 @@ class MoEFFN:
     def forward(self, x, stream=None, timing=None):
         """y = MoE(x) for x [T, d] bf16 on the GPU. Returns the layer's output buffer [T, d] (bf16).
 
-        timing: optional dict; if given, a (start, end) pair of CUDA events is recorded on the stream
-        around each stage ("route", "permute", "gateup", "down", "shared", "combine").
+        timing: optional dict; if given, a (start, end) pair of CUDA events is recorded around each stage
+        ("route", "permute", "gateup", "down", "combine" on the layer's stream; "shared", the always-on
+        expert, on the side stream where it overlaps routing and grouping).
         """
         T = x.shape[0]
         b = self.buffers(T)
@@ -83,6 +87,23 @@ class MoEFFN:
                 timing[name] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             timing[name][0 if first else 1].record(s)
 
+        shared = None
+        if self.shared_f:
+            side = self._side
+            x_ready = torch.cuda.Event()
+            x_ready.record(s)
+            side.wait_event(x_ready)  # also orders after the previous call's combine, which read `shared`
+            if timing is not None:
+                timing["shared"] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                timing["shared"][0].record(side)
+            N.grouped_gemm_gateup(x, self.w_gateup_shared.unsqueeze(0), b["shared_offsets"], b["h_shared"], side)
+            N.grouped_gemm_down(b["h_shared"], self.w_down_shared.unsqueeze(0), b["shared_offsets"], b["shared"],
+                                side)
+            shared_done = torch.cuda.Event()
+            shared_done.record(side)
+            if timing is not None:
+                timing["shared"][1].record(side)
+            shared = b["shared"]
         mark("route", True)
         N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"], s)
         mark("route", False)
@@ -90,20 +111,15 @@ class MoEFFN:
         N.permute(x, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], b["x_perm"],
                   b["ws"], s)
         mark("permute", False)
+        if shared is not None:
+            # the routed GEMMs are persistent kernels sized to every SM: they start once the shared expert is done
+            s.wait_event(shared_done)
         mark("gateup", True)
         N.grouped_gemm_gateup(b["x_perm"], self.w_gateup, b["offsets"], b["h"], s)
         mark("gateup", False)
         mark("down", True)
         N.grouped_gemm_down(b["h"], self.w_down, b["offsets"], b["y_perm"], s)
         mark("down", False)
-        shared = None
-        if self.shared_f:
-            mark("shared", True)
-            N.grouped_gemm_gateup(x, self.w_gateup_shared.unsqueeze(0), b["shared_offsets"], b["h_shared"], s)
-            N.grouped_gemm_down(b["h_shared"], self.w_down_shared.unsqueeze(0), b["shared_offsets"], b["shared"],
-                                s)
-            mark("shared", False)
-            shared = b["shared"]
         mark("combine", True)
         N.unpermute_combine(b["y_perm"], b["inv_perm"], b["topk_w"], shared, b["y"], s)
         mark("combine", False)

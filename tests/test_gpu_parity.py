@@ -241,6 +241,11 @@ RAGGED = [
     ("pair_ragged", [0, 1, 255, 256, 257, 600, 0, 129], 256, 200),
     ("pair_down_240_wide", [300, 0, 700, 45], 480, 136),
     ("pair_one_expert", [0, 0, 2000, 0], 256, 256),
+    # CTA pair with two accumulators (K >= 8192): 240-wide gate|up; 256-wide down
+    ("wide_gateup_240", [300, 0, 700, 45], 8192, 240),
+    ("wide_down_256", [400, 1, 129], 512, 8192),
+    # CTA pair, two K blocks per ring stage (gate|up with K >= 4096), K tail inside the last stage
+    ("pair_two_kblocks_per_stage", [0, 300, 1, 257], 4160, 136),
     # single-CTA kernel, 256 wide (many groups of a few rows) and 64 wide (one small group)
     ("single_wide", [2] * 160, 64, 256),
     ("single_group_narrow", [50], 512, 256),
