@@ -137,8 +137,8 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
  *  - Sizes whose moe_permute_workspace_size(T, E, k) exceeds
  *    MOE_PERMUTE_STATIC_WS_BYTES are rejected with MOE_ERR_WORKSPACE before
  *    anything is launched (the scratch is 4 bytes per expert per block of
- *    4096 assignments: E = 128 allows up to 8,388,608 assignments T*k,
- *    E = 1024 up to 1,048,576).
+ *    1024 assignments: E = 128 allows up to 2,097,152 assignments T*k,
+ *    E = 1024 up to 262,144).
  *  - The first call on a device looks up the array's device address (a
  *    one-time set-up per device); make that first call before capturing a
  *    stream.

@@ -278,6 +278,28 @@ moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cud
     return gateup ? launch_single<64, 8, true>(p, sms, stream) : launch_single<64, 8, false>(p, sms, stream);
 }
 
+template <int BNR>
+moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, const float* bias, int T, int d, int E,
+                              int k, int mode, int fuse, float* logits, int32_t* idx, float* w, int tiles, int cs,
+                              cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * cs));
+    cfg.blockDim = dim3(RTC_THREADS);
+    cfg.dynamicSmemBytes = RouterTcShape<BNR>::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BNR>, tm, tw, bias, T, d, E, k, mode, fuse,
+                                             logits, idx, w);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "router_tc launch: %s", cudaGetErrorString(e));
+    return MOE_OK;
+}
+
 moe_status_t check_gemm_args(const void* a, const void* w, const int32_t* offsets, int G, int M, int d, int f,
                              const void* out) {
     if (!a || !w || !offsets || !out) return fail(MOE_ERR_INVALID_ARG, "null pointer argument");
@@ -365,19 +387,27 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
                             CU_TENSOR_MAP_SWIZZLE_NONE)) != MOE_OK)
             return st;
         const int fuse = k <= RTC_KMAX ? 1 : 0;
-        const int grid = (T + RTC_BM - 1) / RTC_BM;
+        const int tiles = (T + RTC_BM - 1) / RTC_BM;
+        const int kblocks = (d + RTC_BK - 1) / RTC_BK;
+        // split K over a cluster when there are few 128-token tiles (keeps >= 2 K blocks per CTA)
+        int cs = 1;
+        if (tiles * 4 <= di.sms && kblocks >= 8)
+            cs = 4;
+        else if (tiles * 2 <= di.sms && kblocks >= 4)
+            cs = 2;
         if (E <= 16)
-            router_tc_kernel<16><<<grid, RTC_THREADS, RouterTcShape<16>::SMEM_BYTES, stream>>>(
-                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+            st = launch_router_tc<16>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
+                                      stream);
         else if (E <= 32)
-            router_tc_kernel<32><<<grid, RTC_THREADS, RouterTcShape<32>::SMEM_BYTES, stream>>>(
-                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+            st = launch_router_tc<32>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
+                                      stream);
         else if (E <= 64)
-            router_tc_kernel<64><<<grid, RTC_THREADS, RouterTcShape<64>::SMEM_BYTES, stream>>>(
-                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+            st = launch_router_tc<64>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
+                                      stream);
         else
-            router_tc_kernel<128><<<grid, RTC_THREADS, RouterTcShape<128>::SMEM_BYTES, stream>>>(
-                tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w);
+            st = launch_router_tc<128>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles,
+                                       cs, stream);
+        if (st != MOE_OK) return st;
         if ((st = check_launch("router_tc")) != MOE_OK) return st;
         if (fuse) return MOE_OK;
     } else if ((size_t)d * sizeof(float) <= (size_t)kRouterSmallMaxSmem) {

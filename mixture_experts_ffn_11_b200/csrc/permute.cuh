@@ -3,17 +3,17 @@
 // as a stable counting sort: expert histogram -> exclusive scan -> stable scatter, then a gather of
 // x rows into expert-contiguous order ("dispatch tokens to their selected expert weights").
 //
-// Stability without atomics on positions: the assignments are cut into segments of
-// PERM_SEG = 8 warps x 512; segment histograms are scanned in segment order, and inside a segment
-// each warp walks its 512 assignments in order, ranking equal experts within 32 lanes with
-// __match_any_sync. Positions therefore depend only on the input, never on timing.
+// Stability without atomics on positions: the assignments are cut into segments of PERM_SEG = 8 warps x 128
+// (small segments, so even a few thousand tokens spread over many CTAs); segment histograms are scanned in
+// segment order, and inside a segment each warp walks its 128 assignments in order, ranking equal experts
+// within 32 lanes with __match_any_sync. Positions therefore depend only on the input, never on timing.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int PERM_WARPS = 8;
-constexpr int PERM_PER_WARP = 512;
+constexpr int PERM_PER_WARP = 128;
 constexpr int PERM_SEG = PERM_WARPS * PERM_PER_WARP;  // assignments per segment (block)
 constexpr int PERM_THREADS = PERM_WARPS * 32;
 

@@ -12,7 +12,12 @@
 // buffers (as many as fit, up to 8, so the round trip MMA -> drain -> reuse is not on the critical
 // path), and CUDA-core threads add the block partials into fp32 registers with IEEE round-to-nearest.
 //
-// One CTA per 128-token tile (320 threads):
+// Split K across a cluster: a 128-token tile is processed by a cluster of CS CTAs (1, 2 or 4), each taking a
+// contiguous range of K blocks; the partial sums go through shared memory and the cluster's first CTA adds its
+// peers' partials over DSMEM in rank order (deterministic) and runs the epilogue. Small expert counts leave
+// few 128-token tiles, so without the split most SMs would idle.
+//
+// Per CTA (320 threads):
 //   warp 0     TMA of the x tile [128 x 64] bf16 and of the W_r block [BNR x 64] fp32 per K block into a
 //              STAGES-deep ring (the W_r block lands unswizzled, 256 bytes per expert row)
 //   warp 1     TMEM allocation; one lane issues 3 x 4 tcgen05.mma (M=128, N=BNR, K=16) per K block into
@@ -47,15 +52,17 @@ struct RouterTcShape {
     static_assert((3 * STAGES + 2 * NBUF + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
 };
 
-__device__ __forceinline__ void split3_bf16(float w, uint16_t& hi, uint16_t& mid, uint16_t& lo) {
-    const __nv_bfloat16 h = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(h);
-    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(m);
-    const __nv_bfloat16 l = __float2bfloat16_rn(r2);
-    hi = *reinterpret_cast<const uint16_t*>(&h);
-    mid = *reinterpret_cast<const uint16_t*>(&m);
-    lo = *reinterpret_cast<const uint16_t*>(&l);
+// Exact three-way split of two fp32 weights into bf16 pieces, packed in pairs: hi = w truncated to bf16
+// (its top 16 bits), mid = (w - hi) truncated likewise, lo = bf16(w - hi - mid) rounded to nearest; the two
+// subtractions are exact, so hi + mid + lo equals w to ~2^-25 relative.
+__device__ __forceinline__ void split3_pair(float w0, float w1, uint32_t& hi, uint32_t& mid, uint32_t& lo) {
+    const uint32_t u0 = __float_as_uint(w0), u1 = __float_as_uint(w1);
+    const float r0 = w0 - __uint_as_float(u0 & 0xffff0000u), r1 = w1 - __uint_as_float(u1 & 0xffff0000u);
+    const uint32_t v0 = __float_as_uint(r0), v1 = __float_as_uint(r1);
+    const float s0 = r0 - __uint_as_float(v0 & 0xffff0000u), s1 = r1 - __uint_as_float(v1 & 0xffff0000u);
+    hi = __byte_perm(u0, u1, 0x7632);  // upper halves: element 0 in the low 16 bits
+    mid = __byte_perm(v0, v1, 0x7632);
+    lo = pack_bf16x2(s0, s1);
 }
 
 template <int BNR>
@@ -78,8 +85,11 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * RTC_BM;
-    const int KB = (d + RTC_BK - 1) / RTC_BK;
+    const uint32_t rank = cluster_ctarank(), cs = cluster_nctarank();
+    const int m0 = (int)(blockIdx.x / cs) * RTC_BM;
+    const int KB_all = (d + RTC_BK - 1) / RTC_BK;
+    const int kb0 = (int)(rank * KB_all / cs);                          // this CTA's K blocks
+    const int KB = (int)((rank + 1) * KB_all / cs) - kb0;              // (count; the host keeps it >= 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -105,6 +115,15 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    // drain warps (6-9): this thread's row of the tile and its running fp32 partial sums
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
+    const int row = m0 + q * 32 + lane;
+    const bool valid = row < T;
+    const bool is_drain = warp >= 6;
+    float sum[BNR];
+#pragma unroll
+    for (int j = 0; j < BNR; ++j) sum[j] = 0.f;
+    bool drain_ok = false;
 
     if (warp == 0) {
         // ---------------- TMA: x tile ----------------
@@ -121,8 +140,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             if (lane == 0) {
                 uint8_t* sa = smem + stage * S::STAGE_BYTES;
                 mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES + S::W_BYTES);
-                tma_load_2d(sa, &tmX, &full_bar[stage], kb * RTC_BK, m0, pol);
-                tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], kb * RTC_BK, 0, pol_w);
+                tma_load_2d(sa, &tmX, &full_bar[stage], (kb0 + kb) * RTC_BK, m0, pol);
+                tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], (kb0 + kb) * RTC_BK, 0, pol_w);
             }
             ++issued;
             if (++stage == STAGES) {
@@ -194,14 +213,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 const float w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                 uint32_t hi[4], mi[4], lo[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint16_t h0, md0, l0, h1, md1, l1;
-                    split3_bf16(w8[2 * j], h0, md0, l0);
-                    split3_bf16(w8[2 * j + 1], h1, md1, l1);
-                    hi[j] = (uint32_t)h0 | ((uint32_t)h1 << 16);
-                    mi[j] = (uint32_t)md0 | ((uint32_t)md1 << 16);
-                    lo[j] = (uint32_t)l0 | ((uint32_t)l1 << 16);
-                }
+                for (int j = 0; j < 4; ++j) split3_pair(w8[2 * j], w8[2 * j + 1], hi[j], mi[j], lo[j]);
                 const int off = r * 128 + ((c ^ (r & 7)) << 4);
                 *reinterpret_cast<uint4*>(pbase + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<uint4*>(pbase + S::P_BYTES + off) = make_uint4(mi[0], mi[1], mi[2], mi[3]);
@@ -216,13 +228,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         }
     } else {
         // ---------------- drain + epilogue (warps 6-9) ----------------
-        const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
-        const int row = m0 + q * 32 + lane;
-        const bool valid = row < T;
         const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
-        float sum[BNR];
-#pragma unroll
-        for (int j = 0; j < BNR; ++j) sum[j] = 0.f;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             const int acc = kb % NBUF;
@@ -250,6 +256,33 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty_bar[acc]);
         }
+        drain_ok = ok;
+    }
+
+    // ---- split-K reduction over the cluster, then the epilogue in the cluster's first CTA ----
+    tc_fence_before_sync();
+    __syncthreads();  // all roles done: the ring is free, every MMA has been drained
+    if (cs > 1) {
+        float* red = reinterpret_cast<float*>(smem);  // [BNR][128] partial sums (column-major: no bank conflicts)
+        if (is_drain) {
+#pragma unroll
+            for (int j = 0; j < BNR; ++j) red[j * RTC_BM + q * 32 + lane] = sum[j];
+        }
+        cluster_sync();
+        if (rank == 0 && is_drain) {
+            const uint32_t base = smem_u32(red);
+            for (uint32_t r = 1; r < cs; ++r) {
+                const uint32_t peer = mapa_shared(base, r);
+#pragma unroll
+                for (int j = 0; j < BNR; ++j)
+                    sum[j] += ld_shared_cluster_f32(peer + (uint32_t)((j * RTC_BM + q * 32 + lane) * 4));
+            }
+        }
+        cluster_sync();  // no CTA leaves while the first one may still read its shared memory
+        // (a CTA whose pipeline wait gave up has already set the device error word)
+    }
+    if (rank == 0 && is_drain) {
+        bool ok = drain_ok && !*abort_flag;
         if (ok) {
             float* lrow = logits + (size_t)(valid ? row : 0) * E;
             float tv[RTC_KMAX];
@@ -324,8 +357,6 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         }
     }
 
-    tc_fence_before_sync();
-    __syncthreads();
     tc_fence_after_sync();
     if (warp == 1) {
         if (lane == 0) mbar_wait_drain(final_bar, 0);

@@ -39,8 +39,8 @@ def test_every_declared_symbol_is_exported(native):
 def test_workspace_size(native):
     ws = native.permute_workspace_size
     assert ws(0, 8, 2) == 0
-    assert ws(64, 8, 2) == 256  # one 4096-assignment segment x 8 experts x 4 B, rounded to 256
-    assert ws(16384, 128, 8) == 32 * 128 * 4
+    assert ws(64, 8, 2) == 256  # one 1024-assignment segment x 8 experts x 4 B, rounded to 256
+    assert ws(16384, 128, 8) == 128 * 128 * 4
     assert ws(4096, 32, 4) % 256 == 0
 
 
