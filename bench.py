@@ -37,8 +37,8 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu capture, keyed by the
 # kernel, the workload and a hash of the kernel's source files at capture time. A stale hash -> null.
 TRAFFIC = {}
-KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/gemm.cuh", "mixture_experts_ffn_11_b200/csrc/sm100.cuh",
-                  "mixture_experts_ffn_11_b200/csrc/common.cuh"]
+KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
+                  ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "sm100.cuh", "common.cuh", "moe.cu")]
 
 
 def kernel_source_hash() -> str:

@@ -373,7 +373,7 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     if (T == 0) return MOE_OK;
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     if (E <= 128 && T >= kRouterTcMinT) {
-        // tensor cores, W_r split into three bf16 pieces; top-k fused when k <= 8
+        // tensor cores, W_r split into three bf16 pieces; top-k fused (any k <= 32)
         CUtensorMap tm, tw;
         const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)d * 2};

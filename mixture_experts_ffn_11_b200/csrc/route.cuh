@@ -99,15 +99,13 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-constexpr int TOPK_WARPS = 8;
-
-__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ logits, int T, int E,
-                                                                 int k, int mode, int32_t* __restrict__ topk_idx,
-                                                                 float* __restrict__ topk_w) {
+// One warp routes one token: selects its k largest logits (descending; equal values keep the lower expert id
+// first) and computes the routing weights of `mode`. get(e) returns logit e; lane j < k writes slot j of
+// idx_row / w_row. k <= 32.
+template <class Get>
+__device__ __forceinline__ void warp_route_select(Get get, int E, int k, int mode, int32_t* __restrict__ idx_row,
+                                                  float* __restrict__ w_row) {
     const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * TOPK_WARPS + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const float* l = logits + (size_t)t * E;
     const int per = (E + 31) / 32;
     // E <= 256: the token's logits stay in registers (8 per lane) across the k rounds
     constexpr int RPER = 8;
@@ -116,7 +114,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
 #pragma unroll
         for (int s = 0; s < RPER; ++s) {
             const int e = s * 32 + lane;
-            rv[s] = (s < per && e < E) ? l[e] : 0.f;
+            rv[s] = (s < per && e < E) ? get(e) : 0.f;
         }
     }
     uint32_t taken = 0;
@@ -135,7 +133,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
             for (int s = 0; s < per; ++s) {
                 const int e = s * 32 + lane;
                 if (e >= E || (taken >> s) & 1u) continue;
-                const float v = l[e];
+                const float v = get(e);
                 if (c.e == INT_MAX || v > c.v) c = Cand{v, e};
             }
         }
@@ -164,7 +162,7 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
             float part = 0.f;
             for (int s = 0; s < per; ++s) {
                 const int e = s * 32 + lane;
-                if (e < E) part += expf(l[e] - vmax);
+                if (e < E) part += expf(get(e) - vmax);
             }
             const float zall = warp_sum(part);
             const float p = ex / zall;  // probability under the full softmax
@@ -174,9 +172,20 @@ __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __re
         }
     }
     if (mine) {
-        topk_idx[(size_t)t * k + lane] = my_e;
-        topk_w[(size_t)t * k + lane] = w;
+        idx_row[lane] = my_e;
+        w_row[lane] = w;
     }
+}
+
+constexpr int TOPK_WARPS = 8;
+
+__global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ logits, int T, int E,
+                                                                 int k, int mode, int32_t* __restrict__ topk_idx,
+                                                                 float* __restrict__ topk_w) {
+    const int t = blockIdx.x * TOPK_WARPS + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* l = logits + (size_t)t * E;
+    warp_route_select([=](int e) { return l[e]; }, E, k, mode, topk_idx + (size_t)t * k, topk_w + (size_t)t * k);
 }
 
 }  // namespace moe

@@ -11,6 +11,9 @@
 // reaches ~1e-5 of the logit). So each 64-wide K block is accumulated on its own, in one of NBUF TMEM
 // buffers (as many as fit, up to 8, so the round trip MMA -> drain -> reuse is not on the critical
 // path), and CUDA-core threads add the block partials into fp32 registers with IEEE round-to-nearest.
+// When 3 * BNR <= 256 the three pieces sit one after another as the rows of a single B operand, so one MMA
+// per 16-wide K step (N = 3 * BNR) gives the three partial products side by side in TMEM and the drain adds
+// them: 4 MMAs per K block instead of 12 (small-N MMAs cost about as much to issue as large ones).
 //
 // Split K across a cluster: a 128-token tile is processed by a cluster of CS CTAs (1, 2 or 4), each taking a
 // contiguous range of K blocks; the partial sums go through shared memory and the cluster's first CTA adds its
@@ -24,15 +27,22 @@
 //              accumulator buffer (kb % NBUF), starting it afresh
 //   warps 2-5  convert the staged W_r block into the three bf16 pieces, stored in the 128-byte-swizzled
 //              K-major layout the TMA engine writes, then signal conv[stage]
-//   warps 6-9  drain: add each finished block partial of their 32 TMEM lanes into registers; at the end
-//              + bias, store the logits row, select the top-k (k <= 8) by insertion in descending order
-//              (equal logits keep the lower expert id first) and write the routing weights.
+//   warps 6-9  drain: add each finished block partial of their 32 TMEM lanes into registers
+// Epilogue (the cluster's first CTA), top-k by insertion into a sorted list of 8 (descending, equal logits keep
+// the lower expert id first), then the routing weights of the mode:
+//   BNR <= 32, k <= 8: each drain thread routes its own token from its registers (the unrolled insertion is
+//              short for so few experts), storing its logits row itself;
+//   otherwise: the sums + bias go to shared memory; warps 4-9 store the logits row by row (coalesced) while
+//              threads 0-127 route one token each with a loop over the experts that skips logits not above the
+//              current k-th (k > 8: one warp per token runs warp_route_select, the stand-alone top-k code).
 #pragma once
 #include "common.cuh"
+#include "route.cuh"
 
 namespace moe {
 
-constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 320, RTC_KMAX = 8;
+constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 320, RTC_KMAX = 32, RTC_KINS = 8;
+constexpr int RTC_RED_LD = RTC_BM + 1;  // row stride of the [expert][token] sums in shared memory (odd: no bank conflicts)
 
 template <int BNR>
 struct RouterTcShape {
@@ -44,12 +54,16 @@ struct RouterTcShape {
     static_assert(STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
     static constexpr int STAGES = (200 * 1024) / STAGE_BYTES > 8 ? 8 : (200 * 1024) / STAGE_BYTES;
     static_assert(STAGES >= 2, "ring depth");
-    static constexpr int NBUF = 512 / BNR >= 8 ? 8 : 512 / BNR;  // partial-sum buffers in TMEM
-    static constexpr int TMEM_COLS = NBUF * BNR <= 32 ? 32 : (NBUF * BNR <= 64 ? 64 : (NBUF * BNR <= 128 ? 128 : (NBUF * BNR <= 256 ? 256 : 512)));
+    static constexpr bool JOINT = 3 * BNR <= 256;                // one MMA over [hi; mid; lo] per K step
+    static constexpr int ACC_COLS = JOINT ? 3 * BNR : BNR;           // TMEM columns of one K block's result
+    static constexpr int ACC_STRIDE = ACC_COLS <= 64 ? 64 : (ACC_COLS <= 128 ? 128 : 256);
+    static constexpr int NBUF = 512 / ACC_STRIDE >= 8 ? 8 : 512 / ACC_STRIDE;  // partial-sum buffers in TMEM
+    static constexpr int TMEM_COLS = NBUF * ACC_STRIDE <= 256 ? 256 : 512;
     static constexpr int BAR_BYTES = 512;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((3 * STAGES + 2 * NBUF + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert(BNR * RTC_RED_LD * 4 <= STAGES * STAGE_BYTES, "epilogue sums reuse the ring");
 };
 
 // Exact three-way split of two fp32 weights into bf16 pieces, packed in pairs: hi = w truncated to bf16
@@ -63,6 +77,89 @@ __device__ __forceinline__ void split3_pair(float w0, float w1, uint32_t& hi, ui
     hi = __byte_perm(u0, u1, 0x7632);  // upper halves: element 0 in the low 16 bits
     mid = __byte_perm(v0, v1, 0x7632);
     lo = pack_bf16x2(s0, s1);
+}
+
+// Routing weights of the first k entries of a sorted selection (tv descending, te the expert ids):
+//   sigmoid_topk_norm    sigmoid(v_j) / sum of the selected sigmoids
+//   topk_softmax         softmax over the selected logits
+//   softmax_topk_renorm  softmax over all E logits (zall = sum_e exp(v_e - v_max)), renormalised over the selection
+__device__ __forceinline__ void route_weights(const float (&tv)[RTC_KINS], const int (&te)[RTC_KINS], int k, int mode,
+                                              float zall, int32_t* __restrict__ idx_row, float* __restrict__ w_row) {
+    float wv[RTC_KINS];
+    float z = 0.f;
+    if (mode == MOE_ROUTE_SIGMOID_TOPK_NORM) {
+#pragma unroll
+        for (int j = 0; j < RTC_KINS; ++j)
+            if (j < k) {
+                wv[j] = 1.f / (1.f + expf(-tv[j]));
+                z += wv[j];
+            }
+    } else {
+#pragma unroll
+        for (int j = 0; j < RTC_KINS; ++j)
+            if (j < k) {
+                wv[j] = expf(tv[j] - tv[0]);
+                z += wv[j];
+            }
+        if (mode == MOE_ROUTE_SOFTMAX_TOPK_RENORM) {
+            float zp = 0.f;
+#pragma unroll
+            for (int j = 0; j < RTC_KINS; ++j)
+                if (j < k) {
+                    wv[j] = wv[j] / zall;
+                    zp += wv[j];
+                }
+            z = zp;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < RTC_KINS; ++j)
+        if (j < k) {
+            idx_row[j] = te[j];
+            w_row[j] = wv[j] / z;
+        }
+}
+
+// Routes one token from its E logits at col[e * RTC_RED_LD] (shared memory), k <= RTC_KINS: tv/te hold the
+// RTC_KINS largest so far in the order (descending value, lower expert id first); a new logit bubbles down from
+// the top, taking the first slot it beats strictly, so an equal value stays behind the earlier (lower) id.
+// Logits not above the current k-th are skipped (they cannot reach the first k slots).
+__device__ __forceinline__ void route_token_insertion(const float* col, int E, int k, int mode,
+                                                      int32_t* __restrict__ idx_row, float* __restrict__ w_row) {
+    float tv[RTC_KINS];
+    int te[RTC_KINS];
+#pragma unroll
+    for (int i = 0; i < RTC_KINS; ++i) {
+        tv[i] = 0.f;
+        te[i] = INT_MAX;
+    }
+    int filled = 0;  // min(experts seen, k)
+    float kth = 0.f;  // tv[k-1] once filled == k
+#pragma unroll 4
+    for (int e = 0; e < E; ++e) {
+        float cv = col[e * RTC_RED_LD];
+        if (filled == k && !(cv > kth)) continue;
+        int ce = e;
+#pragma unroll
+        for (int i = 0; i < RTC_KINS; ++i) {
+            if (te[i] == INT_MAX || cv > tv[i]) {
+                const float tf = tv[i];
+                const int ti = te[i];
+                tv[i] = cv;
+                te[i] = ce;
+                cv = tf;
+                ce = ti;
+            }
+        }
+        if (filled < k) ++filled;
+#pragma unroll
+        for (int i = 0; i < RTC_KINS; ++i)
+            if (i == k - 1) kth = tv[i];
+    }
+    float zall = 0.f;  // softmax over all E logits, relative to the largest (renormalising mode only)
+    if (mode == MOE_ROUTE_SOFTMAX_TOPK_RENORM)
+        for (int e = 0; e < E; ++e) zall += expf(col[e * RTC_RED_LD] - tv[0]);
+    route_weights(tv, te, k, mode, zall, idx_row, w_row);
 }
 
 template <int BNR>
@@ -117,8 +214,6 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     // drain warps (6-9): this thread's row of the tile and its running fp32 partial sums
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
-    const int row = m0 + q * 32 + lane;
-    const bool valid = row < T;
     const bool is_drain = warp >= 6;
     float sum[BNR];
 #pragma unroll
@@ -155,7 +250,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA: one fresh accumulation per K block ----------------
-        constexpr uint32_t IDESC = idesc_bf16_f32(RTC_BM, BNR);
+        constexpr uint32_t IDESC = idesc_bf16_f32(RTC_BM, S::ACC_COLS);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -172,13 +267,20 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             if (lane == 0) {
                 const uint32_t sa = smem_u32(smem + stage * S::STAGE_BYTES);
                 const uint64_t adesc = smem_desc_sw128(sa);
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BNR);
-#pragma unroll
-                for (int p = 0; p < 3; ++p) {
-                    const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + S::W_BYTES + p * S::P_BYTES);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_STRIDE);
+                if constexpr (S::JOINT) {  // the pieces are consecutive row blocks: one B operand of 3*BNR rows
+                    const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + S::W_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < RTC_BK / 16; ++kk)
-                        umma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (p | kk) != 0 ? 1u : 0u);
+                        umma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, kk != 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 3; ++p) {
+                        const uint64_t bdesc = smem_desc_sw128(sa + S::A_BYTES + S::W_BYTES + p * S::P_BYTES);
+#pragma unroll
+                        for (int kk = 0; kk < RTC_BK / 16; ++kk)
+                            umma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (p | kk) != 0 ? 1u : 0u);
+                    }
                 }
                 umma_commit(&empty_bar[stage]);
                 umma_commit(&tfull_bar[acc]);
@@ -227,7 +329,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             }
         }
     } else {
-        // ---------------- drain + epilogue (warps 6-9) ----------------
+        // ---------------- drain (warps 6-9) ----------------
         const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
@@ -236,17 +338,34 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
-            if constexpr (BNR == 16) {  // a 32-column load would leave the 32-column allocation
-                uint32_t v[16];
-                tmem_load_16cols(t_row + (uint32_t)(acc * BNR), v);
+            const uint32_t t_acc = t_row + (uint32_t)(acc * S::ACC_STRIDE);
+            if constexpr (S::JOINT && BNR == 16) {
+                uint32_t h[16], m[16], l[16];
+                tmem_load_16cols(t_acc, h);
+                tmem_load_16cols(t_acc + 16, m);
+                tmem_load_16cols(t_acc + 32, l);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) sum[j] += __uint_as_float(v[j]);
+                for (int j = 0; j < 16; ++j)
+                    sum[j] += (__uint_as_float(h[j]) + __uint_as_float(m[j])) + __uint_as_float(l[j]);
+            } else if constexpr (S::JOINT) {
+#pragma unroll
+                for (int c0 = 0; c0 < BNR; c0 += 32) {
+                    if (c0 < E) {
+                        uint32_t h[32], m[32], l[32];
+                        tmem_load_32cols(t_acc + c0, h);
+                        tmem_load_32cols(t_acc + BNR + c0, m);
+                        tmem_load_32cols(t_acc + 2 * BNR + c0, l);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            sum[c0 + j] += (__uint_as_float(h[j]) + __uint_as_float(m[j])) + __uint_as_float(l[j]);
+                    }
+                }
             } else {
 #pragma unroll
                 for (int c0 = 0; c0 < BNR; c0 += 32) {
                     if (c0 < E) {
                         uint32_t v[32];
-                        tmem_load_32cols(t_row + (uint32_t)(acc * BNR + c0), v);
+                        tmem_load_32cols(t_acc + c0, v);
 #pragma unroll
                         for (int j = 0; j < 32; ++j) sum[c0 + j] += __uint_as_float(v[j]);
                     }
@@ -262,33 +381,33 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     // ---- split-K reduction over the cluster, then the epilogue in the cluster's first CTA ----
     tc_fence_before_sync();
     __syncthreads();  // all roles done: the ring is free, every MMA has been drained
-    if (cs > 1) {
-        float* red = reinterpret_cast<float*>(smem);  // [BNR][128] partial sums (column-major: no bank conflicts)
-        if (is_drain) {
+    float* red = reinterpret_cast<float*>(smem);  // [BNR][RTC_RED_LD] sums, expert-major
+    if (is_drain && rank != 0) {  // the partials the first CTA will collect
 #pragma unroll
-            for (int j = 0; j < BNR; ++j) red[j * RTC_BM + q * 32 + lane] = sum[j];
-        }
+        for (int j = 0; j < BNR; ++j) red[j * RTC_RED_LD + q * 32 + lane] = sum[j];
+    }
+    if (cs > 1) {
         cluster_sync();
-        if (rank == 0 && is_drain) {
+        if (rank == 0 && is_drain) {  // peers' partials added in rank order: deterministic
             const uint32_t base = smem_u32(red);
             for (uint32_t r = 1; r < cs; ++r) {
                 const uint32_t peer = mapa_shared(base, r);
 #pragma unroll
                 for (int j = 0; j < BNR; ++j)
-                    sum[j] += ld_shared_cluster_f32(peer + (uint32_t)((j * RTC_BM + q * 32 + lane) * 4));
+                    sum[j] += ld_shared_cluster_f32(peer + (uint32_t)((j * RTC_RED_LD + q * 32 + lane) * 4));
             }
         }
         cluster_sync();  // no CTA leaves while the first one may still read its shared memory
         // (a CTA whose pipeline wait gave up has already set the device error word)
     }
-    if (rank == 0 && is_drain) {
-        bool ok = drain_ok && !*abort_flag;
-        if (ok) {
-            float* lrow = logits + (size_t)(valid ? row : 0) * E;
-            float tv[RTC_KMAX];
-            int te[RTC_KMAX];
+    if (rank == 0 && BNR <= 32 && fuse_topk && k <= RTC_KINS) {
+        if (is_drain && drain_ok && !*abort_flag) {
+            const int row = m0 + q * 32 + lane;
+            float* lrow = logits + (size_t)(row < T ? row : 0) * E;
+            float tv[RTC_KINS];
+            int te[RTC_KINS];
 #pragma unroll
-            for (int i = 0; i < RTC_KMAX; ++i) {
+            for (int i = 0; i < RTC_KINS; ++i) {
                 tv[i] = 0.f;
                 te[i] = INT_MAX;
             }
@@ -296,63 +415,57 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             for (int e = 0; e < BNR; ++e) {
                 if (e < E) {
                     sum[e] += bias ? __ldg(bias + e) : 0.f;
-                    if (valid) lrow[e] = sum[e];
-                    if (fuse_topk) {
-                        float cv = sum[e];
-                        int ce = e;
+                    if (row < T) lrow[e] = sum[e];
+                    float cv = sum[e];
+                    int ce = e;
 #pragma unroll
-                        for (int i = 0; i < RTC_KMAX; ++i) {
-                            if (te[i] == INT_MAX || cv > tv[i]) {
-                                const float tf = tv[i];
-                                const int ti = te[i];
-                                tv[i] = cv;
-                                te[i] = ce;
-                                cv = tf;
-                                ce = ti;
-                            }
+                    for (int i = 0; i < RTC_KINS; ++i) {
+                        if (te[i] == INT_MAX || cv > tv[i]) {
+                            const float tf = tv[i];
+                            const int ti = te[i];
+                            tv[i] = cv;
+                            te[i] = ce;
+                            cv = tf;
+                            ce = ti;
                         }
                     }
                 }
             }
-            if (fuse_topk && valid) {
-                float wv[RTC_KMAX];
-                float z = 0.f;
-                if (mode == MOE_ROUTE_SIGMOID_TOPK_NORM) {
+            if (row < T) {
+                float zall = 0.f;  // softmax over all E logits, relative to the largest (renormalising mode only)
+                if (mode == MOE_ROUTE_SOFTMAX_TOPK_RENORM) {
 #pragma unroll
-                    for (int j = 0; j < RTC_KMAX; ++j)
-                        if (j < k) {
-                            wv[j] = 1.f / (1.f + expf(-tv[j]));
-                            z += wv[j];
-                        }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < RTC_KMAX; ++j)
-                        if (j < k) {
-                            wv[j] = expf(tv[j] - tv[0]);
-                            z += wv[j];
-                        }
-                    if (mode == MOE_ROUTE_SOFTMAX_TOPK_RENORM) {
-                        // probabilities under the softmax over all E logits, renormalised over the selection
-                        float zall = 0.f;
-#pragma unroll
-                        for (int e = 0; e < BNR; ++e)
-                            if (e < E) zall += expf(sum[e] - tv[0]);
-                        float zp = 0.f;
-#pragma unroll
-                        for (int j = 0; j < RTC_KMAX; ++j)
-                            if (j < k) {
-                                wv[j] = wv[j] / zall;
-                                zp += wv[j];
-                            }
-                        z = zp;
-                    }
+                    for (int e = 0; e < BNR; ++e)
+                        if (e < E) zall += expf(sum[e] - tv[0]);
                 }
+                route_weights(tv, te, k, mode, zall, topk_idx + (size_t)row * k, topk_w + (size_t)row * k);
+            }
+        }
+    } else if (rank == 0) {
+        if (is_drain) {
 #pragma unroll
-                for (int j = 0; j < RTC_KMAX; ++j)
-                    if (j < k) {
-                        topk_idx[(size_t)row * k + j] = te[j];
-                        topk_w[(size_t)row * k + j] = wv[j] / z;
-                    }
+            for (int j = 0; j < BNR; ++j)
+                if (j < E) red[j * RTC_RED_LD + q * 32 + lane] = sum[j] + (bias ? __ldg(bias + j) : 0.f);
+        }
+        __syncthreads();
+        if (!*abort_flag) {
+            if (warp >= 4) {  // logits, row by row
+                for (int r = warp - 4; r < RTC_BM && m0 + r < T; r += RTC_THREADS / 32 - 4) {
+                    float* lrow = logits + (size_t)(m0 + r) * E;
+                    for (int e = lane; e < E; e += 32) lrow[e] = red[e * RTC_RED_LD + r];
+                }
+            } else if (fuse_topk && k <= RTC_KINS) {
+                const int r = threadIdx.x;  // one token per thread
+                if (m0 + r < T) route_token_insertion(red + r, E, k, mode, topk_idx + (size_t)(m0 + r) * k,
+                                                      topk_w + (size_t)(m0 + r) * k);
+            }
+            if (fuse_topk && k > RTC_KINS) {
+                __syncthreads();  // warps 4-9 join once the logits are out
+                for (int r = warp; r < RTC_BM && m0 + r < T; r += RTC_THREADS / 32) {
+                    const float* col = red + r;
+                    warp_route_select([=](int e) { return col[e * RTC_RED_LD]; }, E, k, mode,
+                                      topk_idx + (size_t)(m0 + r) * k, topk_w + (size_t)(m0 + r) * k);
+                }
             }
         }
     }

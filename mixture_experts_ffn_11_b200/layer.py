@@ -129,9 +129,9 @@ class MoEFFN:
 
     def kernel_launches(self, T: int) -> int:
         """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the
-        tensor-core path with fused top-k is taken (E <= 128, T >= 2048, k <= 8), else logits + top-k;
+        tensor-core path with fused top-k is taken (E <= 128, T >= 2048), else logits + top-k;
         permute 4; gate|up, down, combine 1 each; the shared expert 2 more."""
         if T <= 0:
             return 0
-        route = 1 if (self.E <= 128 and T >= 2048 and self.k <= 8) else 2
+        route = 1 if (self.E <= 128 and T >= 2048) else 2
         return route + 4 + 3 + (2 if self.shared_f else 0)

@@ -121,6 +121,9 @@ ROUTER_CASES = [
     (300, 7168, 256, 8, "sigmoid_topk_norm", True),
     (64, 2880, 32, 4, "topk_softmax", False),
     (1500, 2048, 384, 6, "topk_softmax", False),
+    # fused top-k beyond 8 on the tensor-core path, and k = E (every expert selected) with a split-K cluster
+    (2500, 1024, 128, 16, "softmax_topk_renorm", True),
+    (2300, 640, 17, 17, "sigmoid_topk_norm", False),
 ]
 
 
