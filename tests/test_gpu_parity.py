@@ -244,6 +244,8 @@ RAGGED = [
     ("pair_ragged", [0, 1, 255, 256, 257, 600, 0, 129], 256, 200),
     ("pair_down_240_wide", [300, 0, 700, 45], 480, 136),
     ("pair_one_expert", [0, 0, 2000, 0], 256, 256),
+    # last tiles of <= 128 rows run as M=128 pair MMAs: tails of exactly 128, 64, 65 and 1 rows, 240-wide down
+    ("pair_half_tails", [128, 384, 64, 65, 320, 0, 256, 257], 264, 136),
     # CTA pair with two accumulators (K >= 8192): 240-wide gate|up; 256-wide down
     ("wide_gateup_240", [300, 0, 700, 45], 8192, 240),
     ("wide_down_256", [400, 1, 129], 512, 8192),
