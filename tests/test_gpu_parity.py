@@ -194,6 +194,21 @@ def test_permute_edge_sizes():
     assert N.get_device_error() == 0
 
 
+def test_gather_row_widths():
+    """Row gather x_perm = x[perm_src] bit-exact over row widths from one 16-byte vector to 12296 elements,
+    including widths that are not a multiple of the 32 lanes x 16 bytes a warp moves per step."""
+    rng = np.random.default_rng(4)
+    T, E, k = 301, 5, 3
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    _, _, ps, _ = oracle.permute(idx, E)
+    for d in (8, 2880, 3072, 3080, 6144, 6152, 12288, 12296):
+        x_bits = synth.normal_bf16(5, 0, 0, T * d, 1.0).reshape(T, d)
+        _, out = _gpu_permute(x_bits, idx, E)
+        np.testing.assert_array_equal(out["perm_src"].cpu().numpy(), ps)
+        assert (bf16_bits_of(out["x_perm"]) == x_bits[ps]).all(), d
+    assert N.get_device_error() == 0
+
+
 # ---- expert GEMMs + combine on ragged groups ---------------------------------------------------------
 
 def _gpu_experts(x_bits, gu_bits, dn_bits, idx, w32, shared=None):
