@@ -36,7 +36,21 @@ L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu capture, keyed by the
 # kernel, the workload and a hash of the kernel's source files at capture time. A stale hash -> null.
-TRAFFIC = {}
+# Captured (one pass, full-size workload) with
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none
+#       -k regex:grouped_gemm -s 4 -c 4 --csv python bench.py --steps 3 --warmup 3 --settle-seconds 0
+#       --no-cpu-baseline --no-e2e --workload W
+# averaging the two launches of each GEMM (decode: the routed-expert launches, not the shared expert's).
+TRAFFIC = {
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "efb2e964ac9d632a"): 1260750208,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "efb2e964ac9d632a"): 709572736,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "efb2e964ac9d632a"): 2475728512,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "efb2e964ac9d632a"): 2274745856,
+    ("grouped_gemm_gateup", "zipf-128e", "efb2e964ac9d632a"): 1719376000,
+    ("grouped_gemm_down", "zipf-128e", "efb2e964ac9d632a"): 1080597760,
+    ("grouped_gemm_gateup", "decode-256e-shared", "efb2e964ac9d632a"): 12927184640,
+    ("grouped_gemm_down", "decode-256e-shared", "efb2e964ac9d632a"): 6465172480,
+}
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "sm100.cuh", "common.cuh", "moe.cu")]
 
