@@ -61,7 +61,11 @@ using Wide256GU = GemmWideShape<256, 4, true>;
 using Wide240GU = GemmWideShape<240, 4, true>;
 using Wide256DN = GemmWideShape<256, 4, false>;
 using Wide240DN = GemmWideShape<240, 4, false>;
-constexpr int kWideMinK = 8192;  // the wide tile's epilogue is not overlapped: it pays off on long K only
+// The wide tile's epilogue is not overlapped with the next tile's MMAs, so it pays off on long reductions only:
+// measured (interleaved A/B against the 256-wide pair tile) gate|up K=2880 -8%, K=2048 -23%, K=4096 (against two
+// K blocks per stage) -30%, K=14336 +10%; down K=768 -25%, K=2880 +4%, K=14336 +10%.
+constexpr int kWideMinK = 8192;      // gate|up
+constexpr int kWideMinKDown = 2048;  // down
 
 cudaError_t set_gemm_attributes() {
     const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
@@ -255,7 +259,7 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
 // Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs. Otherwise a single CTA
 // per tile, 256 wide unless that leaves SMs idle (e.g. one small group), then 64 wide.
 moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cudaStream_t stream) {
-    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2 && p.K >= kWideMinK) {
+    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2 && p.K >= (gateup ? kWideMinK : kWideMinKDown)) {
         // columns padded per tile: gate|up NH per tile, down 2*NH per tile; pick the width that pads less
         const long span = gateup ? 1 : 2;
         const long w256 = (long)(p.n_out + 256 * span - 1) / (256 * span) * (256 * span);

@@ -264,6 +264,7 @@ RAGGED = [
     # CTA pair with two accumulators (K >= 8192): 240-wide gate|up; 256-wide down
     ("wide_gateup_240", [300, 0, 700, 45], 8192, 240),
     ("wide_down_256", [400, 1, 129], 512, 8192),
+    ("wide_down_240_mid_k", [300, 0, 700, 45], 960, 2880),
     # CTA pair, two K blocks per ring stage (gate|up with K >= 4096), K tail inside the last stage
     ("pair_two_kblocks_per_stage", [0, 300, 1, 257], 4160, 136),
     # single-CTA kernel, 256 wide (many groups of a few rows) and 64 wide (one small group)
