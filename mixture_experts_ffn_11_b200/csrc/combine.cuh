@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
                                                       const float* __restrict__ topk_w,
                                                       const __nv_bfloat16* __restrict__ shared, int T, int d, int k,
                                                       int R, __nv_bfloat16* __restrict__ y) {
+    grid_dep_wait();
+    grid_dep_trigger();
     const int lane = threadIdx.x & 31;
     const int nvec = d / 8;
     const int nchunk = (nvec + CB_CHUNK_VEC - 1) / CB_CHUNK_VEC;

@@ -50,6 +50,14 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
     return true;
 }
 
+// Programmatic dependent launch. The library launches its kernels so that the next kernel in a stream may
+// start while this one finishes: grid_dep_wait() returns once every earlier kernel in the stream has completed
+// and its memory writes are visible (a no-op when the kernel was launched without the attribute). A kernel reads
+// and writes global memory only after it; what comes before is prologue (barrier setup, TMEM allocation, tensor
+// map prefetch). grid_dep_trigger() allows the next kernel's CTAs to be launched; they take SMs as they free up.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

@@ -94,6 +94,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
         tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
         tmem_relinquish_pair();
     }
+    grid_dep_wait();  // inputs below come from earlier kernels in the stream
+    grid_dep_trigger();
     for (int g = threadIdx.x; g <= G; g += GG_THREADS) {
         int v = args.group_offsets[g];
         if (v < 0 || v > args.M) {

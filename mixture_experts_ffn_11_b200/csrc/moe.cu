@@ -36,10 +36,29 @@ moe_status_t fail(moe_status_t st, const char* fmt, ...) {
     return st;
 }
 
-moe_status_t check_launch(const char* what) {
-    const cudaError_t e = cudaGetLastError();
+// launch_err: what the launch call returned (the error state is read as well)
+moe_status_t check_launch(const char* what, cudaError_t launch_err = cudaSuccess) {
+    const cudaError_t e = launch_err != cudaSuccess ? launch_err : cudaGetLastError();
     if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
     return MOE_OK;
+}
+
+// Every kernel is launched with programmatic stream serialization: the next kernel in the stream may be
+// launched before this one ends, runs its prologue, and waits in grid_dep_wait (common.cuh) for the data.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -222,8 +241,9 @@ moe_status_t launch_single(const GemmProblem& p, int sms, cudaStream_t stream) {
     const long upper = ((long)p.M / GG_BM + p.G) * (long)args.n_tiles;  // >= the real tile count
     const int grid = (int)(upper < sms ? upper : sms);
     const int streamed_once = (long)p.M <= (long)p.G * GG_BM ? 1 : 0;
-    grouped_gemm_kernel<BN, STAGES, GATEUP><<<grid, GG_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args, streamed_once);
-    return check_launch(GATEUP ? "grouped_gemm_gateup" : "grouped_gemm_down");
+    const cudaError_t e = launch_pdl(grouped_gemm_kernel<BN, STAGES, GATEUP>, dim3(grid), dim3(GG_THREADS),
+                                     S::SMEM_BYTES, stream, ta, tb, args, streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup" : "grouped_gemm_down", e);
 }
 
 template <int BN, int STAGES, bool GATEUP, int SUB = 1>
@@ -236,9 +256,9 @@ moe_status_t launch_pair(const GemmProblem& p, int sms, cudaStream_t stream) {
     const long upper = ((long)p.M / GP_BM + p.G) * (long)args.n_tiles;
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GP_BM ? 1 : 0;
-    grouped_gemm_pair_kernel<BN, STAGES, GATEUP, SUB><<<2 * clusters, GG_THREADS, S::SMEM_BYTES, stream>>>(
-        ta, tb, args, streamed_once);
-    return check_launch(GATEUP ? "grouped_gemm_gateup (pair)" : "grouped_gemm_down (pair)");
+    const cudaError_t e = launch_pdl(grouped_gemm_pair_kernel<BN, STAGES, GATEUP, SUB>, dim3(2 * clusters),
+                                     dim3(GG_THREADS), S::SMEM_BYTES, stream, ta, tb, args, streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup (pair)" : "grouped_gemm_down (pair)", e);
 }
 
 template <int NH, int STAGES, bool GATEUP>
@@ -251,9 +271,9 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
     const long upper = ((long)p.M / GP_BM + p.G) * (long)args.n_tiles;
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GP_BM ? 1 : 0;
-    grouped_gemm_wide_kernel<NH, STAGES, GATEUP><<<2 * clusters, GW_THREADS, S::SMEM_BYTES, stream>>>(ta, tb, args,
-                                                                                                      streamed_once);
-    return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)");
+    const cudaError_t e = launch_pdl(grouped_gemm_wide_kernel<NH, STAGES, GATEUP>, dim3(2 * clusters),
+                                     dim3(GW_THREADS), S::SMEM_BYTES, stream, ta, tb, args, streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)", e);
 }
 
 // Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs. Otherwise a single CTA
@@ -291,13 +311,15 @@ moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, cons
     cfg.blockDim = dim3(RTC_THREADS);
     cfg.dynamicSmemBytes = RouterTcShape<BNR>::SMEM_BYTES;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // as launch_pdl
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BNR>, tm, tw, bias, T, d, E, k, mode, fuse,
                                              logits, idx, w);
     if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "router_tc launch: %s", cudaGetErrorString(e));
@@ -419,17 +441,19 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
         int epb = E >= 2 * di.sms ? 4 : (E >= di.sms ? 2 : 1);
         while (epb > 1 && (size_t)epb * d * sizeof(float) > (size_t)kRouterSmallMaxSmem) --epb;
         const int grid = (E + epb - 1) / epb;
-        router_logits_small_kernel<<<grid, RS_THREADS, (size_t)epb * d * sizeof(float), stream>>>(
-            xb, w_router, bias, T, d, E, epb, logits_out);
-        if ((st = check_launch("router_logits_small")) != MOE_OK) return st;
+        const cudaError_t e = launch_pdl(router_logits_small_kernel, dim3(grid), dim3(RS_THREADS),
+                                         (size_t)epb * d * sizeof(float), stream, xb, w_router, bias, T, d, E, epb,
+                                         logits_out);
+        if ((st = check_launch("router_logits_small", e)) != MOE_OK) return st;
     } else {
         dim3 grid((T + RT_TOK - 1) / RT_TOK, (E + RT_EXP - 1) / RT_EXP);
-        router_logits_kernel<<<grid, RT_THREADS, 0, stream>>>(xb, w_router, bias, T, d, E, logits_out);
-        if ((st = check_launch("router_logits")) != MOE_OK) return st;
+        const cudaError_t e = launch_pdl(router_logits_kernel, dim3(grid), dim3(RT_THREADS), 0, stream, xb, w_router,
+                                         bias, T, d, E, logits_out);
+        if ((st = check_launch("router_logits", e)) != MOE_OK) return st;
     }
-    topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, stream>>>(logits_out, T, E, k, (int)mode,
-                                                                                  topk_idx, topk_w);
-    return check_launch("topk");
+    const cudaError_t e = launch_pdl(topk_kernel, dim3((T + TOPK_WARPS - 1) / TOPK_WARPS), dim3(TOPK_WARPS * 32), 0,
+                                     stream, logits_out, T, E, k, (int)mode, topk_idx, topk_w);
+    return check_launch("topk", e);
 }
 
 moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_route_mode_t mode,
@@ -442,9 +466,9 @@ moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
     if (T == 0) return MOE_OK;
-    topk_kernel<<<(T + TOPK_WARPS - 1) / TOPK_WARPS, TOPK_WARPS * 32, 0, stream>>>(logits, T, E, k, (int)mode,
-                                                                                  topk_idx, topk_w);
-    return check_launch("topk");
+    const cudaError_t e = launch_pdl(topk_kernel, dim3((T + TOPK_WARPS - 1) / TOPK_WARPS), dim3(TOPK_WARPS * 32), 0,
+                                     stream, logits, T, E, k, (int)mode, topk_idx, topk_w);
+    return check_launch("topk", e);
 }
 
 size_t moe_permute_workspace_size(int T, int E, int k) {
@@ -481,18 +505,19 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
     }
     int32_t* seg = reinterpret_cast<int32_t*>(ws);
     const int nseg = perm_num_segments(R);
-    permute_hist_kernel<<<nseg, PERM_THREADS, E * sizeof(int32_t), stream>>>(topk_idx, R, E, seg);
-    if ((st = check_launch("permute_hist")) != MOE_OK) return st;
-    permute_scan_kernel<<<1, 1024, 0, stream>>>(seg, nseg, E, expert_counts, expert_offsets);
-    if ((st = check_launch("permute_scan")) != MOE_OK) return st;
-    permute_scatter_kernel<<<nseg, PERM_THREADS, PERM_WARPS * E * sizeof(int32_t), stream>>>(topk_idx, R, E, k, seg,
-                                                                                            perm_src, inv_perm);
-    if ((st = check_launch("permute_scatter")) != MOE_OK) return st;
+    cudaError_t e = launch_pdl(permute_hist_kernel, dim3(nseg), dim3(PERM_THREADS), E * sizeof(int32_t), stream,
+                               topk_idx, R, E, seg);
+    if ((st = check_launch("permute_hist", e)) != MOE_OK) return st;
+    e = launch_pdl(permute_scan_kernel, dim3(1), dim3(1024), 0, stream, seg, nseg, E, expert_counts, expert_offsets);
+    if ((st = check_launch("permute_scan", e)) != MOE_OK) return st;
+    e = launch_pdl(permute_scatter_kernel, dim3(nseg), dim3(PERM_THREADS), PERM_WARPS * E * sizeof(int32_t), stream,
+                   topk_idx, R, E, k, seg, perm_src, inv_perm);
+    if ((st = check_launch("permute_scatter", e)) != MOE_OK) return st;
     if (x) {
         const int grid = grid_cap((R + 7) / 8, di.sms, 16);
-        gather_rows_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(x), perm_src, R, T, d,
-                                                     reinterpret_cast<__nv_bfloat16*>(x_perm));
-        if ((st = check_launch("gather_rows")) != MOE_OK) return st;
+        e = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, stream, reinterpret_cast<const __nv_bfloat16*>(x),
+                       perm_src, R, T, d, reinterpret_cast<__nv_bfloat16*>(x_perm));
+        if ((st = check_launch("gather_rows", e)) != MOE_OK) return st;
     }
     return MOE_OK;
 }
@@ -551,10 +576,11 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
     if (T == 0) return MOE_OK;
     const long items = (long)T * ((d / 8 + CB_CHUNK_VEC - 1) / CB_CHUNK_VEC);
     const int grid = grid_cap((items + 7) / 8, di.sms, 16);
-    combine_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const __nv_bfloat16*>(y_perm), inv_perm, topk_w,
-                                             reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
-                                             reinterpret_cast<__nv_bfloat16*>(y));
-    return check_launch("unpermute_combine");
+    const cudaError_t e = launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, stream,
+                                     reinterpret_cast<const __nv_bfloat16*>(y_perm), inv_perm, topk_w,
+                                     reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
+                                     reinterpret_cast<__nv_bfloat16*>(y));
+    return check_launch("unpermute_combine", e);
 }
 
 moe_status_t moe_get_device_error(unsigned int* out, cudaStream_t stream) {

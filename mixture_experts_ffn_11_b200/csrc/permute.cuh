@@ -24,6 +24,9 @@ __global__ void __launch_bounds__(PERM_THREADS) permute_hist_kernel(const int32_
                                                                     int32_t* __restrict__ seg_hist) {
     extern __shared__ int32_t sh[];  // [E]
     for (int e = threadIdx.x; e < E; e += PERM_THREADS) sh[e] = 0;
+    grid_dep_wait();
+    grid_dep_trigger();
+
     __syncthreads();
     const long base = (long)blockIdx.x * PERM_SEG;
     for (int i = threadIdx.x; i < PERM_SEG; i += PERM_THREADS) {
@@ -46,6 +49,8 @@ __global__ void __launch_bounds__(1024) permute_scan_kernel(int32_t* __restrict_
                                                             int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets) {
     __shared__ int32_t warp_tot[32];
+    grid_dep_wait();
+    grid_dep_trigger();
     const int e = threadIdx.x, lane = e & 31, w = e >> 5;
     int total = 0;
     if (e < E)
@@ -100,6 +105,9 @@ __global__ void __launch_bounds__(PERM_THREADS) permute_scatter_kernel(const int
     extern __shared__ int32_t wh[];  // [PERM_WARPS][E]: warp histograms, then warp running row cursors
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < PERM_WARPS * E; i += PERM_THREADS) wh[i] = 0;
+    grid_dep_wait();
+    grid_dep_trigger();
+
     __syncthreads();
     const long wbase = (long)blockIdx.x * PERM_SEG + (long)warp * PERM_PER_WARP;
     int32_t* my = wh + warp * E;
@@ -147,6 +155,8 @@ __global__ void __launch_bounds__(PERM_THREADS) permute_scatter_kernel(const int
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ x,
                                                           const int32_t* __restrict__ perm_src, int R, int T,
                                                           int d, __nv_bfloat16* __restrict__ x_perm) {
+    grid_dep_wait();
+    grid_dep_trigger();
     const int lane = threadIdx.x & 31;
     const int nvec = d / 8;
     const long nwarps = (long)gridDim.x * (blockDim.x / 32);

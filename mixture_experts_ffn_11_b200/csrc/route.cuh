@@ -18,6 +18,8 @@ __global__ void __launch_bounds__(RT_THREADS) router_logits_kernel(const __nv_bf
                                                                    int E, float* __restrict__ logits) {
     __shared__ __align__(16) float xs[RT_K][RT_TOK + 4];
     __shared__ __align__(16) float ws[RT_K][RT_EXP + 4];
+    grid_dep_wait();
+    grid_dep_trigger();
     const int t0 = blockIdx.x * RT_TOK, e0 = blockIdx.y * RT_EXP;
     const int tid = threadIdx.x;
     const int ty = tid / 8, tx = tid % 8;  // 16 x 8 threads, 4 tokens x 4 experts each
@@ -182,6 +184,8 @@ constexpr int TOPK_WARPS = 8;
 __global__ void __launch_bounds__(TOPK_WARPS * 32) topk_kernel(const float* __restrict__ logits, int T, int E,
                                                                  int k, int mode, int32_t* __restrict__ topk_idx,
                                                                  float* __restrict__ topk_w) {
+    grid_dep_wait();
+    grid_dep_trigger();
     const int t = blockIdx.x * TOPK_WARPS + (threadIdx.x >> 5);
     if (t >= T) return;
     const float* l = logits + (size_t)t * E;

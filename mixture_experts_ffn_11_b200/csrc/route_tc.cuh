@@ -212,6 +212,8 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_slot;
+    grid_dep_wait();  // x, W_r and the outputs' earlier readers: everything below follows earlier kernels
+    grid_dep_trigger();
     // drain warps (6-9): this thread's row of the tile and its running fp32 partial sums
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
     const bool is_drain = warp >= 6;
@@ -491,6 +493,8 @@ __global__ void __launch_bounds__(RS_THREADS) router_logits_small_kernel(const _
                                                                          int d, int E, int epb,
                                                                          float* __restrict__ logits) {
     extern __shared__ float wsm[];  // [epb][d]
+    grid_dep_wait();
+    grid_dep_trigger();
     const int e0 = blockIdx.x * epb;
     const int ne = min(epb, E - e0);
     {
