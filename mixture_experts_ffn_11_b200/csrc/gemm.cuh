@@ -48,6 +48,12 @@ struct GemmArgs {
     __nv_bfloat16* out;  // [M][n_out]
 };
 
+// silu(g) * u, silu(g) = g / (1 + e^-g), with the fast exponential and the fast divide: a few fp32 ulp, far
+// below the bf16 rounding of h, and fewer instructions on the epilogue warps, which share their SM sub-partitions
+// with the TMA and MMA issuing warps (measured: gate|up -2..4%). For g < -88, e^-g is past the divide's range and
+// silu(g) evaluates to 0 (its true magnitude is below 1e-36).
+__device__ __forceinline__ float swiglu(float g, float u) { return __fdividef(g, 1.f + __expf(-g)) * u; }
+
 // Epilogue store of one warp's 32 rows x 32 bf16 columns (thread = row, 16 packed words per thread).
 // A thread's own row is 64 contiguous bytes, but a warp-wide store of one 16-byte piece per row touches
 // 32 rows and only half of each 32-byte sector; L2 then has to fetch the rest of every sector from DRAM.
@@ -305,7 +311,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
                     for (int i = 0; i < 16; ++i) {
                         const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
                         const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
-                        pk[i] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+                        pk[i] = pack_bf16x2(swiglu(g0, u0), swiglu(g1, u1));
                     }
                 } else {
                     uint32_t v[32];

@@ -288,7 +288,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GW_THREADS, 1)
                     for (int i = 0; i < 16; ++i) {
                         const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
                         const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
-                        pk[i] = pack_bf16x2(g0 / (1.f + __expf(-g0)) * u0, g1 / (1.f + __expf(-g1)) * u1);
+                        pk[i] = pack_bf16x2(swiglu(g0, u0), swiglu(g1, u1));
                     }
                     int pc[4];
 #pragma unroll

@@ -362,6 +362,24 @@ def test_full_layer_matches_oracle(name):
     assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
 
 
+def test_layer_at_maximum_sizes():
+    """The API's largest routing sizes through the whole layer: E = 1024 experts, k = 32 per token (router on
+    CUDA cores + the stand-alone top-k, 1024-group permute and GEMMs), every token against the oracle."""
+    wl = synth.workload("tiny", T=300, d=128, f=64, E=1024, k=32, route="softmax_topk_renorm")
+    ref = oracle.LayerReference(wl)
+    inp = synth.device_inputs(wl)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"])
+    y = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
+    np.testing.assert_array_equal(layer.buf["counts"].cpu().numpy(), ref.counts)
+    ties = set(ref.near_ties(NEAR_TIE).tolist())
+    toks = np.array([t for t in range(wl.T) if t not in ties], dtype=np.int32)
+    assert len(toks) > wl.T // 2
+    assert (layer.buf["topk_idx"].cpu().numpy()[toks] == ref.idx[toks]).all()
+    check_close(bf16_to_host_f32(y)[toks], ref.outputs(toks), "E=1024, k=32")
+
+
 def test_layer_is_deterministic():
     wl = synth.workload("gpt-oss-20b-prefill", T=1024)
     inp = synth.device_inputs(wl)
