@@ -60,6 +60,25 @@ __device__ __forceinline__ float swiglu(float g, float u) { return __fdividef(g,
 // So the rows go through a 2 KB per-warp staging buffer (16-byte units XOR-swizzled by row, which keeps
 // both the write and the read at the minimum of four shared-memory wavefronts) and leave it as
 // 8 rows x 64 contiguous bytes per instruction: whole sectors, masked per row and column.
+// The same 32 x 32 block sent by one TMA store when it lies whole inside the rows and columns this tile owns
+// (no masking needed). The staging layout above is the TMA engine's 64-byte swizzle (the 16-byte unit of a
+// 64-byte row is XORed with row / 2), so the tensor map (box 32 x 32, SWIZZLE_64B) reads it as written; the
+// buffer must be 512-byte aligned. Lane 0 issues the store and commits it as a bulk group: the caller waits
+// (bulk_wait_group_read) before writing this buffer again.
+__device__ __forceinline__ void store_warp_block_tma(uint8_t* stage, const uint32_t (&pk)[16], int lane,
+                                                     const CUtensorMap* tm_out, int row_base, int col0) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+        *reinterpret_cast<uint4*>(stage + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4)) =
+            make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+    fence_proxy_async_smem();  // generic writes -> the TMA engine
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tm_out, stage, col0, row_base);
+        bulk_commit_group();
+    }
+}
+
 __device__ __forceinline__ void store_warp_rows_32cols(uint8_t* stage, const uint32_t (&pk)[16], int lane,
                                                        __nv_bfloat16* out, int ld_out, int row_base, int row_end,
                                                        int col0, int n_out, int cols_in_tile) {

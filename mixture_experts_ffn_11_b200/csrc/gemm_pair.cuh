@@ -41,10 +41,10 @@ struct GemmPairShape {
     static constexpr int OUT_COLS = GATEUP ? BN / 2 : BN;
     static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
     static constexpr int BAR_BYTES = 256;
-    static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;  // keeps what follows 128-B aligned
-    static constexpr int EPI_BYTES = 4 * 2048;  // per-epilogue-warp store staging
-    static_assert((STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES) % 128 == 0, "staging buffer alignment");
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES + EPI_BYTES;
+    static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;
+    static constexpr int EPI_BYTES = 4 * 2 * 2048;  // per epilogue warp, two store staging buffers
+    static_assert((STAGES * STAGE_BYTES) % 1024 == 0, "staging buffers (after the ring) stay 1024-byte aligned");
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + TABLE_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
 };
@@ -52,21 +52,22 @@ struct GemmPairShape {
 template <int BN, int STAGES, bool GATEUP, int SUB = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             const GemmArgs args, int weights_streamed_once) {
+                             const __grid_constant__ CUtensorMap tmO, const GemmArgs args, int weights_streamed_once) {
+    // tmO: the output [M][n_out], 32 x 32 boxes, 64-byte swizzle (TMA stores of whole epilogue blocks)
     using S = GemmPairShape<BN, STAGES, GATEUP, SUB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* stages = smem;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES);  // used in the leader
+    uint8_t* epi_stage = smem + STAGES * S::STAGE_BYTES;  // [4 warps][2][2048]
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * S::STAGE_BYTES + S::EPI_BYTES);  // leader
     uint64_t* empty_bar = full_bar + STAGES;
     uint64_t* tfull_bar = empty_bar + STAGES;
     uint64_t* tempty_bar = tfull_bar + 2;  // used in the leader
     uint64_t* final_bar = tempty_bar + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES);
+    int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * S::STAGE_BYTES + S::EPI_BYTES + S::BAR_BYTES);
     int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
-    uint8_t* epi_stage = smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES + S::TABLE_BYTES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -89,6 +90,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
+        tma_prefetch_desc(&tmO);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, S::TMEM_COLS);
@@ -249,18 +251,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
         int acc = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
+        uint32_t blocks = 0;  // output blocks this warp has staged (alternating buffers)
         for (int tile = cluster; tile < total; tile += n_clusters) {
             int g, nb, mb;
             locate(tile, g, nb, mb);
             const int row_end = s_off[g + 1];
             const int row_base = s_off[g] + mb * GP_BM + (int)rank * 128 + q * 32;  // row of lane 0
+            const bool rows_whole = row_base + 32 <= row_end;  // this warp's 32 rows all belong to the group
             if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
             const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const int col_base = nb * S::OUT_COLS;
-            uint8_t* my_stage = epi_stage + (warp - 2) * 2048;
 #pragma unroll 1
             for (int c0 = 0; c0 < S::OUT_COLS; c0 += 32) {
                 const int col0 = col_base + c0;
@@ -283,8 +286,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
                     for (int i = 0; i < 16; ++i)
                         pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                 }
-                store_warp_rows_32cols(my_stage, pk, lane, args.out, args.n_out, row_base, row_end, col0, args.n_out,
-                                       S::OUT_COLS - c0);
+                uint8_t* my_stage = epi_stage + ((warp - 2) * 2 + (int)(blocks & 1u)) * 2048;
+                ++blocks;
+                if (lane == 0) bulk_wait_group_read<1>();  // the TMA store that last read this buffer is done
+                __syncwarp();
+                if (rows_whole && S::OUT_COLS - c0 >= 32)
+                    store_warp_block_tma(my_stage, pk, lane, &tmO, row_base, col0);
+                else {
+                    store_warp_rows_32cols(my_stage, pk, lane, args.out, args.n_out, row_base, row_end, col0,
+                                           args.n_out, S::OUT_COLS - c0);
+                    if (lane == 0) bulk_commit_group();  // an empty group: one group per staged block
+                }
             }
             tc_fence_before_sync();
             __syncwarp();
@@ -292,6 +304,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GG_THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait_all();  // the output stores have landed before the CTA leaves
+        __syncwarp();
     }
 
     tc_fence_before_sync();

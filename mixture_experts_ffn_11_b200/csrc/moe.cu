@@ -218,6 +218,14 @@ moe_status_t make_gemm_maps(const GemmProblem& p, bool gateup, int b_rows, CUten
     return make_tmap(tb, p.w, 3, bdims, bstr, bbox);
 }
 
+// Output [M][n_out] for TMA stores of 32 x 32 epilogue blocks (64-byte swizzle, as the staging layout).
+moe_status_t make_out_map(const GemmProblem& p, CUtensorMap* to) {
+    const cuuint64_t dims[2] = {(cuuint64_t)p.n_out, (cuuint64_t)p.M};
+    const cuuint64_t strides[1] = {(cuuint64_t)p.n_out * 2};
+    const cuuint32_t box[2] = {32, 32};
+    return make_tmap(to, p.out, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 GemmArgs gemm_args(const GemmProblem& p, int out_cols) {
     GemmArgs args;
     args.group_offsets = p.offsets;
@@ -249,15 +257,16 @@ moe_status_t launch_single(const GemmProblem& p, int sms, cudaStream_t stream) {
 template <int BN, int STAGES, bool GATEUP, int SUB = 1>
 moe_status_t launch_pair(const GemmProblem& p, int sms, cudaStream_t stream) {
     using S = GemmPairShape<BN, STAGES, GATEUP, SUB>;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to;
     moe_status_t st = make_gemm_maps(p, GATEUP, BN / 2, &ta, &tb);
+    if (st == MOE_OK) st = make_out_map(p, &to);
     if (st != MOE_OK) return st;
     const GemmArgs args = gemm_args(p, S::OUT_COLS);
     const long upper = ((long)p.M / GP_BM + p.G) * (long)args.n_tiles;
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GP_BM ? 1 : 0;
     const cudaError_t e = launch_pdl(grouped_gemm_pair_kernel<BN, STAGES, GATEUP, SUB>, dim3(2 * clusters),
-                                     dim3(GG_THREADS), S::SMEM_BYTES, stream, ta, tb, args, streamed_once);
+                                     dim3(GG_THREADS), S::SMEM_BYTES, stream, ta, tb, to, args, streamed_once);
     return check_launch(GATEUP ? "grouped_gemm_gateup (pair)" : "grouped_gemm_down (pair)", e);
 }
 
