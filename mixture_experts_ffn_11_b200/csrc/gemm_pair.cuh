@@ -26,7 +26,7 @@ namespace moe {
 constexpr int GP_BM = 256;  // rows per pair tile (128 per CTA)
 
 // SUB: 64-wide K blocks per ring stage. Two halve the barrier round trips per FLOP (8 MMAs per stage); measured
-// faster on long reductions (gate|up with K >= 4096).
+// faster for gate|up from K = 2048 on.
 template <int BN, int STAGES, bool GATEUP, int SUB = 1>
 struct GemmPairShape {
     static_assert(BN % 32 == 0 || (!GATEUP && BN % 16 == 0), "tile width");
