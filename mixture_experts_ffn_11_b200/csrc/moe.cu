@@ -313,9 +313,9 @@ moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cud
 }
 
 template <int BNR>
-moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, const float* bias, int T, int d, int E,
-                              int k, int mode, int fuse, float* logits, int32_t* idx, float* w, int tiles, int cs,
-                              cudaStream_t stream) {
+moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, const float* w_router, const float* bias,
+                              int T, int d, int E, int k, int mode, int fuse, float* logits, int32_t* idx, float* w,
+                              int tiles, int cs, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tiles * cs));
     cfg.blockDim = dim3(RTC_THREADS);
@@ -330,7 +330,7 @@ moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, cons
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BNR>, tm, tw, bias, T, d, E, k, mode, fuse,
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BNR>, tm, tw, w_router, bias, T, d, E, k, mode, fuse,
                                              logits, idx, w);
     if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "router_tc launch: %s", cudaGetErrorString(e));
     return MOE_OK;
@@ -432,16 +432,16 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
         else if (tiles * 2 <= di.sms && kblocks >= 4)
             cs = 2;
         if (E <= 16)
-            st = launch_router_tc<16>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
+            st = launch_router_tc<16>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
                                       stream);
         else if (E <= 32)
-            st = launch_router_tc<32>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
+            st = launch_router_tc<32>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
                                       stream);
         else if (E <= 64)
-            st = launch_router_tc<64>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
+            st = launch_router_tc<64>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
                                       stream);
         else
-            st = launch_router_tc<128>(tm, tw, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles,
+            st = launch_router_tc<128>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles,
                                        cs, stream);
         if (st != MOE_OK) return st;
         if ((st = check_launch("router_tc")) != MOE_OK) return st;

@@ -48,7 +48,10 @@ template <int BNR>
 struct RouterTcShape {
     static_assert(BNR % 16 == 0 && BNR >= 16 && BNR <= 128, "UMMA N (and the drain's register budget)");
     static constexpr int A_BYTES = RTC_BM * RTC_BK * 2;  // x tile, bf16
-    static constexpr int W_BYTES = BNR * RTC_BK * 4;     // W_r block, fp32 as loaded
+    // BNR = 128: the converters read their W_r values from global memory (L2; loads issued before the stage
+    // wait) instead of a TMA-staged fp32 block, which leaves room for a 3-stage ring (64 KB stages, not 96 KB)
+    static constexpr bool W_DIRECT = BNR > 64;
+    static constexpr int W_BYTES = W_DIRECT ? 0 : BNR * RTC_BK * 4;  // W_r block, fp32 as loaded
     static constexpr int P_BYTES = BNR * RTC_BK * 2;     // one bf16 piece
     static constexpr int STAGE_BYTES = A_BYTES + W_BYTES + 3 * P_BYTES;
     static_assert(STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
@@ -162,10 +165,30 @@ __device__ __forceinline__ void route_token_insertion(const float* col, int E, i
     route_weights(tv, te, k, mode, zall, idx_row, w_row);
 }
 
+// Converter thread ct's share of one 64-wide K block of W_r, read from global memory: item it is expert row
+// (ct + 128*it) / 8, columns col0 + 8*((ct + 128*it) % 8) .. +8; rows past E and columns past d are zeros (d is a
+// multiple of 8, so a chunk is all in or all out).
+template <int ITEMS, int N>
+__device__ __forceinline__ void router_load_w_chunks(float4 (&wv)[N][2], const float* __restrict__ w_router, int ct,
+                                                     int col0, int E, int d) {
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+        const int item = ct + 128 * it;
+        const int r = item >> 3, col = col0 + (item & 7) * 8;
+        if (r < E && col < d) {
+            const float4* src = reinterpret_cast<const float4*>(w_router + (size_t)r * d + col);
+            wv[it][0] = __ldg(src);
+            wv[it][1] = __ldg(src + 1);
+        } else {
+            wv[it][0] = wv[it][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
+}
+
 template <int BNR>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     const float* __restrict__ bias, int T, int d, int E, int k, int mode, int fuse_topk,
+                     const float* __restrict__ w_router, const float* __restrict__ bias, int T, int d, int E, int k, int mode, int fuse_topk,
                      float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
     using S = RouterTcShape<BNR>;
     constexpr int STAGES = S::STAGES;
@@ -214,13 +237,13 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     grid_dep_wait();  // x, W_r and the outputs' earlier readers: everything below follows earlier kernels
     grid_dep_trigger();
-    // drain warps (6-9): this thread's row of the tile and its running fp32 partial sums
+    // drain warps (6-9): this thread's row of the tile
     const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
     const bool is_drain = warp >= 6;
-    float sum[BNR];
-#pragma unroll
-    for (int j = 0; j < BNR; ++j) sum[j] = 0.f;
     bool drain_ok = false;
+    // [BNR][RTC_RED_LD] row sums, expert-major, over the ring once the last K block is drained (the ring is then
+    // idle: every TMA copy, conversion and MMA of this CTA has completed)
+    float* red = reinterpret_cast<float*>(smem);
 
     if (warp == 0) {
         // ---------------- TMA: x tile ----------------
@@ -238,7 +261,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
                 uint8_t* sa = smem + stage * S::STAGE_BYTES;
                 mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES + S::W_BYTES);
                 tma_load_2d(sa, &tmX, &full_bar[stage], (kb0 + kb) * RTC_BK, m0, pol);
-                tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], (kb0 + kb) * RTC_BK, 0, pol_w);
+                if (!S::W_DIRECT) tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], (kb0 + kb) * RTC_BK, 0, pol_w);
             }
             ++issued;
             if (++stage == STAGES) {
@@ -296,13 +319,15 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (lane == 0) umma_commit(final_bar);
         __syncwarp();
     } else if (warp < 6) {
-        // ---------------- converters: staged W_r block (fp32) -> hi/mid/lo bf16 pieces ----------------
+        // ---------------- converters: W_r block (fp32) -> hi/mid/lo bf16 pieces ----------------
         const int ct = threadIdx.x - 64;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         constexpr int ITEMS = BNR * (RTC_BK / 8) / 128;  // 16-byte output chunks per thread per piece
         for (int kb = 0; kb < KB; ++kb) {
+            float4 wv[S::W_DIRECT ? ITEMS : 1][2];  // W_DIRECT: this K block's chunks, in flight during the wait
+            if constexpr (S::W_DIRECT) router_load_w_chunks<ITEMS>(wv, w_router, ct, (kb0 + kb) * RTC_BK, E, d);
             if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
@@ -312,8 +337,15 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             for (int it = 0; it < ITEMS; ++it) {
                 const int item = ct + 128 * it;
                 const int r = item >> 3, c = item & 7;  // expert row, 8-element chunk of the 64-wide block
-                const float4* src = reinterpret_cast<const float4*>(wbase + r * (RTC_BK * 4) + c * 32);
-                const float4 v0 = src[0], v1 = src[1];  // rows past E and columns past d arrive as zeros
+                float4 v0, v1;  // rows past E and columns past d are zeros
+                if constexpr (S::W_DIRECT) {
+                    v0 = wv[it][0];
+                    v1 = wv[it][1];
+                } else {
+                    const float4* src = reinterpret_cast<const float4*>(wbase + r * (RTC_BK * 4) + c * 32);
+                    v0 = src[0];
+                    v1 = src[1];
+                }
                 const float w8[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
                 uint32_t hi[4], mi[4], lo[4];
 #pragma unroll
@@ -333,6 +365,9 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
     } else {
         // ---------------- drain (warps 6-9) ----------------
         const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+        float sum[BNR];  // this thread's row: running fp32 sums of the K-block partials
+#pragma unroll
+        for (int j = 0; j < BNR; ++j) sum[j] = 0.f;
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
             const int acc = kb % NBUF;
@@ -378,26 +413,30 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             if (lane == 0) mbar_arrive(&tempty_bar[acc]);
         }
         drain_ok = ok;
+        if (ok) {
+#pragma unroll
+            for (int j = 0; j < BNR; ++j) red[j * RTC_RED_LD + q * 32 + lane] = sum[j];
+        }
     }
 
     // ---- split-K reduction over the cluster, then the epilogue in the cluster's first CTA ----
     tc_fence_before_sync();
-    __syncthreads();  // all roles done: the ring is free, every MMA has been drained
-    float* red = reinterpret_cast<float*>(smem);  // [BNR][RTC_RED_LD] sums, expert-major
-    if (is_drain && rank != 0) {  // the partials the first CTA will collect
-#pragma unroll
-        for (int j = 0; j < BNR; ++j) red[j * RTC_RED_LD + q * 32 + lane] = sum[j];
-    }
+    __syncthreads();  // all roles done, every partial sum is in red
     if (cs > 1) {
         cluster_sync();
-        if (rank == 0 && is_drain) {  // peers' partials added in rank order: deterministic
+        if (rank == 0 && is_drain) {  // own partial, then the peers' in rank order: deterministic
             const uint32_t base = smem_u32(red);
+            float v[BNR];
+#pragma unroll
+            for (int j = 0; j < BNR; ++j) v[j] = red[j * RTC_RED_LD + q * 32 + lane];
             for (uint32_t r = 1; r < cs; ++r) {
                 const uint32_t peer = mapa_shared(base, r);
 #pragma unroll
-                for (int j = 0; j < BNR; ++j)
-                    sum[j] += ld_shared_cluster_f32(peer + (uint32_t)((j * RTC_RED_LD + q * 32 + lane) * 4));
+                for (int j = 0; j < BNR; ++j)  // independent remote loads, all in flight
+                    v[j] += ld_shared_cluster_f32(peer + (uint32_t)((j * RTC_RED_LD + q * 32 + lane) * 4));
             }
+#pragma unroll
+            for (int j = 0; j < BNR; ++j) red[j * RTC_RED_LD + q * 32 + lane] = v[j];
         }
         cluster_sync();  // no CTA leaves while the first one may still read its shared memory
         // (a CTA whose pipeline wait gave up has already set the device error word)
@@ -406,6 +445,9 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (is_drain && drain_ok && !*abort_flag) {
             const int row = m0 + q * 32 + lane;
             float* lrow = logits + (size_t)(row < T ? row : 0) * E;
+            float sum[BNR];
+#pragma unroll
+            for (int j = 0; j < BNR; ++j) sum[j] = red[j * RTC_RED_LD + q * 32 + lane];
             float tv[RTC_KINS];
             int te[RTC_KINS];
 #pragma unroll
@@ -447,7 +489,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (is_drain) {
 #pragma unroll
             for (int j = 0; j < BNR; ++j)
-                if (j < E) red[j * RTC_RED_LD + q * 32 + lane] = sum[j] + (bias ? __ldg(bias + j) : 0.f);
+                if (j < E) red[j * RTC_RED_LD + q * 32 + lane] += bias ? __ldg(bias + j) : 0.f;
         }
         __syncthreads();
         if (!*abort_flag) {
