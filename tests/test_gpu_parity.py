@@ -261,6 +261,9 @@ RAGGED = [
     ("pair_one_expert", [0, 0, 2000, 0], 256, 256),
     # last tiles of <= 128 rows run as M=128 pair MMAs: tails of exactly 128, 64, 65 and 1 rows, 240-wide down
     ("pair_half_tails", [128, 384, 64, 65, 320, 0, 256, 257], 264, 136),
+    # gate|up whose last N tile is part-filled (f = 360, f = 120 < 128): one and two K blocks per stage
+    ("pair_partial_h_tile", [300, 0, 700, 45], 264, 360),
+    ("pair_partial_h_tile_two_kblocks", [129, 400, 260], 2112, 120),
     # CTA pair with two accumulators (K >= 8192): 240-wide gate|up; 256-wide down
     ("wide_gateup_240", [300, 0, 700, 45], 8192, 240),
     ("wide_down_256", [400, 1, 129], 512, 8192),
