@@ -60,6 +60,11 @@ typedef enum {
     MOE_ERR_DEVICE = 5       /* returned by moe_get_device_error() when the error word was set */
 } moe_status_t;
 
+/* Empty problems: a call with T = 0 (router, top-k, permute, combine) or
+ * M = 0 (grouped GEMMs) launches nothing and returns MOE_OK once its sizes
+ * check out; pointers to arrays that are then empty may be NULL. moe_permute
+ * still writes its [E] counts and [E+1] offsets (all zero). */
+
 /* Bits of the device error word. */
 #define MOE_DEVERR_WAIT_TIMEOUT 0x1u  /* a pipeline wait in a GEMM gave up after its time limit */
 #define MOE_DEVERR_EXPERT_RANGE 0x2u  /* an expert id outside [0, E) reached moe_permute */

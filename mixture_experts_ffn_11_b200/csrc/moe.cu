@@ -336,9 +336,10 @@ moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, cons
     return MOE_OK;
 }
 
+// With M = 0 the activation and output arrays are empty and their pointers may be null.
 moe_status_t check_gemm_args(const void* a, const void* w, const int32_t* offsets, int G, int M, int d, int f,
                              const void* out) {
-    if (!a || !w || !offsets || !out) return fail(MOE_ERR_INVALID_ARG, "null pointer argument");
+    if (!w || !offsets || (M > 0 && (!a || !out))) return fail(MOE_ERR_INVALID_ARG, "null pointer argument");
     if (!aligned16(a) || !aligned16(w) || !aligned16(out))
         return fail(MOE_ERR_INVALID_ARG, "activation, weight and output pointers must be 16-byte aligned");
     if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return fail(MOE_ERR_INVALID_ARG, "offsets misaligned");
@@ -402,11 +403,11 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     if (mode < MOE_ROUTE_TOPK_SOFTMAX || mode > MOE_ROUTE_SIGMOID_TOPK_NORM)
         return fail(MOE_ERR_INVALID_ARG, "unknown routing mode %d", (int)mode);
     if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (T == 0) return MOE_OK;  // nothing to route (the empty arrays' pointers may be null)
     if (!x || !w_router || !logits_out || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(x) || !aligned16(w_router)) return fail(MOE_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
-    if (T == 0) return MOE_OK;
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     if (E <= 128 && T >= kRouterTcMinT) {
         // tensor cores, W_r split into three bf16 pieces; top-k fused (any k <= 32)
@@ -472,10 +473,10 @@ moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_
     if (st != MOE_OK) return st;
     if (mode < MOE_ROUTE_TOPK_SOFTMAX || mode > MOE_ROUTE_SIGMOID_TOPK_NORM)
         return fail(MOE_ERR_INVALID_ARG, "unknown routing mode %d", (int)mode);
+    if (T == 0) return MOE_OK;
     if (!logits || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "null pointer");
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
-    if (T == 0) return MOE_OK;
     const cudaError_t e = launch_pdl(topk_kernel, dim3((T + TOPK_WARPS - 1) / TOPK_WARPS), dim3(TOPK_WARPS * 32), 0,
                                      stream, logits, T, E, k, (int)mode, topk_idx, topk_w);
     return check_launch("topk", e);
@@ -492,8 +493,16 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
                          moe_bf16_t* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream) {
     moe_status_t st = check_route_sizes(T, E, k);
     if (st != MOE_OK) return st;
-    if (!topk_idx || !expert_counts || !expert_offsets || !perm_src || !inv_perm)
-        return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!expert_counts || !expert_offsets) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (T == 0) {  // no assignments: counts and offsets all zero (the empty arrays' pointers may be null)
+        DeviceInfo di;
+        if ((st = device_info(di)) != MOE_OK) return st;
+        cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), stream);
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+        return MOE_OK;
+    }
+    if (!topk_idx || !perm_src || !inv_perm) return fail(MOE_ERR_INVALID_ARG, "null pointer");
     if ((x == nullptr) != (x_perm == nullptr)) return fail(MOE_ERR_INVALID_ARG, "x and x_perm: give both or neither");
     if (x) {
         if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
@@ -507,12 +516,6 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
     const int R = T * k;
-    if (R == 0) {  // no assignments: counts are zero, offsets all zero
-        cudaError_t e = cudaMemsetAsync(expert_counts, 0, sizeof(int32_t) * E, stream);
-        if (e == cudaSuccess) e = cudaMemsetAsync(expert_offsets, 0, sizeof(int32_t) * (E + 1), stream);
-        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
-        return MOE_OK;
-    }
     int32_t* seg = reinterpret_cast<int32_t*>(ws);
     const int nseg = perm_num_segments(R);
     cudaError_t e = launch_pdl(permute_hist_kernel, dim3(nseg), dim3(PERM_THREADS), E * sizeof(int32_t), stream,
@@ -576,6 +579,7 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
                                    cudaStream_t stream) {
     if (T < 0 || k < 1 || k > 32) return fail(MOE_ERR_INVALID_ARG, "T=%d, k=%d (need T >= 0, 1 <= k <= 32)", T, k);
     if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (T == 0) return MOE_OK;  // nothing to combine (the empty arrays' pointers may be null)
     if (!y_perm || !inv_perm || !topk_w || !y) return fail(MOE_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(y_perm) || !aligned16(y) || (shared && !aligned16(shared)))
         return fail(MOE_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
@@ -583,7 +587,6 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
     DeviceInfo di;
     moe_status_t st = device_info(di);
     if (st != MOE_OK) return st;
-    if (T == 0) return MOE_OK;
     const long items = (long)T * ((d / 8 + CB_CHUNK_VEC - 1) / CB_CHUNK_VEC);
     const int grid = grid_cap((items + 7) / 8, di.sms, 16);
     const cudaError_t e = launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, stream,

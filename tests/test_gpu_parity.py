@@ -383,6 +383,41 @@ def test_layer_at_maximum_sizes():
     check_close(bf16_to_host_f32(y)[toks], ref.outputs(toks), "E=1024, k=32")
 
 
+@pytest.mark.parametrize("T,d,f,E,k,route", [
+    (5, 8, 8, 3, 3, "softmax_topk_renorm"),  # smallest dims the API takes, k = E (every expert selected)
+    (1, 64, 16, 1, 1, "topk_softmax"),       # one token, one expert: a dense SwiGLU with weight 1
+    (7, 16, 24, 4, 2, "sigmoid_topk_norm"),  # d, f not multiples of 16
+])
+def test_layer_degenerate_shapes(T, d, f, E, k, route):
+    wl = synth.workload("tiny", T=T, d=d, f=f, E=E, k=k, route=route)
+    ref = oracle.LayerReference(wl)
+    inp = synth.device_inputs(wl)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"])
+    y = layer(inp["x"]).clone()
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
+    ties = set(ref.near_ties(NEAR_TIE).tolist())
+    toks = np.array([t for t in range(T) if t not in ties], dtype=np.int32)
+    assert (layer.buf["topk_idx"].cpu().numpy()[toks] == ref.idx[toks]).all()
+    check_close(bf16_to_host_f32(y)[toks], ref.outputs(toks), f"T={T} d={d} f={f} E={E} k={k}")
+
+
+def test_layer_empty_batch():
+    """T = 0: every call returns at once and the output is empty (no launch reads an empty buffer)."""
+    wl = synth.workload("tiny")
+    inp = synth.device_inputs(wl)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"])
+    y = layer(inp["x"][:0].contiguous())
+    torch.cuda.synchronize()
+    assert tuple(y.shape) == (0, wl.d)
+    assert layer.kernel_launches(0) == 0
+    assert N.get_device_error() == 0
+    # and a normal batch afterwards still matches the first call of the same inputs
+    a = layer(inp["x"]).clone()
+    b = layer(inp["x"]).clone()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_layer_is_deterministic():
     wl = synth.workload("gpt-oss-20b-prefill", T=1024)
     inp = synth.device_inputs(wl)
