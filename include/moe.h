@@ -101,6 +101,30 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
                             int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx, float* topk_w,
                             cudaStream_t stream);
 
+/* The router's fp32 weights as three bf16 pieces, written once and then
+ * reused by moe_route_topk_split: w = hi + mid + lo with hi = w truncated to
+ * bf16, mid = (w - hi) truncated, lo = bf16(w - hi - mid) rounded to nearest
+ * (the tensor-core router multiplies x by the three pieces, carrying ~24
+ * bits of w). Router weights do not change between forward calls, so the
+ * split belongs with loading them (the blog post converts checkpoint
+ * tensors into the layout its kernels want at load time: "Dynamic Weight
+ * Loading with WeightConverter").
+ *   w_router  [E][d] fp32
+ *   w_pieces  [3][E][d] bf16, written: plane 0 hi, 1 mid, 2 lo
+ * Limits: 1 <= E <= 1024, d >= 8 a multiple of 8. */
+moe_status_t moe_router_split_weights(const float* w_router, int E, int d, moe_bf16_t* w_pieces,
+                                      cudaStream_t stream);
+
+/* moe_route_topk with the pieces written by moe_router_split_weights for
+ * this w_router: the same results, bit for bit, without re-splitting W_r in
+ * every call (the tensor-core router loads the pieces by TMA). w_router is
+ * still read where the router runs on CUDA cores (T < 2048 or E > 128).
+ * Arguments and limits otherwise as moe_route_topk; w_pieces must not be
+ * NULL. */
+moe_status_t moe_route_topk_split(const moe_bf16_t* x, const float* w_router, const moe_bf16_t* w_pieces,
+                                  const float* bias, int T, int d, int E, int k, moe_route_mode_t mode,
+                                  float* logits_out, int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
 /* Top-k selection and routing weights from given fp32 logits [T][E] (bias, if
  * any, already included). Same outputs and limits as moe_route_topk. */
 moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_route_mode_t mode,

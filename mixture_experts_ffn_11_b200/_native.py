@@ -22,7 +22,7 @@ DEVERR = {0x1: "wait timeout", 0x2: "expert id out of range", 0x4: "group offset
 ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm": 2}
 
 # every entry point of include/moe.h
-EXPORTS = ("moe_route_topk", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
+EXPORTS = ("moe_route_topk", "moe_router_split_weights", "moe_route_topk_split", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
            "moe_permute_static_ws",
            "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_unpermute_combine", "moe_get_device_error",
            "moe_last_error_string")
@@ -42,6 +42,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
     sig = {
         "moe_route_topk": [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp],
+        "moe_router_split_weights": [vp, ci, ci, vp, vp],
+        "moe_route_topk_split": [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp],
         "moe_topk_from_logits": [vp, ci, ci, ci, ci, vp, vp, vp],
         "moe_permute_workspace_size": [ci, ci, ci],
         "moe_permute": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, sz, vp],
@@ -103,6 +105,31 @@ def route_topk(x, w_router, bias, k, mode, logits, topk_idx, topk_w, stream=None
     _need(topk_w, torch.float32, (T, k), "topk_w")
     _check(_lib.moe_route_topk(_p(x), _p(w_router), _p(bias), T, d, E, k, ROUTE_MODES[mode], _p(logits),
                                _p(topk_idx), _p(topk_w), _stream(stream)), "moe_route_topk")
+
+
+def router_split_weights(w_router, w_pieces, stream=None):
+    """w_pieces [3, E, d] bf16 <- the hi / mid / lo split of w_router [E, d] fp32 (once per weight update)."""
+    E, d = w_router.shape
+    _need(w_router, torch.float32, (E, d), "w_router")
+    _need(w_pieces, torch.bfloat16, (3, E, d), "w_pieces")
+    _check(_lib.moe_router_split_weights(_p(w_router), E, d, _p(w_pieces), _stream(stream)),
+           "moe_router_split_weights")
+
+
+def route_topk_split(x, w_router, w_pieces, bias, k, mode, logits, topk_idx, topk_w, stream=None):
+    """route_topk with the pieces written by router_split_weights for this w_router."""
+    T, d = x.shape
+    E = w_router.shape[0]
+    _need(x, torch.bfloat16, (T, d), "x")
+    _need(w_router, torch.float32, (E, d), "w_router")
+    _need(w_pieces, torch.bfloat16, (3, E, d), "w_pieces")
+    if bias is not None:
+        _need(bias, torch.float32, (E,), "bias")
+    _need(logits, torch.float32, (T, E), "logits")
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    _check(_lib.moe_route_topk_split(_p(x), _p(w_router), _p(w_pieces), _p(bias), T, d, E, k, ROUTE_MODES[mode],
+                                     _p(logits), _p(topk_idx), _p(topk_w), _stream(stream)), "moe_route_topk_split")
 
 
 def topk_from_logits(logits, k, mode, topk_idx, topk_w, stream=None):

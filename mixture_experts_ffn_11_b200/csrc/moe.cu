@@ -110,8 +110,12 @@ constexpr int kRouterTcMinT = 2048;               // token count from which the 
 
 template <int BNR>
 cudaError_t set_router_tc_attr() {
-    return cudaFuncSetAttribute(router_tc_kernel<BNR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                RouterTcShape<BNR>::SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BNR, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         RouterTcShape<BNR, false>::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(router_tc_kernel<BNR, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 RouterTcShape<BNR, true>::SMEM_BYTES);
+    return e;
 }
 
 cudaError_t set_router_attributes() {
@@ -312,14 +316,15 @@ moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cud
     return gateup ? launch_single<64, 8, true>(p, sms, stream) : launch_single<64, 8, false>(p, sms, stream);
 }
 
-template <int BNR>
-moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, const float* w_router, const float* bias,
-                              int T, int d, int E, int k, int mode, int fuse, float* logits, int32_t* idx, float* w,
-                              int tiles, int cs, cudaStream_t stream) {
+template <int BNR, bool PRESPLIT>
+moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, const CUtensorMap& tp,
+                              const float* w_router, const float* bias, int T, int d, int E, int k, int mode,
+                              int fuse, float* logits, int32_t* idx, float* w, int tiles, int cs,
+                              cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(tiles * cs));
     cfg.blockDim = dim3(RTC_THREADS);
-    cfg.dynamicSmemBytes = RouterTcShape<BNR>::SMEM_BYTES;
+    cfg.dynamicSmemBytes = RouterTcShape<BNR, PRESPLIT>::SMEM_BYTES;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -330,8 +335,8 @@ moe_status_t launch_router_tc(const CUtensorMap& tm, const CUtensorMap& tw, cons
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BNR>, tm, tw, w_router, bias, T, d, E, k, mode, fuse,
-                                             logits, idx, w);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, router_tc_kernel<BNR, PRESPLIT>, tm, tw, tp, w_router, bias, T, d,
+                                             E, k, mode, fuse, logits, idx, w);
     if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "router_tc launch: %s", cudaGetErrorString(e));
     return MOE_OK;
 }
@@ -395,9 +400,35 @@ moe_status_t static_ws_address(void** out) {
 
 extern "C" {
 
-moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const float* bias, int T, int d, int E,
-                            int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx, float* topk_w,
-                            cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+template <bool PRESPLIT>
+moe_status_t launch_router_tc_bnr(int bnr, const CUtensorMap& tm, const CUtensorMap& tw, const CUtensorMap& tp,
+                                  const float* w_router, const float* bias, int T, int d, int E, int k, int mode,
+                                  int fuse, float* logits, int32_t* idx, float* w, int tiles, int cs,
+                                  cudaStream_t stream) {
+    switch (bnr) {
+        case 16:
+            return launch_router_tc<16, PRESPLIT>(tm, tw, tp, w_router, bias, T, d, E, k, mode, fuse, logits, idx, w,
+                                                  tiles, cs, stream);
+        case 32:
+            return launch_router_tc<32, PRESPLIT>(tm, tw, tp, w_router, bias, T, d, E, k, mode, fuse, logits, idx, w,
+                                                  tiles, cs, stream);
+        case 64:
+            return launch_router_tc<64, PRESPLIT>(tm, tw, tp, w_router, bias, T, d, E, k, mode, fuse, logits, idx, w,
+                                                  tiles, cs, stream);
+        default:
+            return launch_router_tc<128, PRESPLIT>(tm, tw, tp, w_router, bias, T, d, E, k, mode, fuse, logits, idx,
+                                                   w, tiles, cs, stream);
+    }
+}
+
+// moe_route_topk and moe_route_topk_split; w_pieces (nullable): the [3][E][d] bf16 split of w_router
+moe_status_t route_impl(const moe_bf16_t* x, const float* w_router, const moe_bf16_t* w_pieces, const float* bias,
+                        int T, int d, int E, int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx,
+                        float* topk_w, cudaStream_t stream) {
     moe_status_t st = check_route_sizes(T, E, k);
     if (st != MOE_OK) return st;
     if (mode < MOE_ROUTE_TOPK_SOFTMAX || mode > MOE_ROUTE_SIGMOID_TOPK_NORM)
@@ -405,13 +436,14 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
     if (T == 0) return MOE_OK;  // nothing to route (the empty arrays' pointers may be null)
     if (!x || !w_router || !logits_out || !topk_idx || !topk_w) return fail(MOE_ERR_INVALID_ARG, "null pointer");
-    if (!aligned16(x) || !aligned16(w_router)) return fail(MOE_ERR_INVALID_ARG, "x / w_router not 16-byte aligned");
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_pieces))
+        return fail(MOE_ERR_INVALID_ARG, "x / w_router / w_pieces not 16-byte aligned");
     DeviceInfo di;
     if ((st = device_info(di)) != MOE_OK) return st;
     const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
     if (E <= 128 && T >= kRouterTcMinT) {
-        // tensor cores, W_r split into three bf16 pieces; top-k fused (any k <= 32)
-        CUtensorMap tm, tw;
+        // tensor cores, W_r as three bf16 pieces (split here, or given); top-k fused (any k <= 32)
+        CUtensorMap tm, tw, tp;
         const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)T};
         const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
         const cuuint32_t box[2] = {RTC_BK, RTC_BM};
@@ -423,6 +455,14 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
         if ((st = make_tmap(&tw, w_router, 2, wdims, wstrides, wbox, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                             CU_TENSOR_MAP_SWIZZLE_NONE)) != MOE_OK)
             return st;
+        if (w_pieces) {  // [3][E][d] bf16: one box brings a K block of all three pieces
+            const cuuint64_t pdims[3] = {(cuuint64_t)d, (cuuint64_t)E, 3};
+            const cuuint64_t pstrides[2] = {(cuuint64_t)d * 2, (cuuint64_t)E * d * 2};
+            const cuuint32_t pbox[3] = {RTC_BK, (cuuint32_t)bnr, 3};
+            if ((st = make_tmap(&tp, w_pieces, 3, pdims, pstrides, pbox)) != MOE_OK) return st;
+        } else {
+            tp = tw;  // unused
+        }
         const int fuse = k <= RTC_KMAX ? 1 : 0;
         const int tiles = (T + RTC_BM - 1) / RTC_BM;
         const int kblocks = (d + RTC_BK - 1) / RTC_BK;
@@ -432,18 +472,10 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
             cs = 4;
         else if (tiles * 2 <= di.sms && kblocks >= 4)
             cs = 2;
-        if (E <= 16)
-            st = launch_router_tc<16>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
-                                      stream);
-        else if (E <= 32)
-            st = launch_router_tc<32>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
-                                      stream);
-        else if (E <= 64)
-            st = launch_router_tc<64>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles, cs,
-                                      stream);
-        else
-            st = launch_router_tc<128>(tm, tw, w_router, bias, T, d, E, k, (int)mode, fuse, logits_out, topk_idx, topk_w, tiles,
-                                       cs, stream);
+        st = w_pieces ? launch_router_tc_bnr<true>(bnr, tm, tw, tp, w_router, bias, T, d, E, k, (int)mode, fuse,
+                                                   logits_out, topk_idx, topk_w, tiles, cs, stream)
+                      : launch_router_tc_bnr<false>(bnr, tm, tw, tp, w_router, bias, T, d, E, k, (int)mode, fuse,
+                                                    logits_out, topk_idx, topk_w, tiles, cs, stream);
         if (st != MOE_OK) return st;
         if ((st = check_launch("router_tc")) != MOE_OK) return st;
         if (fuse) return MOE_OK;
@@ -465,6 +497,41 @@ moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const fl
     const cudaError_t e = launch_pdl(topk_kernel, dim3((T + TOPK_WARPS - 1) / TOPK_WARPS), dim3(TOPK_WARPS * 32), 0,
                                      stream, logits_out, T, E, k, (int)mode, topk_idx, topk_w);
     return check_launch("topk", e);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const float* bias, int T, int d, int E,
+                            int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx, float* topk_w,
+                            cudaStream_t stream) {
+    return route_impl(x, w_router, nullptr, bias, T, d, E, k, mode, logits_out, topk_idx, topk_w, stream);
+}
+
+moe_status_t moe_router_split_weights(const float* w_router, int E, int d, moe_bf16_t* w_pieces,
+                                      cudaStream_t stream) {
+    if (E < 1 || E > 1024) return fail(MOE_ERR_INVALID_ARG, "E=%d outside [1, 1024]", E);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (!w_router || !w_pieces) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(w_router) || !aligned16(w_pieces))
+        return fail(MOE_ERR_INVALID_ARG, "w_router / w_pieces not 16-byte aligned");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const long pairs = (long)E * d / 2;
+    uint32_t* base = reinterpret_cast<uint32_t*>(w_pieces);
+    const int grid = grid_cap((pairs + 255) / 256, di.sms, 8);
+    const cudaError_t e = launch_pdl(router_split_kernel, dim3(grid), dim3(256), 0, stream, w_router, pairs, base,
+                                     base + pairs, base + 2 * pairs);
+    return check_launch("router_split", e);
+}
+
+moe_status_t moe_route_topk_split(const moe_bf16_t* x, const float* w_router, const moe_bf16_t* w_pieces,
+                                  const float* bias, int T, int d, int E, int k, moe_route_mode_t mode,
+                                  float* logits_out, int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+    if (!w_pieces) return fail(MOE_ERR_INVALID_ARG, "w_pieces is required (moe_route_topk takes none)");
+    return route_impl(x, w_router, w_pieces, bias, T, d, E, k, mode, logits_out, topk_idx, topk_w, stream);
 }
 
 moe_status_t moe_topk_from_logits(const float* logits, int T, int E, int k, moe_route_mode_t mode,

@@ -44,14 +44,16 @@ namespace moe {
 constexpr int RTC_BM = 128, RTC_BK = 64, RTC_THREADS = 320, RTC_KMAX = 32, RTC_KINS = 8;
 constexpr int RTC_RED_LD = RTC_BM + 1;  // row stride of the [expert][token] sums in shared memory (odd: no bank conflicts)
 
-template <int BNR>
+// PRESPLIT: the three bf16 pieces of W_r were written once by router_split_kernel ([3][E][d], as the weights do
+// not change between calls) and arrive with the x tile by TMA; the converter warps then have nothing to do.
+template <int BNR, bool PRESPLIT = false>
 struct RouterTcShape {
     static_assert(BNR % 16 == 0 && BNR >= 16 && BNR <= 128, "UMMA N (and the drain's register budget)");
     static constexpr int A_BYTES = RTC_BM * RTC_BK * 2;  // x tile, bf16
     // BNR = 128: the converters read their W_r values from global memory (L2; loads issued before the stage
     // wait) instead of a TMA-staged fp32 block, which leaves room for a 3-stage ring (64 KB stages, not 96 KB)
-    static constexpr bool W_DIRECT = BNR > 64;
-    static constexpr int W_BYTES = W_DIRECT ? 0 : BNR * RTC_BK * 4;  // W_r block, fp32 as loaded
+    static constexpr bool W_DIRECT = BNR > 64 && !PRESPLIT;
+    static constexpr int W_BYTES = (W_DIRECT || PRESPLIT) ? 0 : BNR * RTC_BK * 4;  // W_r block, fp32 as loaded
     static constexpr int P_BYTES = BNR * RTC_BK * 2;     // one bf16 piece
     static constexpr int STAGE_BYTES = A_BYTES + W_BYTES + 3 * P_BYTES;
     static_assert(STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
@@ -185,12 +187,14 @@ __device__ __forceinline__ void router_load_w_chunks(float4 (&wv)[N][2], const f
     }
 }
 
-template <int BNR>
+template <int BNR, bool PRESPLIT = false>
 __global__ void __launch_bounds__(RTC_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                     const float* __restrict__ w_router, const float* __restrict__ bias, int T, int d, int E, int k, int mode, int fuse_topk,
+                     const __grid_constant__ CUtensorMap tmP, const float* __restrict__ w_router,
+                     const float* __restrict__ bias, int T, int d, int E, int k, int mode, int fuse_topk,
                      float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-    using S = RouterTcShape<BNR>;
+    using S = RouterTcShape<BNR, PRESPLIT>;
+    // tmP (PRESPLIT): the pieces [3][E][d] bf16, boxes of 64 x BNR x 3 (all three pieces of a K block at once)
     constexpr int STAGES = S::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -225,7 +229,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
-        tma_prefetch_desc(&tmW);
+        tma_prefetch_desc(PRESPLIT ? &tmP : &tmW);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -259,9 +263,12 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             if (!ok) break;
             if (lane == 0) {
                 uint8_t* sa = smem + stage * S::STAGE_BYTES;
-                mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES + S::W_BYTES);
+                mbar_arrive_expect_tx(&full_bar[stage], S::A_BYTES + (PRESPLIT ? 3 * S::P_BYTES : S::W_BYTES));
                 tma_load_2d(sa, &tmX, &full_bar[stage], (kb0 + kb) * RTC_BK, m0, pol);
-                if (!S::W_DIRECT) tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], (kb0 + kb) * RTC_BK, 0, pol_w);
+                if (PRESPLIT)  // hi, mid, lo land as the three consecutive piece blocks the MMA reads
+                    tma_load_3d(sa + S::A_BYTES, &tmP, &full_bar[stage], (kb0 + kb) * RTC_BK, 0, 0, pol_w);
+                else if (!S::W_DIRECT)
+                    tma_load_2d(sa + S::A_BYTES, &tmW, &full_bar[stage], (kb0 + kb) * RTC_BK, 0, pol_w);
             }
             ++issued;
             if (++stage == STAGES) {
@@ -284,7 +291,7 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
             if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], ((kb / NBUF) & 1) ^ 1u, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            if (lane == 0) ok = mbar_wait_bounded(&conv_bar[stage], phase, abort_flag) &&
+            if (lane == 0) ok = (PRESPLIT || mbar_wait_bounded(&conv_bar[stage], phase, abort_flag)) &&
                                 mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
@@ -319,13 +326,13 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (lane == 0) umma_commit(final_bar);
         __syncwarp();
     } else if (warp < 6) {
-        // ---------------- converters: W_r block (fp32) -> hi/mid/lo bf16 pieces ----------------
+        // ---------------- converters: W_r block (fp32) -> hi/mid/lo bf16 pieces (idle if PRESPLIT) ----------------
         const int ct = threadIdx.x - 64;  // 0..127
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         constexpr int ITEMS = BNR * (RTC_BK / 8) / 128;  // 16-byte output chunks per thread per piece
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < (PRESPLIT ? 0 : KB); ++kb) {
             float4 wv[S::W_DIRECT ? ITEMS : 1][2];  // W_DIRECT: this K block's chunks, in flight during the wait
             if constexpr (S::W_DIRECT) router_load_w_chunks<ITEMS>(wv, w_router, ct, (kb0 + kb) * RTC_BK, E, d);
             if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);
@@ -519,6 +526,23 @@ __global__ void __launch_bounds__(RTC_THREADS, 1)
         if (lane == 0) mbar_wait_drain(final_bar, 0);
         __syncwarp();
         tmem_dealloc(tmem_base, S::TMEM_COLS);
+    }
+}
+
+// The three bf16 pieces of W_r ([E][d] fp32 -> hi, mid, lo planes of [E][d] bf16, split3_pair on each pair of
+// weights): written once, read by router_tc_kernel<.., true> on every call.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ w, long n_pairs,
+                                                           uint32_t* __restrict__ hi, uint32_t* __restrict__ mid,
+                                                           uint32_t* __restrict__ lo) {
+    grid_dep_wait();
+    grid_dep_trigger();
+    for (long i = (long)blockIdx.x * 256 + threadIdx.x; i < n_pairs; i += (long)gridDim.x * 256) {
+        const float2 v = reinterpret_cast<const float2*>(w)[i];
+        uint32_t h, m, l;
+        split3_pair(v.x, v.y, h, m, l);
+        hi[i] = h;
+        mid[i] = m;
+        lo[i] = l;
     }
 }
 

@@ -37,9 +37,19 @@ class MoEFFN:
         self.device = w_gateup.device
         self._T = None
         self.buf = {}
+        # the tensor-core router (E <= 128) reads W_r as three bf16 pieces: split once here, not in every call
+        self.w_pieces = None
+        if self.E <= 128:
+            self.w_pieces = torch.empty(3, self.E, self.d, dtype=torch.bfloat16, device=self.device)
+            self.refresh_router()
         # the shared expert depends only on x: it runs on a side stream, beside routing and grouping (which
         # leave most SMs free), and the routed GEMMs wait for it
         self._side = torch.cuda.Stream(self.device) if self.shared_f else None
+
+    def refresh_router(self):
+        """Re-split the router weights; call after changing w_router in place."""
+        if self.w_pieces is not None:
+            N.router_split_weights(self.w_router, self.w_pieces)
 
     def buffers(self, T: int) -> dict:
         """Allocate (once per T) every intermediate the layer writes."""
@@ -105,7 +115,11 @@ class MoEFFN:
                 timing["shared"][1].record(side)
             shared = b["shared"]
         mark("route", True)
-        N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"], s)
+        if self.w_pieces is not None:
+            N.route_topk_split(x, self.w_router, self.w_pieces, self.bias, self.k, self.route, b["logits"],
+                               b["topk_idx"], b["topk_w"], s)
+        else:
+            N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"], s)
         mark("route", False)
         mark("permute", True)
         N.permute(x, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], b["x_perm"],

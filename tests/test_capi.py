@@ -59,6 +59,9 @@ def test_invalid_arguments_rejected_before_any_launch(native):
     assert lib.moe_grouped_gemm_down(16, 16, 16, 4096, 8, 8, 8, 16, null) == native.MOE_ERR_INVALID_ARG
     # k > 32 in combine
     assert lib.moe_unpermute_combine(16, 16, 16, null, 4, 8, 33, 16, null) == native.MOE_ERR_INVALID_ARG
+    # split router: no pieces; E out of range for the split
+    assert lib.moe_route_topk_split(16, 16, null, null, 4, 8, 8, 2, 0, 16, 16, 16, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_router_split_weights(16, 0, 8, 16, null) == native.MOE_ERR_INVALID_ARG
     # missing workspace
     st = lib.moe_permute(null, 16, 64, 0, 8, 2, 16, 16, 16, 16, null, null, 0, null)
     assert st == native.MOE_ERR_WORKSPACE

@@ -147,6 +147,46 @@ def test_router_paths_match_oracle(T, d, E, k, mode, with_bias):
     np.testing.assert_allclose(w.cpu().numpy()[keep], w_ref[keep], rtol=2e-5, atol=2e-6)
 
 
+def test_router_split_weights_pieces():
+    """hi + mid + lo reproduces W_r to the split's bound: hi is W_r truncated to bf16, mid the truncated rest,
+    lo the rounded remainder, so |W_r - (hi + mid + lo)| <= 2^-24 |W_r| (and hi, mid exact prefixes)."""
+    E, d = 100, 520
+    wr = synth.normal_f32(7, 1, 0, E * d, 0.02).reshape(E, d)
+    wr[0, :4] = [0.0, -0.0, 1e-30, -3.5]
+    wt = torch.from_numpy(wr).cuda()
+    pieces = torch.empty(3, E, d, dtype=torch.bfloat16, device="cuda")
+    N.router_split_weights(wt, pieces)
+    pc = pieces.float().cpu().numpy().astype(np.float64)
+    w64 = wr.astype(np.float64)
+    assert (np.abs(w64 - pc.sum(0)) <= 2.0 ** -24 * np.abs(w64)).all()
+    hi_bits = wr.view(np.uint32) & np.uint32(0xFFFF0000)
+    assert (pc[0] == hi_bits.view(np.float32)).all()  # hi = truncation of W_r to its top 16 bits
+
+
+@pytest.mark.parametrize("T,d,E,k,mode,with_bias", [c for c in ROUTER_CASES if c[0] >= 2048 and c[2] <= 128] +
+                         [(300, 7168, 64, 8, "sigmoid_topk_norm", True)])
+def test_route_topk_split_is_bit_identical(T, d, E, k, mode, with_bias):
+    """The pre-split router gives the same logits, ids and weights as the one that splits W_r itself."""
+    x = to_dev_bf16(synth.normal_bf16(8, 0, 0, T * d, 1.0).reshape(T, d))
+    wr = torch.from_numpy(synth.normal_f32(8, 1, 0, E * d, 0.02).reshape(E, d)).cuda()
+    bias = torch.from_numpy(synth.normal_f32(8, 4, 0, E, 1.0)).cuda() if with_bias else None
+    pieces = torch.empty(3, E, d, dtype=torch.bfloat16, device="cuda")
+    N.router_split_weights(wr, pieces)
+    outs = []
+    for split in (False, True):
+        lg = torch.empty(T, E, device="cuda")
+        idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, k, device="cuda")
+        if split:
+            N.route_topk_split(x, wr, pieces, bias, k, mode, lg, idx, w)
+        else:
+            N.route_topk(x, wr, bias, k, mode, lg, idx, w)
+        outs.append((lg, idx, w))
+    assert N.get_device_error() == 0
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.int32), b.view(torch.int32))
+
+
 # ---- permutation -----------------------------------------------------------------------------------
 
 def _gpu_permute(x_bits, idx_np, E):
