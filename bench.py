@@ -42,14 +42,14 @@ L2_FLUSH_BYTES = 256 << 20
 #       --no-cpu-baseline --no-e2e --workload W
 # averaging the two launches of each GEMM (decode: the routed-expert launches, not the shared expert's).
 TRAFFIC = {
-    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "f91a357509acda65"): 1249761536,
-    ("grouped_gemm_down", "gpt-oss-20b-prefill", "f91a357509acda65"): 714729600,
-    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "f91a357509acda65"): 2475303168,
-    ("grouped_gemm_down", "mixtral-8x7b-prefill", "f91a357509acda65"): 2166406400,
-    ("grouped_gemm_gateup", "zipf-128e", "f91a357509acda65"): 1602022400,
-    ("grouped_gemm_down", "zipf-128e", "f91a357509acda65"): 1079367808,
-    ("grouped_gemm_gateup", "decode-256e-shared", "f91a357509acda65"): 12927863296,
-    ("grouped_gemm_down", "decode-256e-shared", "f91a357509acda65"): 6464820480,
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "dbe1869900003c2d"): 1248037760,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "dbe1869900003c2d"): 713720448,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "dbe1869900003c2d"): 2475335040,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "dbe1869900003c2d"): 3088177664,
+    ("grouped_gemm_gateup", "zipf-128e", "dbe1869900003c2d"): 1631391488,
+    ("grouped_gemm_down", "zipf-128e", "dbe1869900003c2d"): 1081674880,
+    ("grouped_gemm_gateup", "decode-256e-shared", "dbe1869900003c2d"): 12926854144,
+    ("grouped_gemm_down", "decode-256e-shared", "dbe1869900003c2d"): 6464814848,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "sm100.cuh", "common.cuh", "moe.cu")]
