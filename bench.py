@@ -35,30 +35,36 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu capture, keyed by the
-# kernel, the workload and a hash of the kernel's source files at capture time. A stale hash -> null.
+# kernel, the workload and a hash of the GEMM sources (comments stripped) at capture time. A stale hash -> null.
 # Captured (one pass, full-size workload) with
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none
 #       -k regex:grouped_gemm -s 4 -c 4 --csv python bench.py --steps 3 --warmup 3 --settle-seconds 0
 #       --no-cpu-baseline --no-e2e --workload W
 # averaging the two launches of each GEMM (decode: the routed-expert launches, not the shared expert's).
 TRAFFIC = {
-    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "dbe1869900003c2d"): 1248037760,
-    ("grouped_gemm_down", "gpt-oss-20b-prefill", "dbe1869900003c2d"): 713720448,
-    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "dbe1869900003c2d"): 2475335040,
-    ("grouped_gemm_down", "mixtral-8x7b-prefill", "dbe1869900003c2d"): 3088177664,
-    ("grouped_gemm_gateup", "zipf-128e", "dbe1869900003c2d"): 1631391488,
-    ("grouped_gemm_down", "zipf-128e", "dbe1869900003c2d"): 1081674880,
-    ("grouped_gemm_gateup", "decode-256e-shared", "dbe1869900003c2d"): 12926854144,
-    ("grouped_gemm_down", "decode-256e-shared", "dbe1869900003c2d"): 6464814848,
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "fe180d49317877c2"): 1248037760,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "fe180d49317877c2"): 713720448,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "fe180d49317877c2"): 2475335040,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "fe180d49317877c2"): 3088177664,
+    ("grouped_gemm_gateup", "zipf-128e", "fe180d49317877c2"): 1631391488,
+    ("grouped_gemm_down", "zipf-128e", "fe180d49317877c2"): 1081674880,
+    ("grouped_gemm_gateup", "decode-256e-shared", "fe180d49317877c2"): 12926854144,
+    ("grouped_gemm_down", "decode-256e-shared", "fe180d49317877c2"): 6464814848,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "sm100.cuh", "common.cuh", "moe.cu")]
 
 
 def kernel_source_hash() -> str:
+    """Hash of the GEMM sources with comments and blank lines removed (a comment edit keeps the figures)."""
+    import re
+
     h = hashlib.sha256()
     for p in KERNEL_SOURCES:
-        h.update(open(os.path.join(ROOT, p), "rb").read())
+        src = open(os.path.join(ROOT, p)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        lines = (re.sub(r"//.*$", "", ln).rstrip() for ln in src.splitlines())
+        h.update("\n".join(ln for ln in lines if ln).encode())
     return h.hexdigest()[:16]
 
 

@@ -6,8 +6,8 @@
 // tile, and each barrier round trip of the shared-memory ring covers 8 MMAs instead of 4. The price: the two
 // accumulators fill TMEM (2*NH <= 512 columns), so the epilogue of a tile cannot overlap the next tile's
 // mainloop; it is spread over 8 warps to keep it short. Measured on B200: faster than the double-buffered pair
-// tile on long reductions (K >= 8192, e.g. a 14336-wide down projection), slower on shorter ones, which is
-// how the host chooses.
+// tile on long reductions, slower on short ones, which is how the host chooses (gate|up from K = 8192, the
+// down projection from K = 2048).
 //
 // Column mapping. Each CTA's B buffer holds NH rows; MMA a (a = 0, 1) reads rows [a*NH/2, (a+1)*NH/2) of
 // both CTAs' buffers (the leader's first, then the peer's), so accumulator a, column c = h*NH/2 + cc

@@ -1,10 +1,11 @@
 // Router on the tensor cores, for large token counts, with top-k fused into the epilogue.
 //
 // logits[t][e] = sum_i x[t][i] * W_r[e][i] + bias[e] with x bf16 and W_r fp32. The fp32 weights are split
-// on the fly into three bf16 pieces, W_r = hi + mid + lo (hi = bf16(w), mid = bf16(w - hi),
-// lo = bf16(w - hi - mid); both differences are exact in fp32), so the product is three bf16 MMAs:
-// x*hi + x*mid + x*lo, which carries ~24 bits of W_r (relative error ~2^-27 per weight). bf16*bf16
-// products are exact in fp32.
+// into three bf16 pieces, W_r = hi + mid + lo (hi = w truncated to bf16, mid = (w - hi) truncated, lo =
+// bf16(w - hi - mid); the differences are exact, and for normal weights so is the sum: 24 significand bits
+// are 8 + 8 + 8), so the product is three bf16 MMAs x*hi + x*mid + x*lo. bf16*bf16 products are exact in
+// fp32. The pieces are either written once beforehand (PRESPLIT, router_split_kernel) and loaded by TMA, or
+// made in every call by converter warps.
 //
 // The tensor core's fp32 accumulator drops low-order bits when it adds (a bias toward zero that grows
 // with the number of accumulation steps and the size of the running sum; on a 3 x 4096-long reduction it
@@ -21,12 +22,14 @@
 // few 128-token tiles, so without the split most SMs would idle.
 //
 // Per CTA (320 threads):
-//   warp 0     TMA of the x tile [128 x 64] bf16 and of the W_r block [BNR x 64] fp32 per K block into a
-//              STAGES-deep ring (the W_r block lands unswizzled, 256 bytes per expert row)
-//   warp 1     TMEM allocation; one lane issues 3 x 4 tcgen05.mma (M=128, N=BNR, K=16) per K block into
-//              accumulator buffer (kb % NBUF), starting it afresh
-//   warps 2-5  convert the staged W_r block into the three bf16 pieces, stored in the 128-byte-swizzled
-//              K-major layout the TMA engine writes, then signal conv[stage]
+//   warp 0     TMA of the x tile [128 x 64] bf16 per K block into a STAGES-deep ring, with (PRESPLIT) the
+//              three pieces [3 x BNR x 64] bf16 in one box, or (BNR <= 64) the W_r block [BNR x 64] fp32
+//              (unswizzled, 256 bytes per expert row)
+//   warp 1     TMEM allocation; one lane issues the K block's tcgen05.mma (M=128; 4 of N = 3*BNR, or 3 x 4 of
+//              N = BNR) into accumulator buffer (kb % NBUF), starting it afresh
+//   warps 2-5  (not PRESPLIT) convert the W_r block (staged, or read from L2 when BNR = 128) into the three
+//              bf16 pieces, stored in the 128-byte-swizzled K-major layout the TMA engine writes, then signal
+//              conv[stage]
 //   warps 6-9  drain: add each finished block partial of their 32 TMEM lanes into registers
 // Epilogue (the cluster's first CTA), top-k by insertion into a sorted list of 8 (descending, equal logits keep
 // the lower expert id first), then the routing weights of the mode:

@@ -111,8 +111,8 @@ def test_topk_ties_and_modes_small():
 
 
 ROUTER_CASES = [
-    # T, d, E, k, mode, with bias: both sides of the tensor-core threshold (T >= 2048), fused (k <= 8) and
-    # unfused top-k, padded expert counts, every mode
+    # T, d, E, k, mode, with bias: both sides of the tensor-core threshold (T >= 2048, E <= 128; top-k fused
+    # there, a separate kernel otherwise), padded expert counts, every mode
     (2047, 256, 8, 2, "softmax_topk_renorm", False),
     (2048, 256, 8, 2, "softmax_topk_renorm", True),
     (2100, 520, 100, 8, "topk_softmax", True),
@@ -304,11 +304,11 @@ RAGGED = [
     # gate|up whose last N tile is part-filled (f = 360, f = 120 < 128): one and two K blocks per stage
     ("pair_partial_h_tile", [300, 0, 700, 45], 264, 360),
     ("pair_partial_h_tile_two_kblocks", [129, 400, 260], 2112, 120),
-    # CTA pair with two accumulators (K >= 8192): 240-wide gate|up; 256-wide down
+    # CTA pair with two accumulators (gate|up K >= 8192, down K >= 2048): 240-wide gate|up; 256-wide down
     ("wide_gateup_240", [300, 0, 700, 45], 8192, 240),
     ("wide_down_256", [400, 1, 129], 512, 8192),
     ("wide_down_240_mid_k", [300, 0, 700, 45], 960, 2880),
-    # CTA pair, two K blocks per ring stage (gate|up with K >= 4096), K tail inside the last stage
+    # CTA pair, two K blocks per ring stage (gate|up with K >= 2048), K tail inside the last stage
     ("pair_two_kblocks_per_stage", [0, 300, 1, 257], 4160, 136),
     # single-CTA kernel, 256 wide (many groups of a few rows) and 64 wide (one small group)
     ("single_wide", [2] * 160, 64, 256),
