@@ -268,7 +268,7 @@ class OracleStep:
 
 
 def calibrate_sample(step: OracleStep, seconds: float, cap: int) -> int:
-    n0 = min(8, cap)
+    n0 = min(64, cap)  # enough tokens to keep every host thread busy, so the per-token time is representative
     step.prepare(n0)
     t = time.perf_counter()
     step.run(n0)
