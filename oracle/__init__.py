@@ -17,6 +17,14 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   moe_tokens     pinned: dense-masked brute force over all experts (numpy fp64);
                  E=1,k=1 dense SwiGLU (torch fp64); identical experts; linearity
                  in W_down; hand-derived golden values
+  e2m1_value     pinned: the FP4 E2M1 value table of the OCP MX v1.0 specification
+                 (tests/golden/e2m1_values.txt)
+  mxfp4_quantize pinned: round-trip of encodable blocks; the tie and clamp cases of
+                 round-to-nearest-even on the E2M1 grid; closed-form scales (zero,
+                 subnormal and power-of-two blocks); the error bound of the grid;
+                 a hand-packed word of the documented nibble layout
+  mxfp4_dequantize pinned: inverse of the above on every code and scale range;
+                 numpy decode of the documented layout
 """
 from __future__ import annotations
 
@@ -53,6 +61,12 @@ def load(path: str | None = None):
     lib.oracle_permute.restype = ci
     lib.oracle_moe_tokens.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, ci, vp, ci, vp, ci]
     lib.oracle_moe_tokens.restype = ci
+    lib.oracle_e2m1_value.argtypes = [ci]
+    lib.oracle_e2m1_value.restype = ctypes.c_double
+    lib.oracle_mxfp4_quantize.argtypes = [vp, ci, ci, ci, vp, vp]
+    lib.oracle_mxfp4_quantize.restype = ci
+    lib.oracle_mxfp4_dequantize.argtypes = [vp, vp, ci, ci, ci, vp]
+    lib.oracle_mxfp4_dequantize.restype = ci
     return lib
 
 
@@ -170,6 +184,54 @@ def moe_tokens(x_bits, expert_gateup, expert_down, idx, w, tokens, shared_gateup
     return out
 
 
+def e2m1_value(code: int, lib=None) -> float:
+    """Value of one FP4 E2M1 code (OCP Microscaling Formats v1.0 element format)."""
+    return (lib or _L()).oracle_e2m1_value(int(code))
+
+
+def mxfp4_quantize(w_bits: np.ndarray, lib=None):
+    """MXFP4 encoding of bf16 weights [G, N, K] (or [N, K]) along K: blocks of 32 share one E8M0 scale, each
+    element is an E2M1 code (the "native mxfp4 quantization" of gpt-oss, blog post section "From Dense to
+    Sparse: What Are MoEs?"). Returns codes [G, N, K/2] uint8 and scales [G, K/32, N] uint8 (layout in
+    moe_oracle.c)."""
+    lib = lib or _L()
+    w = _c(w_bits, np.uint16)
+    squeeze = w.ndim == 2
+    if squeeze:
+        w = w[None]
+    G, N, K = w.shape
+    q = np.empty((G, N, K // 2), dtype=np.uint8)
+    s = np.empty((G, K // 32, N), dtype=np.uint8)
+    if lib.oracle_mxfp4_quantize(w.ctypes.data, G, N, K, q.ctypes.data, s.ctypes.data):
+        raise ValueError(f"oracle_mxfp4_quantize: K={K} is not a multiple of 32")
+    return (q[0], s[0]) if squeeze else (q, s)
+
+
+def mxfp4_dequantize(q: np.ndarray, s: np.ndarray, lib=None) -> np.ndarray:
+    """The bf16 weights (bits) that MXFP4 codes [G, N, K/2] and scales [G, K/32, N] encode (exactly)."""
+    lib = lib or _L()
+    q = _c(q, np.uint8)
+    s = _c(s, np.uint8)
+    squeeze = q.ndim == 2
+    if squeeze:
+        q, s = q[None], s[None]
+    G, N, K2 = q.shape
+    K = 2 * K2
+    if s.shape != (G, K // 32, N):
+        raise ValueError(f"scales {s.shape} do not match codes {q.shape}")
+    w = np.empty((G, N, K), dtype=np.uint16)
+    rc = lib.oracle_mxfp4_dequantize(q.ctypes.data, s.ctypes.data, G, N, K, w.ctypes.data)
+    if rc:
+        raise ValueError(f"oracle_mxfp4_dequantize failed ({rc}): a value is not a finite bf16 number")
+    return w[0] if squeeze else w
+
+
+def mxfp4_round_trip(w_bits: np.ndarray, lib=None) -> np.ndarray:
+    """The weights an MXFP4 layer computes with: bf16 weights encoded, then decoded."""
+    q, s = mxfp4_quantize(w_bits, lib=lib)
+    return mxfp4_dequantize(q, s, lib=lib)
+
+
 class LayerReference:
     """The whole layer for one synthetic workload, computed by the oracle.
 
@@ -203,12 +265,14 @@ class LayerReference:
         wl = self.wl
         tokens = np.asarray(tokens, dtype=np.int32)
         need = np.unique(self.idx[tokens].ravel()) if len(tokens) else np.zeros(0, np.int32)
+        # MXFP4 workloads compute with the weights their encoding represents
+        enc = (lambda a: mxfp4_round_trip(a, lib=self.lib)) if wl.weights == "mxfp4" else (lambda a: a)
         for e in need:
             if self._gu[e] is None:
-                self._gu[e] = synth.w_gateup_expert_host(wl, int(e))
-                self._dn[e] = synth.w_down_expert_host(wl, int(e))
+                self._gu[e] = enc(synth.w_gateup_expert_host(wl, int(e)))
+                self._dn[e] = enc(synth.w_down_expert_host(wl, int(e)))
         if wl.shared_f and self._shared is None:
-            self._shared = synth.shared_host(wl)
+            self._shared = tuple(enc(a) for a in synth.shared_host(wl))
         sgu, sdn = self._shared if self._shared else (None, None)
         if len(tokens) == 0:
             return np.zeros((0, wl.d))

@@ -270,3 +270,111 @@ int oracle_moe_tokens(const uint16_t* x, int T, int d, int f, int E, int k, cons
     free(jobs); free(th); free(started);
     return status;
 }
+
+/*
+ * MXFP4 expert weights. The blog post's section "From Dense to Sparse: What Are MoEs?" estimates gpt-oss-20b's
+ * generation speed as memory bandwidth over the bytes of its active parameters, and notes that kernels for the
+ * model's native mxfp4 quantization would be faster still: fewer bytes per weight. The format is the OCP
+ * Microscaling Formats (MX) v1.0 one: blocks of 32 consecutive elements along the reduction axis share one
+ * E8M0 scale (an 8-bit power-of-two exponent, bias 127), and each element is an FP4 E2M1 code (sign bit, two
+ * exponent bits with bias 1, one mantissa bit; exponent field 0 holds the subnormals 0 and 0.5).
+ *
+ * Readings taken where the specification leaves a choice open:
+ *   - a block whose elements are all zero gets scale code 0 (its codes are all zero whatever the scale);
+ *   - the shared exponent is clamped to the E8M0 range [-127, 127]; code 255 (NaN) is never written;
+ *   - the sign bit of every code is the sign bit of the input, also when the magnitude rounds to 0;
+ *   - inputs must be finite.
+ * Memory layout (this library's, the specification fixes none): codes [G][N][K/2] bytes, each little-endian
+ * 32-bit word holding 8 consecutive elements k0..k0+7 of one row, nibble i (bits 4i..4i+3) being element
+ * k0+2i for i < 4 and element k0+2(i-4)+1 for i >= 4 (even elements in the low half, odd ones in the high
+ * half); scales [G][K/32][N] bytes (the scale of row n's block b at [g][b][n]).
+ */
+
+/* Value of an FP4 E2M1 code, from the element format's definition. */
+double oracle_e2m1_value(int code) {
+    const int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -mag : mag;
+}
+
+/* Nearest E2M1 magnitude code (0..7) to p >= 0, ties to the code with mantissa bit 0 (round to nearest even);
+   beyond the largest magnitude (6) the nearest is 6, which is the clamp the conversion asks for. */
+static int e2m1_nearest(double p) {
+    int best = 0;
+    double bestd = fabs(p - oracle_e2m1_value(0));
+    for (int c = 1; c < 8; ++c) {
+        const double dist = fabs(p - oracle_e2m1_value(c));
+        if (dist < bestd || (dist == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            best = c;
+            bestd = dist;
+        }
+    }
+    return best;
+}
+
+/* w [G][N][K] bf16 -> codes q [G][N][K/2], scales s [G][K/32][N]. Per block of 32: the shared exponent is
+   floor(log2(max |v|)) minus 2 (the exponent of E2M1's largest magnitude, 6 = 1.5 * 2^2), each element is
+   v / 2^shared rounded to the nearest E2M1 value. Returns 0, or -1 when K is not a multiple of 32. */
+int oracle_mxfp4_quantize(const uint16_t* w, int G, int N, int K, uint8_t* q, uint8_t* s) {
+    if (K % 32 != 0 || G < 0 || N < 0) return -1;
+    const int nb = K / 32;
+    for (long g = 0; g < G; ++g)
+        for (long n = 0; n < N; ++n)
+            for (int b = 0; b < nb; ++b) {
+                const uint16_t* v = w + ((size_t)g * N + n) * K + (size_t)b * 32;
+                double amax = 0.0;
+                for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(bf16_to_double(v[i])));
+                int shared = -127;
+                if (amax > 0.0) {
+                    int ex;
+                    frexp(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1): floor(log2(amax)) = ex - 1 */
+                    shared = ex - 1 - 2;
+                    if (shared < -127) shared = -127;
+                    if (shared > 127) shared = 127;
+                }
+                int code[32];
+                for (int i = 0; i < 32; ++i) {
+                    const double p = fabs(bf16_to_double(v[i])) / ldexp(1.0, shared);
+                    code[i] = e2m1_nearest(p) | ((v[i] >> 15) ? 8 : 0);
+                }
+                uint8_t* out = q + ((size_t)g * N + n) * (size_t)(K / 2) + (size_t)b * 16;
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t word = 0;
+                    for (int i = 0; i < 4; ++i) {
+                        word |= (uint32_t)code[8 * j + 2 * i] << (4 * i);
+                        word |= (uint32_t)code[8 * j + 2 * i + 1] << (16 + 4 * i);
+                    }
+                    for (int byte = 0; byte < 4; ++byte) out[4 * j + byte] = (uint8_t)(word >> (8 * byte));
+                }
+                s[((size_t)g * nb + b) * N + n] = (uint8_t)(shared + 127);
+            }
+    return 0;
+}
+
+/* Codes and scales -> the weights they encode, as bf16 bits: code value * 2^(scale - 127). Every such value
+   with scale <= 252 is exactly a bf16 number; returns -1 for a value that is not (overflow, scale 255),
+   -2 for a bad K. */
+int oracle_mxfp4_dequantize(const uint8_t* q, const uint8_t* s, int G, int N, int K, uint16_t* w) {
+    if (K % 32 != 0 || G < 0 || N < 0) return -2;
+    const int nb = K / 32;
+    for (long g = 0; g < G; ++g)
+        for (long n = 0; n < N; ++n)
+            for (int k = 0; k < K; ++k) {
+                const int b = k / 32, j = (k % 32) / 8, e = k % 8;
+                const uint8_t* blk = q + ((size_t)g * N + n) * (size_t)(K / 2) + (size_t)b * 16 + 4 * j;
+                const uint32_t word = (uint32_t)blk[0] | ((uint32_t)blk[1] << 8) | ((uint32_t)blk[2] << 16) |
+                                      ((uint32_t)blk[3] << 24);
+                const int nib = (e % 2 == 0) ? e / 2 : 4 + e / 2;
+                const int code = (int)((word >> (4 * nib)) & 15u);
+                const int sc = s[((size_t)g * nb + b) * N + n];
+                if (sc == 255) return -1;
+                const double val = oracle_e2m1_value(code) * ldexp(1.0, sc - 127);
+                const float fv = (float)val;
+                if ((double)fv != val || isinf(fv)) return -1;
+                uint32_t u;
+                memcpy(&u, &fv, 4);
+                if (u & 0xFFFFu) return -1;
+                w[((size_t)g * N + n) * K + k] = (uint16_t)(u >> 16);
+            }
+    return 0;
+}

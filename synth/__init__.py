@@ -141,6 +141,7 @@ class Workload:
     zipf_s: float = 0.0  # > 0: per-expert router bias so popularity follows Zipf(s)
     shared_f: int = 0  # > 0: one always-on shared SwiGLU expert of this width
     seed: int = 0
+    weights: str = "bf16"  # storage of the expert weights: "bf16", or "mxfp4" (encoded from the bf16 draws)
     note: str = field(default="", compare=False)
 
     @property
@@ -162,6 +163,9 @@ WORKLOADS = {
                           note="128 small experts, Zipf(1.2) skewed load"),
     "decode-256e-shared": Workload("decode-256e-shared", 64, 7168, 2048, 256, 8, route="sigmoid_topk_norm",
                                    shared_f=2048, note="256-expert decode with one shared expert"),
+    "decode-256e-shared-mxfp4": Workload("decode-256e-shared-mxfp4", 64, 7168, 2048, 256, 8,
+                                         route="sigmoid_topk_norm", shared_f=2048, weights="mxfp4",
+                                         note="the 256-expert decode layer with MXFP4 expert weights"),
 }
 
 

@@ -280,6 +280,127 @@ def pin_shared_expert(lib):
     np.testing.assert_allclose(both, routed + _dense_swiglu_torch(x, sgu, sdn), rtol=1e-10, atol=1e-12)
 
 
+# ---- MXFP4 weights -----------------------------------------------------------------------------------
+
+def _mx_golden():
+    return json.load(open(os.path.join(GOLDEN, "mxfp4_e2m1.json")))
+
+
+def _num(v):
+    return -0.0 if v == "-0" else float(v)
+
+
+def _pack_codes(codes):
+    """Codes [..., N, K] (0..15) -> bytes [..., N, K/2] in the documented layout, written independently of the
+    oracle: within each group of 8 elements, even elements fill the low 16 bits, odd ones the high 16 bits."""
+    c = np.asarray(codes, dtype=np.uint32)
+    *lead, K = c.shape
+    c = c.reshape(*lead, K // 8, 4, 2)  # [..., word, i, parity]
+    shifts = (np.arange(4, dtype=np.uint32) * 4)[:, None] + np.array([0, 16], dtype=np.uint32)[None, :]
+    words = (c << shifts).sum(axis=(-1, -2)).astype("<u4")
+    return words.view(np.uint8).reshape(*lead, K // 2)
+
+
+def _unpack_codes(q):
+    w = np.ascontiguousarray(q).view("<u4").astype(np.uint32)
+    nib = (w[..., None] >> (np.arange(8, dtype=np.uint32) * 4)) & 15  # [..., word, nibble]
+    order = np.array([0, 4, 1, 5, 2, 6, 3, 7])  # element e of the word sits in nibble order[e]
+    return nib[..., order].reshape(*q.shape[:-1], q.shape[-1] * 2)
+
+
+def pin_e2m1_table(lib):
+    vals = [_num(v) for v in _mx_golden()["values"]]
+    for code, want in enumerate(vals):
+        got = oracle.e2m1_value(code, lib=lib)
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), (code, got, want)
+
+
+def pin_mxfp4_rounding_golden(lib):
+    g = _mx_golden()["rounding"]
+    vals = [_num(v) for v in g["inputs"]] + [0.0] * (32 - len(g["inputs"]))
+    w = _bf16(np.array(vals, dtype=np.float32))[None, :]
+    q, s = oracle.mxfp4_quantize(w, lib=lib)
+    assert s.shape == (1, 1) and int(s[0, 0]) == g["scale_code"]
+    codes = _unpack_codes(q)[0]
+    assert codes[: len(g["codes"])].tolist() == g["codes"], codes.tolist()
+    assert (codes[len(g["codes"]):] == 0).all()
+
+
+def pin_mxfp4_packing_golden(lib):
+    g = _mx_golden()
+    vals = [_num(g["values"][c]) for c in g["packing"]["codes"]] + [0.0] * 24
+    q, s = oracle.mxfp4_quantize(_bf16(np.array(vals, dtype=np.float32))[None, :], lib=lib)
+    assert q[0, :4].tolist() == g["packing"]["bytes"]
+    assert int(s[0, 0]) == 127
+
+
+def pin_mxfp4_round_trip(lib):
+    """Blocks made of E2M1 values times a power of two, with at least one magnitude of 4 or 6 (which fixes the
+    scale), decode to exact bf16 numbers and encode back to the same bytes; the decode agrees with an
+    independent numpy decode of the documented layout and the specification's value table."""
+    rng = _rng(20)
+    G, N, K = 3, 5, 96  # N != K/32, so a transposed scale layout would show
+    codes = rng.integers(0, 16, size=(G, N, K))
+    codes[..., ::32] = rng.choice([6, 7, 14, 15], size=(G, N, K // 32))
+    scales = rng.integers(0, 253, size=(G, K // 32, N)).astype(np.uint8)
+    scales[0, 0, :] = [0, 1, 126, 127, 252]
+    q = _pack_codes(codes)
+    w = oracle.mxfp4_dequantize(q, scales, lib=lib)
+    table = np.array([_num(v) for v in _mx_golden()["values"]])
+    sc = np.repeat(np.transpose(scales, (0, 2, 1)).astype(np.float64), 32, axis=-1)  # [G, N, K]
+    want = table[_unpack_codes(q)] * np.exp2(sc - 127)
+    np.testing.assert_array_equal(_f64(w), want)
+    q2, s2 = oracle.mxfp4_quantize(w, lib=lib)
+    np.testing.assert_array_equal(s2, scales)
+    np.testing.assert_array_equal(q2, q)
+
+
+def pin_mxfp4_scale_closed_form(lib):
+    """Shared scale = 2^(floor(log2 max|v|) - 2), clamped to the E8M0 range; an all-zero block gets code 0."""
+    cases = [  # (max |v| of the block, expected scale code)
+        (0.0, 0), (1.0, 125), (0.02, 119), (4.0, 127), (7.9, 127), (8.0, 128),
+        (2.0 ** -130, 0), (2.0 ** -120, 5), (3.0e38, 252),
+    ]
+    rows = []
+    for amax, _ in cases:
+        r = np.zeros(32, dtype=np.float32)
+        r[7] = -amax
+        r[3] = amax / 3
+        rows.append(r)
+    w = _bf16(np.stack(rows))
+    q, s = oracle.mxfp4_quantize(w, lib=lib)
+    assert s[0].tolist() == [c for _, c in cases], s[0].tolist()
+    # the element holding max |v| decodes to -4 or -6 times the scale whenever it is not clamped away
+    amax_bf = np.abs(_f64(w[:, 7]))
+    dq = _f64(oracle.mxfp4_dequantize(q, s, lib=lib))
+    for i, (amax, code) in enumerate(cases):
+        X = 2.0 ** (int(code) - 127)
+        if amax == 0:
+            assert (dq[i] == 0).all()
+        elif amax_bf[i] / X >= 4:
+            assert abs(dq[i, 7]) in (4 * X, 6 * X) and dq[i, 7] < 0
+
+
+def pin_mxfp4_error_bound(lib):
+    """Encode then decode of random weights: max|v| / scale lies in [4, 8); every element is within half the
+    E2M1 grid spacing at its magnitude (0.25 below 2, 0.5 in [2, 4), 1 in [4, 6]) times the scale, and
+    magnitudes above 6 times the scale decode to exactly 6 times the scale."""
+    rng = _rng(21)
+    w = _random_bf16(rng, (4, 64, 256), 0.02)
+    q, s = oracle.mxfp4_quantize(w, lib=lib)
+    dq = _f64(oracle.mxfp4_dequantize(q, s, lib=lib))
+    v = _f64(w)
+    X = np.repeat(np.exp2(np.transpose(s, (0, 2, 1)).astype(np.float64) - 127), 32, axis=-1)
+    p = np.abs(v) / X
+    blocks = p.reshape(4, 64, 8, 32).max(-1)
+    assert ((blocks >= 4) & (blocks < 8)).all()
+    half = np.where(p < 2, 0.25, np.where(p < 4, 0.5, 1.0))
+    inside = p <= 6
+    assert (np.abs(dq - v)[inside] <= half[inside] * X[inside]).all()
+    assert (np.abs(dq)[~inside] == 6 * X[~inside]).all()
+    assert (np.signbit(dq) == np.signbit(v)).all()
+
+
 PINS = [
     pin_router_logits_numpy,
     pin_topk_golden,
@@ -295,4 +416,10 @@ PINS = [
     pin_down_linearity,
     pin_swiglu_golden,
     pin_shared_expert,
+    pin_e2m1_table,
+    pin_mxfp4_rounding_golden,
+    pin_mxfp4_packing_golden,
+    pin_mxfp4_round_trip,
+    pin_mxfp4_scale_closed_form,
+    pin_mxfp4_error_bound,
 ]

@@ -36,6 +36,22 @@ MUTATIONS = {
     "routing_weight_dropped": ("acc[c] += scale * s;", "acc[c] += s;"),
     "last_expert_dropped": ("for (int j = 0; j < J->k; ++j) {", "for (int j = 0; j < J->k - 1; ++j) {"),
     "shared_expert_half_weight": ("J->wd_s, 1.0, h, acc)", "J->wd_s, 0.5, h, acc)"),
+    "e2m1_exponent_bias_dropped": ("ldexp(1.0 + 0.5 * m, e - 1)", "ldexp(1.0 + 0.5 * m, e)"),
+    "e2m1_subnormal_as_one": ("e == 0 ? 0.5 * m :", "e == 0 ? 1.0 * m :"),
+    "mxfp4_ties_to_lower_code": ("(dist == bestd && (c & 1) == 0 && (best & 1) == 1)", "0"),
+    "mxfp4_ties_away_from_zero": ("(dist == bestd && (c & 1) == 0 && (best & 1) == 1)", "dist == bestd"),
+    "mxfp4_scale_emax_off_by_one": ("shared = ex - 1 - 2;", "shared = ex - 1 - 1;"),
+    "mxfp4_scale_ceil_not_floor": ("shared = ex - 1 - 2;", "shared = ex - 2;"),
+    "mxfp4_sign_dropped": ("e2m1_nearest(p) | ((v[i] >> 15) ? 8 : 0)", "e2m1_nearest(p)"),
+    "mxfp4_natural_nibble_order": (
+        "word |= (uint32_t)code[8 * j + 2 * i] << (4 * i);\n                        word |= (uint32_t)code[8 * j + 2 * i + 1] << (16 + 4 * i);",
+        "word |= (uint32_t)code[8 * j + 2 * i] << (8 * i);\n                        word |= (uint32_t)code[8 * j + 2 * i + 1] << (8 * i + 4);"),
+    "mxfp4_scale_layout_row_major": ("s[((size_t)g * nb + b) * N + n] = (uint8_t)(shared + 127);",
+                                     "s[((size_t)g * N + n) * nb + b] = (uint8_t)(shared + 127);"),
+    "mxfp4_zero_block_scale_max": ("int shared = -127;", "int shared = 127;"),
+    "mxfp4_decode_odd_even_swapped": ("const int nib = (e % 2 == 0) ? e / 2 : 4 + e / 2;",
+                                      "const int nib = (e % 2 == 1) ? e / 2 : 4 + e / 2;"),
+    "mxfp4_decode_scale_bias": ("oracle_e2m1_value(code) * ldexp(1.0, sc - 127)", "oracle_e2m1_value(code) * ldexp(1.0, sc - 126)"),
 }
 
 
