@@ -195,18 +195,24 @@ class ClockSampler:
 
 # ---- roofline arithmetic -------------------------------------------------------------------------------
 
+def weight_bytes(wl) -> float:
+    """Bytes per expert weight: 2 for bf16; MXFP4 stores a 4-bit code plus one 8-bit scale per 32 weights."""
+    return 0.5 + 1.0 / 32 if wl.weights == "mxfp4" else 2.0
+
+
 def gemm_figures(wl, counts):
     """Algorithmic FLOPs and DRAM bytes per launch of the two grouped GEMMs, from the realised routing."""
-    R, d, f = wl.R, wl.d, wl.f
+    R, d, f, wb = wl.R, wl.d, wl.f, weight_bytes(wl)
     active = int((counts > 0).sum())
-    gateup = {"flop": 4.0 * R * d * f, "bytes": active * 2 * f * d * 2 + R * d * 2 + R * f * 2}
-    down = {"flop": 2.0 * R * f * d, "bytes": active * d * f * 2 + R * f * 2 + R * d * 2}
+    gateup = {"flop": 4.0 * R * d * f, "bytes": active * 2 * f * d * wb + R * d * 2 + R * f * 2}
+    down = {"flop": 2.0 * R * f * d, "bytes": active * d * f * wb + R * f * 2 + R * d * 2}
     return active, gateup, down
 
 
 def layer_figures(wl, active):
     flop = wl.flops()
-    bytes_ = (active * 3 * wl.d * wl.f * 2 + 3 * wl.d * wl.shared_f * 2 + wl.T * wl.d * 2 * 2 + wl.E * wl.d * 4)
+    wb = weight_bytes(wl)
+    bytes_ = (active * 3 * wl.d * wl.f * wb + 3 * wl.d * wl.shared_f * wb + wl.T * wl.d * 2 * 2 + wl.E * wl.d * 4)
     return flop, bytes_
 
 
@@ -242,7 +248,9 @@ class OracleStep:
         self.order = np.random.default_rng(1234).permutation(wl.T).astype(np.int32)
         self.gu = [None] * wl.E
         self.dn = [None] * wl.E
-        self.shared = synth.shared_host(wl) if wl.shared_f else (None, None)
+        # MXFP4 workloads compute with the weights the encoding represents
+        self.enc = (lambda a: oracle.mxfp4_round_trip(a)) if wl.weights == "mxfp4" else (lambda a: a)
+        self.shared = tuple(self.enc(a) for a in synth.shared_host(wl)) if wl.shared_f else (None, None)
         self.threads = max(1, len(os.sched_getaffinity(0)))
 
     def prepare(self, n):
@@ -254,8 +262,8 @@ class OracleStep:
         idx, _ = self.oracle.topk(l, self.wl.k, self.wl.route)
         for e in self.np.unique(idx):
             if self.gu[e] is None:
-                self.gu[e] = synth.w_gateup_expert_host(self.wl, int(e))
-                self.dn[e] = synth.w_down_expert_host(self.wl, int(e))
+                self.gu[e] = self.enc(synth.w_gateup_expert_host(self.wl, int(e)))
+                self.dn[e] = self.enc(synth.w_down_expert_host(self.wl, int(e)))
 
     def run(self, n):
         o, np = self.oracle, self.np
@@ -290,7 +298,7 @@ def cpu_baseline(wl, seconds: float) -> dict:
 
 def workload_config(wl) -> dict:
     return {"workload": wl.name, "T": wl.T, "d": wl.d, "f": wl.f, "E": wl.E, "k": wl.k, "route": wl.route,
-            "shared_f": wl.shared_f, "zipf_s": wl.zipf_s, "seed": wl.seed,
+            "shared_f": wl.shared_f, "zipf_s": wl.zipf_s, "seed": wl.seed, "expert_weights": wl.weights,
             "l2": "flushed (256 MiB write) before every timed step, outside the events"}
 
 
@@ -346,7 +354,11 @@ def run_ours(args):
     synth.build_cuda()
     inp = synth.device_inputs(wl, dev)
     layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
-                   inp["w_gateup_shared"], inp["w_down_shared"])
+                   inp["w_gateup_shared"], inp["w_down_shared"], weights=wl.weights)
+    if wl.weights != "bf16":  # the layer keeps only its encoded weights
+        for key in ("w_gateup", "w_down", "w_gateup_shared", "w_down_shared"):
+            inp[key] = None
+        torch.cuda.empty_cache()
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -400,8 +412,7 @@ def run_ours(args):
     # reuse of a buffer after the last reader of its previous contents.
     e2e = None
     if not args.no_e2e:
-        layers = [layer, MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
-                                inp["w_gateup_shared"], inp["w_down_shared"])]
+        layers = [layer, layer.sibling()]
         x_host = [x.cpu().pin_memory() for _ in range(2)]
         y_host = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
         x_dev = [torch.empty_like(x) for _ in range(2)]

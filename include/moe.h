@@ -17,6 +17,9 @@
  *   moe_grouped_gemm_down   y_perm = h Wd^T, per expert
  *   moe_unpermute_combine   y[t] = sum_j w[t,j] * y_perm[row of (t,j)] (+ shared[t])
  *
+ * With MXFP4 expert weights (encoded once by moe_mxfp4_quantize) the two
+ * grouped GEMMs are moe_grouped_gemm_gateup_mxfp4 / moe_grouped_gemm_down_mxfp4.
+ *
  * Conventions (all entry points):
  *  - Every pointer argument is a DEVICE pointer to memory the caller allocated
  *    and owns, unless stated otherwise. The library allocates no device memory
@@ -204,6 +207,58 @@ moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_ga
  *   h [M][f] bf16, y [M][d] bf16, group_offsets as above. */
 moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down, const int32_t* group_offsets,
                                    int G, int M, int d, int f, moe_bf16_t* y, cudaStream_t stream);
+
+/* ---- MXFP4 expert weights ----
+ * The blog post's section "From Dense to Sparse: What Are MoEs?" estimates
+ * generation speed as memory bandwidth over the bytes of the active
+ * parameters and notes that kernels for gpt-oss's native mxfp4 quantization
+ * would be faster. MXFP4 is the OCP Microscaling Formats (MX) v1.0 format:
+ * along the reduction axis (K), blocks of 32 elements share one E8M0 scale
+ * (value 2^(s-127)) and each element is an FP4 E2M1 code (sign bit, two
+ * exponent bits with bias 1, one mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6). Layout of a [G][N][K] weight tensor (this library's; the format
+ * fixes no memory order):
+ *   q [G][N][K/2] uint8: each little-endian 32-bit word holds 8 consecutive
+ *     elements k0..k0+7 of a row; nibble i (bits 4i..4i+3) is element k0+2i
+ *     for i < 4 and element k0+2(i-4)+1 for i >= 4 (even elements in the low
+ *     16 bits, odd ones in the high 16 bits);
+ *   s [G][K/32][N] uint8: the scale of row n's block b is s[g][b][n].
+ * A gate|up tensor [G][2f][d] is encoded along d, a down tensor [G][d][f]
+ * along f. */
+
+/* Encode bf16 weights w [G][N][K] as MXFP4 codes q and scales s (layout
+ * above). Per block of 32: the scale exponent is floor(log2(max |v|)) - 2
+ * (2 being the exponent of E2M1's largest magnitude 6), clamped to
+ * [-127, 127]; an all-zero block gets s = 0. Every v / 2^(s-127) is rounded
+ * to the nearest E2M1 magnitude, ties to the one with mantissa bit 0, values
+ * above 6 clamped to 6; the sign bit is w's, also for a magnitude of 0.
+ * Inputs must be finite. Deterministic and exact (integer decisions only).
+ *   w 16-byte aligned; q 16-byte aligned; K a positive multiple of 32;
+ *   G = 0 or N = 0 is an empty no-op. */
+moe_status_t moe_mxfp4_quantize(const moe_bf16_t* w, int G, int N, int K, uint8_t* q, uint8_t* s,
+                                cudaStream_t stream);
+
+/* moe_grouped_gemm_gateup with MXFP4 weights: the same h, computed with the
+ * weights the codes encode (decoded exactly to bf16; bf16 products, fp32
+ * accumulation, h rounded to bf16).
+ *   wq_gateup [G][2f][d/2], ws_gateup [G][d/32][2f] (gate rows, then up rows,
+ *   as in moe_grouped_gemm_gateup), encoded along d.
+ * Built for few rows per expert (decode), where streaming the weights is the
+ * cost: weight rows are the MMA's M dimension and the group's rows its N
+ * dimension (16, 32 or 64 per tile, chosen from M / G); groups larger than the
+ * tile are covered by several tiles, each decoding the weights again.
+ * Limits: d, f positive multiples of 32; all pointers 16-byte aligned; the
+ * other arguments as for moe_grouped_gemm_gateup. Scale codes above 252 are
+ * not supported (the decoded weight would overflow bf16). */
+moe_status_t moe_grouped_gemm_gateup_mxfp4(const moe_bf16_t* a, const uint8_t* wq_gateup, const uint8_t* ws_gateup,
+                                           const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* h,
+                                           cudaStream_t stream);
+
+/* moe_grouped_gemm_down with MXFP4 weights wq_down [G][d][f/2],
+ * ws_down [G][f/32][d] (encoded along f); limits as above. */
+moe_status_t moe_grouped_gemm_down_mxfp4(const moe_bf16_t* h, const uint8_t* wq_down, const uint8_t* ws_down,
+                                         const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* y,
+                                         cudaStream_t stream);
 
 /* Apply the routing weights and return to token order ("apply the routing
  * weights and then collect and reorder the results", section "Expert

@@ -24,8 +24,8 @@ ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm":
 # every entry point of include/moe.h
 EXPORTS = ("moe_route_topk", "moe_router_split_weights", "moe_route_topk_split", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
            "moe_permute_static_ws",
-           "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_unpermute_combine", "moe_get_device_error",
-           "moe_last_error_string")
+           "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_mxfp4_quantize", "moe_grouped_gemm_gateup_mxfp4",
+           "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_get_device_error", "moe_last_error_string")
 
 
 class MoEError(RuntimeError):
@@ -50,6 +50,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_permute_static_ws": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp],
         "moe_grouped_gemm_gateup": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_down": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_mxfp4_quantize": [vp, ci, ci, ci, vp, vp, vp],
+        "moe_grouped_gemm_gateup_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_grouped_gemm_down_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_unpermute_combine": [vp, vp, vp, vp, ci, ci, ci, vp, vp],
         "moe_get_device_error": [ctypes.POINTER(ctypes.c_uint), vp],
         "moe_last_error_string": [],
@@ -206,6 +209,40 @@ def grouped_gemm_down(h, w_down, group_offsets, y, stream=None):
     _need(y, torch.bfloat16, (M, d), "y")
     _check(_lib.moe_grouped_gemm_down(_p(h), _p(w_down), _p(group_offsets), G, M, d, f, _p(y), _stream(stream)),
            "moe_grouped_gemm_down")
+
+
+def mxfp4_quantize(w, q, s, stream=None):
+    """Encode bf16 weights w [G, N, K] as MXFP4 codes q [G, N, K/2] (uint8) and scales s [G, K/32, N] (uint8)."""
+    G, N, K = w.shape
+    _need(w, torch.bfloat16, (G, N, K), "w")
+    _need(q, torch.uint8, (G, N, K // 2), "q")
+    _need(s, torch.uint8, (G, K // 32, N), "s")
+    _check(_lib.moe_mxfp4_quantize(_p(w), G, N, K, _p(q), _p(s), _stream(stream)), "moe_mxfp4_quantize")
+
+
+def grouped_gemm_gateup_mxfp4(a, wq_gateup, ws_gateup, group_offsets, h, stream=None):
+    M, d = a.shape
+    G, two_f, _ = wq_gateup.shape
+    f = two_f // 2
+    _need(a, torch.bfloat16, (M, d), "a")
+    _need(wq_gateup, torch.uint8, (G, 2 * f, d // 2), "wq_gateup")
+    _need(ws_gateup, torch.uint8, (G, d // 32, 2 * f), "ws_gateup")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(h, torch.bfloat16, (M, f), "h")
+    _check(_lib.moe_grouped_gemm_gateup_mxfp4(_p(a), _p(wq_gateup), _p(ws_gateup), _p(group_offsets), G, M, d, f,
+                                              _p(h), _stream(stream)), "moe_grouped_gemm_gateup_mxfp4")
+
+
+def grouped_gemm_down_mxfp4(h, wq_down, ws_down, group_offsets, y, stream=None):
+    M, f = h.shape
+    G, d, _ = wq_down.shape
+    _need(h, torch.bfloat16, (M, f), "h")
+    _need(wq_down, torch.uint8, (G, d, f // 2), "wq_down")
+    _need(ws_down, torch.uint8, (G, f // 32, d), "ws_down")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(y, torch.bfloat16, (M, d), "y")
+    _check(_lib.moe_grouped_gemm_down_mxfp4(_p(h), _p(wq_down), _p(ws_down), _p(group_offsets), G, M, d, f, _p(y),
+                                            _stream(stream)), "moe_grouped_gemm_down_mxfp4")
 
 
 def unpermute_combine(y_perm, inv_perm, topk_w, shared, y, stream=None):

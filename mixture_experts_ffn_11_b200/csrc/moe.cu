@@ -18,6 +18,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_wide.cuh"
+#include "gemm_fp4.cuh"
 #include "combine.cuh"
 
 using namespace moe;
@@ -102,6 +103,12 @@ cudaError_t set_gemm_attributes() {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, true>, a, Wide240GU::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<256, 4, false>, a, Wide256DN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, false>, a, Wide240DN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<16, true>, a, GemmFp4Shape<16, true>::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<32, true>, a, GemmFp4Shape<32, true>::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<64, true>, a, GemmFp4Shape<64, true>::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<16, false>, a, GemmFp4Shape<16, false>::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<32, false>, a, GemmFp4Shape<32, false>::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<64, false>, a, GemmFp4Shape<64, false>::SMEM_BYTES);
     return e;
 }
 
@@ -314,6 +321,74 @@ moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cud
     if (wide_tiles >= sms)
         return gateup ? launch_single<256, 4, true>(p, sms, stream) : launch_single<256, 4, false>(p, sms, stream);
     return gateup ? launch_single<64, 8, true>(p, sms, stream) : launch_single<64, 8, false>(p, sms, stream);
+}
+
+// ---- MXFP4 weights ----
+struct Fp4Problem {
+    const void* a;        // activations [M][K] bf16
+    const uint8_t* q;     // codes [G][rows][K/2]
+    const uint8_t* s;     // scales [G][K/32][rows]
+    const int32_t* offsets;
+    int G, M, K, n_out, f, rows;  // rows: weight rows per group (2f for gate|up, d for down)
+    void* out;
+};
+
+template <int NT, bool GATEUP>
+moe_status_t launch_fp4(const Fp4Problem& p, int sms, cudaStream_t stream) {
+    using S = GemmFp4Shape<NT, GATEUP>;
+    CUtensorMap tx, tq, ts;
+    const cuuint64_t xdims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
+    const cuuint64_t xstr[1] = {(cuuint64_t)p.K * 2};
+    const cuuint32_t xbox[2] = {64, (cuuint32_t)NT};
+    moe_status_t st = make_tmap(&tx, p.a, 2, xdims, xstr, xbox);
+    if (st != MOE_OK) return st;
+    const cuuint64_t qdims[3] = {(cuuint64_t)p.K / 2, (cuuint64_t)p.rows, (cuuint64_t)p.G};
+    const cuuint64_t qstr[2] = {(cuuint64_t)p.K / 2, (cuuint64_t)p.rows * (p.K / 2)};
+    const cuuint32_t qbox[3] = {GF_KS / 2, GF_BM, 1};
+    if ((st = make_tmap(&tq, p.q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_DATA_TYPE_UINT8)) != MOE_OK) return st;
+    const cuuint64_t sdims[3] = {(cuuint64_t)p.rows, (cuuint64_t)p.K / 32, (cuuint64_t)p.G};
+    const cuuint64_t sstr[2] = {(cuuint64_t)p.rows, (cuuint64_t)p.rows * (p.K / 32)};
+    const cuuint32_t sbox[3] = {GF_BM, GF_KS / 32, 1};
+    if ((st = make_tmap(&ts, p.s, 3, sdims, sstr, sbox, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
+        MOE_OK)
+        return st;
+    GemmArgs args;
+    args.group_offsets = p.offsets;
+    args.G = p.G;
+    args.M = p.M;
+    args.K = p.K;
+    args.n_out = p.n_out;
+    args.f = p.f;
+    args.n_tiles = (p.n_out + GF_BM - 1) / GF_BM;
+    args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    const long upper = ((long)p.M / NT + p.G) * (long)args.n_tiles;  // >= the real tile count
+    const int grid = (int)(upper < sms ? upper : sms);
+    const int streamed_once = (long)p.M <= (long)p.G * NT ? 1 : 0;
+    const cudaError_t e = launch_pdl(grouped_gemm_fp4_kernel<NT, GATEUP>, dim3(grid), dim3(GF_THREADS), S::SMEM_BYTES,
+                                     stream, tx, tq, ts, args, streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup_mxfp4" : "grouped_gemm_down_mxfp4", e);
+}
+
+// Token tile: the smallest of 16, 32, 64 that holds an average group (decode: 2 rows of 512 over 256 experts;
+// a shared expert: all T rows in one group). Larger groups take several token tiles.
+template <bool GATEUP>
+moe_status_t launch_fp4_nt(const Fp4Problem& p, int sms, cudaStream_t stream) {
+    if ((long)p.M <= 8L * p.G) return launch_fp4<16, GATEUP>(p, sms, stream);
+    if ((long)p.M <= 24L * p.G) return launch_fp4<32, GATEUP>(p, sms, stream);
+    return launch_fp4<64, GATEUP>(p, sms, stream);
+}
+
+moe_status_t check_fp4_args(const void* a, const uint8_t* q, const uint8_t* s, const int32_t* offsets, int G, int M,
+                            int d, int f, const void* out) {
+    if (!q || !s || !offsets || (M > 0 && (!a || !out))) return fail(MOE_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(a) || !aligned16(q) || !aligned16(s) || !aligned16(out))
+        return fail(MOE_ERR_INVALID_ARG, "activation, code, scale and output pointers must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(offsets) & 3u) != 0) return fail(MOE_ERR_INVALID_ARG, "offsets misaligned");
+    if (G < 1 || G > GG_MAX_GROUPS) return fail(MOE_ERR_INVALID_ARG, "G=%d outside [1, %d]", G, GG_MAX_GROUPS);
+    if (M < 0) return fail(MOE_ERR_INVALID_ARG, "M=%d < 0", M);
+    if (d < 32 || f < 32 || d % 32 || f % 32)
+        return fail(MOE_ERR_INVALID_ARG, "d=%d and f=%d must be positive multiples of 32 (MXFP4 blocks)", d, f);
+    return MOE_OK;
 }
 
 template <int BNR, bool PRESPLIT>
@@ -639,6 +714,48 @@ moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down
     if (M == 0) return MOE_OK;
     const GemmProblem p{h, w_down, group_offsets, G, M, f, d, f, y};
     return launch_grouped_gemm(p, false, di.sms, stream);
+}
+
+moe_status_t moe_mxfp4_quantize(const moe_bf16_t* w, int G, int N, int K, uint8_t* q, uint8_t* s,
+                                cudaStream_t stream) {
+    if (G < 0 || N < 0) return fail(MOE_ERR_INVALID_ARG, "G=%d, N=%d must be >= 0", G, N);
+    if (K < 32 || K % 32) return fail(MOE_ERR_INVALID_ARG, "K=%d must be a positive multiple of 32", K);
+    if (G == 0 || N == 0) return MOE_OK;
+    if (!w || !q || !s) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(w) || !aligned16(q)) return fail(MOE_ERR_INVALID_ARG, "w and q must be 16-byte aligned");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const long rows = (long)G * N;
+    const long blocks = rows * (K / 32);
+    const int grid = grid_cap((blocks + 255) / 256, di.sms, 8);
+    const cudaError_t e = launch_pdl(mxfp4_quantize_kernel, dim3(grid), dim3(256), 0, stream,
+                                     reinterpret_cast<const __nv_bfloat16*>(w), rows, N, K, q, s);
+    return check_launch("mxfp4_quantize", e);
+}
+
+moe_status_t moe_grouped_gemm_gateup_mxfp4(const moe_bf16_t* a, const uint8_t* wq_gateup, const uint8_t* ws_gateup,
+                                           const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* h,
+                                           cudaStream_t stream) {
+    moe_status_t st = check_fp4_args(a, wq_gateup, ws_gateup, group_offsets, G, M, d, f, h);
+    if (st != MOE_OK) return st;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    const Fp4Problem p{a, wq_gateup, ws_gateup, group_offsets, G, M, d, f, f, 2 * f, h};
+    return launch_fp4_nt<true>(p, di.sms, stream);
+}
+
+moe_status_t moe_grouped_gemm_down_mxfp4(const moe_bf16_t* h, const uint8_t* wq_down, const uint8_t* ws_down,
+                                         const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* y,
+                                         cudaStream_t stream) {
+    moe_status_t st = check_fp4_args(h, wq_down, ws_down, group_offsets, G, M, d, f, y);
+    if (st != MOE_OK) return st;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    const Fp4Problem p{h, wq_down, ws_down, group_offsets, G, M, f, d, f, d, y};
+    return launch_fp4_nt<false>(p, di.sms, stream);
 }
 
 moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w,

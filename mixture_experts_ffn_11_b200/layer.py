@@ -11,9 +11,20 @@ library entry points in order on one stream. It does no arithmetic of its own.
 """
 from __future__ import annotations
 
+import copy
+
 import torch
 
 from . import _native as N
+
+
+def _encode_mxfp4(w):
+    """bf16 weights [G, N, K] -> (codes [G, N, K/2], scales [G, K/32, N]) on the weights' device."""
+    G, Nr, K = w.shape
+    q = torch.empty(G, Nr, K // 2, dtype=torch.uint8, device=w.device)
+    s = torch.empty(G, K // 32, Nr, dtype=torch.uint8, device=w.device)
+    N.mxfp4_quantize(w, q, s)
+    return q, s
 
 
 class MoEFFN:
@@ -21,20 +32,33 @@ class MoEFFN:
 
     w_router [E, d] fp32; w_gateup [E, 2f, d] bf16 (gate rows, then up rows); w_down [E, d, f] bf16;
     bias [E] fp32 or None; optional shared expert w_gateup_shared [2fs, d], w_down_shared [d, fs].
+    weights: "bf16" keeps the expert weights as given; "mxfp4" encodes them once (moe_mxfp4_quantize, 4.25 bits
+    per weight) and the layer then computes with the weights the encoding represents, through the MXFP4 grouped
+    GEMMs; the bf16 tensors are not kept.
     """
 
     def __init__(self, w_router, w_gateup, w_down, k: int, route: str = "topk_softmax", bias=None,
-                 w_gateup_shared=None, w_down_shared=None):
+                 w_gateup_shared=None, w_down_shared=None, weights: str = "bf16"):
         self.E, self.d = w_router.shape
         self.f = w_gateup.shape[1] // 2
         self.k = k
         self.route = route
         if route not in N.ROUTE_MODES:
             raise ValueError(f"unknown routing mode {route!r}")
+        if weights not in ("bf16", "mxfp4"):
+            raise ValueError(f"unknown weight format {weights!r}")
+        self.weights = weights
         self.w_router, self.w_gateup, self.w_down, self.bias = w_router, w_gateup, w_down, bias
         self.w_gateup_shared, self.w_down_shared = w_gateup_shared, w_down_shared
         self.shared_f = w_gateup_shared.shape[0] // 2 if w_gateup_shared is not None else 0
         self.device = w_gateup.device
+        if weights == "mxfp4":
+            self.mx_gateup = _encode_mxfp4(w_gateup)
+            self.mx_down = _encode_mxfp4(w_down)
+            if self.shared_f:
+                self.mx_gateup_shared = _encode_mxfp4(w_gateup_shared.unsqueeze(0))
+                self.mx_down_shared = _encode_mxfp4(w_down_shared.unsqueeze(0))
+            self.w_gateup = self.w_down = self.w_gateup_shared = self.w_down_shared = None
         self._T = None
         self.buf = {}
         # the tensor-core router (E <= 128) reads W_r as three bf16 pieces: split once here, not in every call
@@ -45,6 +69,14 @@ class MoEFFN:
         # the shared expert depends only on x: it runs on a side stream, beside routing and grouping (which
         # leave most SMs free), and the routed GEMMs wait for it
         self._side = torch.cuda.Stream(self.device) if self.shared_f else None
+
+    def sibling(self) -> "MoEFFN":
+        """Another layer over the same weights (nothing is copied or re-encoded) with its own intermediate buffers
+        and side stream, so that two calls can be in flight at once."""
+        twin = copy.copy(self)
+        twin.buf, twin._T = {}, None
+        twin._side = torch.cuda.Stream(self.device) if self.shared_f else None
+        return twin
 
     def refresh_router(self):
         """Re-split the router weights; call after changing w_router in place."""
@@ -106,9 +138,8 @@ class MoEFFN:
             if timing is not None:
                 timing["shared"] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 timing["shared"][0].record(side)
-            N.grouped_gemm_gateup(x, self.w_gateup_shared.unsqueeze(0), b["shared_offsets"], b["h_shared"], side)
-            N.grouped_gemm_down(b["h_shared"], self.w_down_shared.unsqueeze(0), b["shared_offsets"], b["shared"],
-                                side)
+            self._gateup(x, "shared", b["shared_offsets"], b["h_shared"], side)
+            self._down(b["h_shared"], "shared", b["shared_offsets"], b["shared"], side)
             shared_done = torch.cuda.Event()
             shared_done.record(side)
             if timing is not None:
@@ -129,10 +160,10 @@ class MoEFFN:
             # the routed GEMMs are persistent kernels sized to every SM: they start once the shared expert is done
             s.wait_event(shared_done)
         mark("gateup", True)
-        N.grouped_gemm_gateup(b["x_perm"], self.w_gateup, b["offsets"], b["h"], s)
+        self._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)
         mark("gateup", False)
         mark("down", True)
-        N.grouped_gemm_down(b["h"], self.w_down, b["offsets"], b["y_perm"], s)
+        self._down(b["h"], "routed", b["offsets"], b["y_perm"], s)
         mark("down", False)
         mark("combine", True)
         N.unpermute_combine(b["y_perm"], b["inv_perm"], b["topk_w"], shared, b["y"], s)
@@ -140,6 +171,22 @@ class MoEFFN:
         return b["y"]
 
     __call__ = forward
+
+    def _gateup(self, a, which, offsets, h, stream):
+        if self.weights == "mxfp4":
+            q, sc = self.mx_gateup if which == "routed" else self.mx_gateup_shared
+            N.grouped_gemm_gateup_mxfp4(a, q, sc, offsets, h, stream)
+        else:
+            w = self.w_gateup if which == "routed" else self.w_gateup_shared.unsqueeze(0)
+            N.grouped_gemm_gateup(a, w, offsets, h, stream)
+
+    def _down(self, h, which, offsets, y, stream):
+        if self.weights == "mxfp4":
+            q, sc = self.mx_down if which == "routed" else self.mx_down_shared
+            N.grouped_gemm_down_mxfp4(h, q, sc, offsets, y, stream)
+        else:
+            w = self.w_down if which == "routed" else self.w_down_shared.unsqueeze(0)
+            N.grouped_gemm_down(h, w, offsets, y, stream)
 
     def kernel_launches(self, T: int) -> int:
         """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the

@@ -63,9 +63,9 @@ def load(path: str | None = None):
     lib.oracle_moe_tokens.restype = ci
     lib.oracle_e2m1_value.argtypes = [ci]
     lib.oracle_e2m1_value.restype = ctypes.c_double
-    lib.oracle_mxfp4_quantize.argtypes = [vp, ci, ci, ci, vp, vp]
+    lib.oracle_mxfp4_quantize.argtypes = [vp, ci, ci, ci, vp, vp, ci]
     lib.oracle_mxfp4_quantize.restype = ci
-    lib.oracle_mxfp4_dequantize.argtypes = [vp, vp, ci, ci, ci, vp]
+    lib.oracle_mxfp4_dequantize.argtypes = [vp, vp, ci, ci, ci, vp, ci]
     lib.oracle_mxfp4_dequantize.restype = ci
     return lib
 
@@ -78,6 +78,10 @@ def _L():
     if _lib is None:
         _lib = load()
     return _lib
+
+
+def _threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
 
 
 def _c(a, dtype):
@@ -202,7 +206,7 @@ def mxfp4_quantize(w_bits: np.ndarray, lib=None):
     G, N, K = w.shape
     q = np.empty((G, N, K // 2), dtype=np.uint8)
     s = np.empty((G, K // 32, N), dtype=np.uint8)
-    if lib.oracle_mxfp4_quantize(w.ctypes.data, G, N, K, q.ctypes.data, s.ctypes.data):
+    if lib.oracle_mxfp4_quantize(w.ctypes.data, G, N, K, q.ctypes.data, s.ctypes.data, _threads()):
         raise ValueError(f"oracle_mxfp4_quantize: K={K} is not a multiple of 32")
     return (q[0], s[0]) if squeeze else (q, s)
 
@@ -220,7 +224,7 @@ def mxfp4_dequantize(q: np.ndarray, s: np.ndarray, lib=None) -> np.ndarray:
     if s.shape != (G, K // 32, N):
         raise ValueError(f"scales {s.shape} do not match codes {q.shape}")
     w = np.empty((G, N, K), dtype=np.uint16)
-    rc = lib.oracle_mxfp4_dequantize(q.ctypes.data, s.ctypes.data, G, N, K, w.ctypes.data)
+    rc = lib.oracle_mxfp4_dequantize(q.ctypes.data, s.ctypes.data, G, N, K, w.ctypes.data, _threads())
     if rc:
         raise ValueError(f"oracle_mxfp4_dequantize failed ({rc}): a value is not a finite bf16 number")
     return w[0] if squeeze else w

@@ -312,69 +312,127 @@ static int e2m1_nearest(double p) {
     return best;
 }
 
+/* Rows [first, last) of a [G*N][K] weight tensor, shared by the threads that encode or decode it. */
+typedef struct {
+    const uint16_t* w;
+    uint16_t* w_out;
+    const uint8_t* qin;
+    const uint8_t* sin;
+    uint8_t* q;
+    uint8_t* s;
+    int N, K;
+    long first, last;
+    int status;
+} mx_job_t;
+
+static void* mx_quantize_rows(void* p) {
+    mx_job_t* J = (mx_job_t*)p;
+    const int N = J->N, K = J->K, nb = K / 32;
+    for (long row = J->first; row < J->last; ++row) {
+        const long g = row / N, n = row % N;
+        for (int b = 0; b < nb; ++b) {
+            const uint16_t* v = J->w + (size_t)row * K + (size_t)b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(bf16_to_double(v[i])));
+            int shared = -127;
+            if (amax > 0.0) {
+                int ex;
+                frexp(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1): floor(log2(amax)) = ex - 1 */
+                shared = ex - 1 - 2;
+                if (shared < -127) shared = -127;
+                if (shared > 127) shared = 127;
+            }
+            int code[32];
+            for (int i = 0; i < 32; ++i) {
+                const double p = fabs(bf16_to_double(v[i])) / ldexp(1.0, shared);
+                code[i] = e2m1_nearest(p) | ((v[i] >> 15) ? 8 : 0);
+            }
+            uint8_t* out = J->q + (size_t)row * (size_t)(K / 2) + (size_t)b * 16;
+            for (int j = 0; j < 4; ++j) {
+                uint32_t word = 0;
+                for (int i = 0; i < 4; ++i) {
+                    word |= (uint32_t)code[8 * j + 2 * i] << (4 * i);
+                    word |= (uint32_t)code[8 * j + 2 * i + 1] << (16 + 4 * i);
+                }
+                for (int byte = 0; byte < 4; ++byte) out[4 * j + byte] = (uint8_t)(word >> (8 * byte));
+            }
+            J->s[((size_t)g * nb + b) * N + n] = (uint8_t)(shared + 127);
+        }
+    }
+    return NULL;
+}
+
+static void* mx_dequantize_rows(void* p) {
+    mx_job_t* J = (mx_job_t*)p;
+    const int N = J->N, K = J->K, nb = K / 32;
+    for (long row = J->first; row < J->last; ++row) {
+        const long g = row / N, n = row % N;
+        for (int k = 0; k < K; ++k) {
+            const int b = k / 32, j = (k % 32) / 8, e = k % 8;
+            const uint8_t* blk = J->qin + (size_t)row * (size_t)(K / 2) + (size_t)b * 16 + 4 * j;
+            const uint32_t word = (uint32_t)blk[0] | ((uint32_t)blk[1] << 8) | ((uint32_t)blk[2] << 16) |
+                                  ((uint32_t)blk[3] << 24);
+            const int nib = (e % 2 == 0) ? e / 2 : 4 + e / 2;
+            const int code = (int)((word >> (4 * nib)) & 15u);
+            const int sc = J->sin[((size_t)g * nb + b) * N + n];
+            if (sc == 255) { J->status = -1; return NULL; }
+            const double val = oracle_e2m1_value(code) * ldexp(1.0, sc - 127);
+            const float fv = (float)val;
+            if ((double)fv != val || isinf(fv)) { J->status = -1; return NULL; }
+            uint32_t u;
+            memcpy(&u, &fv, 4);
+            if (u & 0xFFFFu) { J->status = -1; return NULL; }
+            J->w_out[(size_t)row * K + k] = (uint16_t)(u >> 16);
+        }
+    }
+    return NULL;
+}
+
+/* Split rows over host threads (the arithmetic per row is the same whatever the split). */
+static int mx_run(void* (*fn)(void*), mx_job_t proto, long rows, int nthreads) {
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nthreads > rows) nthreads = rows > 0 ? (int)rows : 1;
+    mx_job_t jobs[256];
+    pthread_t th[256];
+    char started[256];
+    const long per = (rows + nthreads - 1) / nthreads;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i] = proto;
+        jobs[i].first = i * per;
+        jobs[i].last = (i + 1) * per < rows ? (i + 1) * per : rows;
+        jobs[i].status = 0;
+        started[i] = 0;
+        if (jobs[i].first >= jobs[i].last) continue;
+        if (nthreads == 1 || pthread_create(&th[i], NULL, fn, &jobs[i]) != 0)
+            fn(&jobs[i]);
+        else
+            started[i] = 1;
+    }
+    int status = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        if (started[i]) pthread_join(th[i], NULL);
+        if (jobs[i].status) status = jobs[i].status;
+    }
+    return status;
+}
+
 /* w [G][N][K] bf16 -> codes q [G][N][K/2], scales s [G][K/32][N]. Per block of 32: the shared exponent is
    floor(log2(max |v|)) minus 2 (the exponent of E2M1's largest magnitude, 6 = 1.5 * 2^2), each element is
    v / 2^shared rounded to the nearest E2M1 value. Returns 0, or -1 when K is not a multiple of 32. */
-int oracle_mxfp4_quantize(const uint16_t* w, int G, int N, int K, uint8_t* q, uint8_t* s) {
+int oracle_mxfp4_quantize(const uint16_t* w, int G, int N, int K, uint8_t* q, uint8_t* s, int nthreads) {
     if (K % 32 != 0 || G < 0 || N < 0) return -1;
-    const int nb = K / 32;
-    for (long g = 0; g < G; ++g)
-        for (long n = 0; n < N; ++n)
-            for (int b = 0; b < nb; ++b) {
-                const uint16_t* v = w + ((size_t)g * N + n) * K + (size_t)b * 32;
-                double amax = 0.0;
-                for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(bf16_to_double(v[i])));
-                int shared = -127;
-                if (amax > 0.0) {
-                    int ex;
-                    frexp(amax, &ex); /* amax = m * 2^ex, m in [0.5, 1): floor(log2(amax)) = ex - 1 */
-                    shared = ex - 1 - 2;
-                    if (shared < -127) shared = -127;
-                    if (shared > 127) shared = 127;
-                }
-                int code[32];
-                for (int i = 0; i < 32; ++i) {
-                    const double p = fabs(bf16_to_double(v[i])) / ldexp(1.0, shared);
-                    code[i] = e2m1_nearest(p) | ((v[i] >> 15) ? 8 : 0);
-                }
-                uint8_t* out = q + ((size_t)g * N + n) * (size_t)(K / 2) + (size_t)b * 16;
-                for (int j = 0; j < 4; ++j) {
-                    uint32_t word = 0;
-                    for (int i = 0; i < 4; ++i) {
-                        word |= (uint32_t)code[8 * j + 2 * i] << (4 * i);
-                        word |= (uint32_t)code[8 * j + 2 * i + 1] << (16 + 4 * i);
-                    }
-                    for (int byte = 0; byte < 4; ++byte) out[4 * j + byte] = (uint8_t)(word >> (8 * byte));
-                }
-                s[((size_t)g * nb + b) * N + n] = (uint8_t)(shared + 127);
-            }
-    return 0;
+    mx_job_t J = {0};
+    J.w = w; J.q = q; J.s = s; J.N = N; J.K = K;
+    return mx_run(mx_quantize_rows, J, (long)G * N, nthreads);
 }
 
 /* Codes and scales -> the weights they encode, as bf16 bits: code value * 2^(scale - 127). Every such value
    with scale <= 252 is exactly a bf16 number; returns -1 for a value that is not (overflow, scale 255),
    -2 for a bad K. */
-int oracle_mxfp4_dequantize(const uint8_t* q, const uint8_t* s, int G, int N, int K, uint16_t* w) {
+int oracle_mxfp4_dequantize(const uint8_t* q, const uint8_t* s, int G, int N, int K, uint16_t* w, int nthreads) {
     if (K % 32 != 0 || G < 0 || N < 0) return -2;
-    const int nb = K / 32;
-    for (long g = 0; g < G; ++g)
-        for (long n = 0; n < N; ++n)
-            for (int k = 0; k < K; ++k) {
-                const int b = k / 32, j = (k % 32) / 8, e = k % 8;
-                const uint8_t* blk = q + ((size_t)g * N + n) * (size_t)(K / 2) + (size_t)b * 16 + 4 * j;
-                const uint32_t word = (uint32_t)blk[0] | ((uint32_t)blk[1] << 8) | ((uint32_t)blk[2] << 16) |
-                                      ((uint32_t)blk[3] << 24);
-                const int nib = (e % 2 == 0) ? e / 2 : 4 + e / 2;
-                const int code = (int)((word >> (4 * nib)) & 15u);
-                const int sc = s[((size_t)g * nb + b) * N + n];
-                if (sc == 255) return -1;
-                const double val = oracle_e2m1_value(code) * ldexp(1.0, sc - 127);
-                const float fv = (float)val;
-                if ((double)fv != val || isinf(fv)) return -1;
-                uint32_t u;
-                memcpy(&u, &fv, 4);
-                if (u & 0xFFFFu) return -1;
-                w[((size_t)g * N + n) * K + k] = (uint16_t)(u >> 16);
-            }
-    return 0;
+    mx_job_t J = {0};
+    J.qin = q; J.sin = s; J.w_out = w; J.N = N; J.K = K;
+    return mx_run(mx_dequantize_rows, J, (long)G * N, nthreads);
 }

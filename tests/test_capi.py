@@ -62,6 +62,11 @@ def test_invalid_arguments_rejected_before_any_launch(native):
     # split router: no pieces; E out of range for the split
     assert lib.moe_route_topk_split(16, 16, null, null, 4, 8, 8, 2, 0, 16, 16, 16, null) == native.MOE_ERR_INVALID_ARG
     assert lib.moe_router_split_weights(16, 0, 8, 16, null) == native.MOE_ERR_INVALID_ARG
+    # MXFP4: K not a multiple of 32; f not a multiple of 32; null scales; misaligned codes
+    assert lib.moe_mxfp4_quantize(16, 1, 8, 48, 16, 16, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_gateup_mxfp4(16, 16, 16, 16, 1, 8, 64, 40, 16, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_down_mxfp4(16, 16, null, 16, 1, 8, 64, 64, 16, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_down_mxfp4(16, 24, 16, 16, 1, 8, 64, 64, 16, null) == native.MOE_ERR_INVALID_ARG
     # missing workspace
     st = lib.moe_permute(null, 16, 64, 0, 8, 2, 16, 16, 16, 16, null, null, 0, null)
     assert st == native.MOE_ERR_WORKSPACE

@@ -4,6 +4,9 @@ Inputs come from the seeded generator; expected values come only from the oracle
 (routing indices, counts, offsets, permutation, gathered rows) must match bit for bit; the layer output
 must meet the bar in gpu_util (per element and relative Frobenius).
 """
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -364,7 +367,7 @@ def test_identical_experts_equal_dense_swiglu():
 # ---- full layer at the benchmark's sizes -------------------------------------------------------------
 
 SAMPLE = {"tiny": None, "gpt-oss-20b-prefill": 48, "mixtral-8x7b-prefill": 24, "zipf-128e": 48,
-          "decode-256e-shared": 8}
+          "decode-256e-shared": 8, "decode-256e-shared-mxfp4": 8}
 
 
 def _sample_tokens(ref, n, rng):
@@ -379,13 +382,13 @@ def _sample_tokens(ref, n, rng):
     return np.array(sorted(toks), dtype=np.int32)
 
 
-@pytest.mark.parametrize("name", CONFIGS)
+@pytest.mark.parametrize("name", CONFIGS + ["decode-256e-shared-mxfp4"])
 def test_full_layer_matches_oracle(name):
     wl = synth.workload(name)
     ref = layer_ref(name)
     inp = synth.device_inputs(wl)
     layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
-                   inp["w_gateup_shared"], inp["w_down_shared"])
+                   inp["w_gateup_shared"], inp["w_down_shared"], weights=wl.weights)
     y = layer(inp["x"]).clone()
     torch.cuda.synchronize()
     assert N.get_device_error() == 0
@@ -403,6 +406,156 @@ def test_full_layer_matches_oracle(name):
     # run again: bitwise identical (deterministic path)
     y2 = layer(inp["x"])
     assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+
+
+# ---- MXFP4 expert weights -----------------------------------------------------------------------------
+
+def _gpu_quantize(w_bits):
+    w = to_dev_bf16(w_bits)
+    G, Nr, K = w.shape
+    q = torch.empty(G, Nr, K // 2, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(G, K // 32, Nr, dtype=torch.uint8, device="cuda")
+    N.mxfp4_quantize(w, q, sc)
+    return q, sc
+
+
+def test_mxfp4_quantize_bit_exact():
+    """The encoder against the oracle, byte for byte: normal weights, zero blocks, signed zeros, bf16 subnormals,
+    huge magnitudes, the golden tie cases, and every code and scale range through a decode-encode round trip."""
+    rng = np.random.default_rng(30)
+    cases = []
+    w = synth.normal_bf16(30, 2, 0, 3 * 200 * 96, 0.02).reshape(3, 200, 96)
+    w[0, 0, :32] = 0
+    w[0, 1, :32] = 0x8000
+    w[1, 2, 32:64] = (rng.integers(1, 128, 32) | (rng.integers(0, 2, 32) << 15)).astype(np.uint16)  # subnormals
+    w[2, 3, 64:] = synth.f32_to_bf16_bits(rng.standard_normal(32).astype(np.float32) * 3e37)
+    cases.append(w)
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "mxfp4_e2m1.json")))["rounding"]
+    vals = [(-0.0 if v == "-0" else float(v)) for v in g["inputs"]] + [0.0] * (32 - len(g["inputs"]))
+    cases.append(synth.f32_to_bf16_bits(np.array(vals, dtype=np.float32)).reshape(1, 1, 32))
+    codes = rng.integers(0, 16, size=(2, 48, 128))
+    codes[..., ::32] = rng.choice([6, 7, 14, 15], size=(2, 48, 4))
+    scales = rng.integers(0, 253, size=(2, 4, 48)).astype(np.uint8)
+    cases.append(oracle.mxfp4_dequantize(_pack_codes_layout(codes), scales))  # exact E2M1 values times scales
+    cases.append(synth.normal_bf16(31, 3, 0, 4 * 7168 * 64, 0.02).reshape(4, 64, 7168))
+    for w in cases:
+        q, sc = _gpu_quantize(w)
+        rq, rs = oracle.mxfp4_quantize(w)
+        np.testing.assert_array_equal(q.cpu().numpy(), rq)
+        np.testing.assert_array_equal(sc.cpu().numpy(), rs)
+    assert N.get_device_error() == 0
+
+
+def _pack_codes_layout(codes):
+    c = np.asarray(codes, dtype=np.uint32)
+    *lead, K = c.shape
+    c = c.reshape(*lead, K // 8, 4, 2)
+    shifts = (np.arange(4, dtype=np.uint32) * 4)[:, None] + np.array([0, 16], dtype=np.uint32)[None, :]
+    return (c << shifts).sum(axis=(-1, -2)).astype("<u4").view(np.uint8).reshape(*lead, K // 2)
+
+
+def _gpu_experts_mxfp4(x_bits, gu_bits, dn_bits, idx, w32, shared=None):
+    """permute -> MXFP4 gate|up -> MXFP4 down -> combine on the GPU, weights encoded on the GPU."""
+    T, d = x_bits.shape
+    E, two_f, _ = gu_bits.shape
+    f = two_f // 2
+    R = T * idx.shape[1]
+    x, p = _gpu_permute(x_bits, idx, E)
+    qgu, sgu = _gpu_quantize(gu_bits)
+    qdn, sdn = _gpu_quantize(dn_bits)
+    h = torch.empty(R, f, dtype=torch.bfloat16, device="cuda")
+    y_perm = torch.empty(R, d, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    N.grouped_gemm_gateup_mxfp4(p["x_perm"], qgu, sgu, p["offsets"], h)
+    N.grouped_gemm_down_mxfp4(h, qdn, sdn, p["offsets"], y_perm)
+    sh = None
+    if shared is not None:
+        fs = shared[0].shape[0] // 2
+        q1, s1 = _gpu_quantize(shared[0][None])
+        q2, s2 = _gpu_quantize(shared[1][None])
+        so = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+        hs = torch.empty(T, fs, dtype=torch.bfloat16, device="cuda")
+        sh = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        N.grouped_gemm_gateup_mxfp4(x, q1, s1, so, hs)
+        N.grouped_gemm_down_mxfp4(hs, q2, s2, so, sh)
+    N.unpermute_combine(y_perm, p["inv_perm"], torch.from_numpy(w32).cuda(), sh, y)
+    assert N.get_device_error() == 0
+    return bf16_to_host_f32(y), p, h
+
+
+MXFP4_RAGGED = [
+    # (name, counts per expert, d, f): token tiles of 16 (M <= 8 G), 32 (M <= 24 G) and 64 rows, groups larger than
+    # the tile, empty groups, weight blocks cut by f or d (not multiples of 128), K tails inside the last 256-stage
+    ("nt16_decode_like", [2, 0, 1, 3, 2, 0, 5, 16, 17, 1], 256, 128),
+    ("nt16_tails", [1, 0, 9, 0, 2, 33], 288, 96),
+    ("nt32_ragged", [20, 0, 31, 33, 1, 40], 160, 224),
+    ("nt64_one_group", [200], 352, 160),
+    ("nt64_many", [0, 65, 64, 130, 7], 512, 544),
+]
+
+
+@pytest.mark.parametrize("name,counts,d,f", MXFP4_RAGGED, ids=[r[0] for r in MXFP4_RAGGED])
+def test_mxfp4_ragged_groups_match_oracle(name, counts, d, f):
+    rng = np.random.default_rng(32)
+    E = len(counts)
+    idx = _routing_with_counts(counts, 1, rng)
+    T = idx.shape[0]
+    x = synth.normal_bf16(33, 0, 0, T * d, 1.0).reshape(T, d)
+    gu = synth.normal_bf16(33, 2, 0, E * 2 * f * d, 0.05).reshape(E, 2 * f, d)
+    dn = synth.normal_bf16(33, 3, 0, E * d * f, 0.05).reshape(E, d, f)
+    w = np.ones((T, 1), dtype=np.float32)
+    y, p, _ = _gpu_experts_mxfp4(x, gu, dn, idx, w)
+    np.testing.assert_array_equal(p["counts"].cpu().numpy(), counts)
+    gu_dq = oracle.mxfp4_round_trip(gu)
+    dn_dq = oracle.mxfp4_round_trip(dn)
+    ref = oracle.moe_tokens(x, list(gu_dq), list(dn_dq), idx, w.astype(np.float64), np.arange(T))
+    check_close(y, ref, name)
+
+
+def test_mxfp4_large_scales_and_shared_expert():
+    """Scale codes above 128 (the decoder's two-step multiply) next to ordinary ones, k = 2 routing with
+    weights, and an MXFP4 shared expert; the encoded weights are exact E2M1 values times the scales."""
+    rng = np.random.default_rng(34)
+    T, d, f, E, k, fs = 90, 256, 160, 6, 2, 96
+    idx = np.stack([rng.choice(E, size=k, replace=False) for _ in range(T)]).astype(np.int32)
+    wts = rng.dirichlet(np.ones(k), size=T).astype(np.float32)
+    x = synth.f32_to_bf16_bits((rng.standard_normal((T, d)) * 1e-3).astype(np.float32))
+
+    def encoded(shape, lo, hi):
+        G, Nr, K = shape
+        codes = rng.integers(0, 16, size=shape)
+        codes[..., ::32] = rng.choice([6, 7, 14, 15], size=(G, Nr, K // 32))
+        scales = rng.integers(lo, hi, size=(G, K // 32, Nr)).astype(np.uint8)
+        return oracle.mxfp4_dequantize(_pack_codes_layout(codes), scales)
+
+    gu = encoded((E, 2 * f, d), 100, 140)   # weights up to 6 * 2^12
+    dn = encoded((E, d, f), 110, 131)
+    sgu = encoded((1, 2 * fs, d), 115, 135)[0]
+    sdn = encoded((1, d, fs), 118, 130)[0]
+    y, _, _ = _gpu_experts_mxfp4(x, gu, dn, idx, wts, shared=(sgu, sdn))
+    # the weights are their own encoding, so the oracle uses them as they are
+    ref = oracle.moe_tokens(x, list(gu), list(dn), idx, wts.astype(np.float64), np.arange(T), sgu, sdn)
+    check_close(y, ref, "mxfp4 large scales + shared")
+
+
+def test_mxfp4_gateup_matches_bf16_gemm_on_decoded_weights():
+    """Decode-shaped problem: h from the MXFP4 kernel equals h from the bf16 grouped GEMM given the decoded
+    weights, up to fp32 summation order (both round h to bf16 from fp32 sums of the same products)."""
+    rng = np.random.default_rng(35)
+    counts = [int(c) for c in rng.multinomial(512, np.ones(256) / 256)]
+    idx = _routing_with_counts(counts, 1, rng)
+    T, d, f = idx.shape[0], 1024, 256
+    x_bits = synth.normal_bf16(35, 0, 0, T * d, 1.0).reshape(T, d)
+    gu = synth.normal_bf16(35, 2, 0, 256 * 2 * f * d, 0.02).reshape(256, 2 * f, d)
+    _, p = _gpu_permute(x_bits, idx, 256)
+    q, sc = _gpu_quantize(gu)
+    h4 = torch.empty(T, f, dtype=torch.bfloat16, device="cuda")
+    N.grouped_gemm_gateup_mxfp4(p["x_perm"], q, sc, p["offsets"], h4)
+    hb = torch.empty(T, f, dtype=torch.bfloat16, device="cuda")
+    N.grouped_gemm_gateup(p["x_perm"], to_dev_bf16(oracle.mxfp4_round_trip(gu)), p["offsets"], hb)
+    a, b = bf16_to_host_f32(h4).astype(np.float64), bf16_to_host_f32(hb).astype(np.float64)
+    assert np.abs(a - b).max() <= 2 ** -7 * np.abs(b).max() + 1e-6
+    assert N.get_device_error() == 0
 
 
 def test_layer_at_maximum_sizes():

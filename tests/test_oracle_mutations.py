@@ -44,8 +44,8 @@ MUTATIONS = {
     "mxfp4_scale_ceil_not_floor": ("shared = ex - 1 - 2;", "shared = ex - 2;"),
     "mxfp4_sign_dropped": ("e2m1_nearest(p) | ((v[i] >> 15) ? 8 : 0)", "e2m1_nearest(p)"),
     "mxfp4_natural_nibble_order": (
-        "word |= (uint32_t)code[8 * j + 2 * i] << (4 * i);\n                        word |= (uint32_t)code[8 * j + 2 * i + 1] << (16 + 4 * i);",
-        "word |= (uint32_t)code[8 * j + 2 * i] << (8 * i);\n                        word |= (uint32_t)code[8 * j + 2 * i + 1] << (8 * i + 4);"),
+        "word |= (uint32_t)code[8 * j + 2 * i] << (4 * i);\n                    word |= (uint32_t)code[8 * j + 2 * i + 1] << (16 + 4 * i);",
+        "word |= (uint32_t)code[8 * j + 2 * i] << (8 * i);\n                    word |= (uint32_t)code[8 * j + 2 * i + 1] << (8 * i + 4);"),
     "mxfp4_scale_layout_row_major": ("s[((size_t)g * nb + b) * N + n] = (uint8_t)(shared + 127);",
                                      "s[((size_t)g * N + n) * nb + b] = (uint8_t)(shared + 127);"),
     "mxfp4_zero_block_scale_max": ("int shared = -127;", "int shared = 127;"),
