@@ -37,6 +37,25 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// As mbar_wait_bounded, for a role that is off the critical path (a warp waiting a whole tile for its turn): it
+// sleeps `sleep_ns` between polls instead of spinning, leaving issue slots to the warps that do the work.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  unsigned sleep_ns) {
+    const uint32_t addr = smem_u32(bar);
+    if (mbar_try_wait(addr, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(addr, parity)) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            flag_error(MOE_DEVERR_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
 // Bounded wait without an abort flag (used while draining on the way out).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     const uint32_t addr = smem_u32(bar);

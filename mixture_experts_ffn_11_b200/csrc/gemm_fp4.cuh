@@ -127,30 +127,29 @@ __device__ __forceinline__ uint32_t bf16x2_pow2(int e) {
 // 2^(126 + sc - 127) = 2^(sc - 1) then gives the weight exactly; for sc > 128 that factor is not a bf16 number
 // and the multiply is split in two. The word layout puts element 2i in nibble i and element 2i+1 in nibble
 // i+4, so the pair (2i, 2i+1) needs the same shift for both halves of the output word.
-__device__ __forceinline__ void mxfp4_decode_unit(const uint4 c, int sc, uint32_t* out) {
+__device__ __forceinline__ void mxfp4_decode_patterns(const uint4 c, uint32_t* out) {
     constexpr uint32_t MAG = 0x01C001C0u, SGN = 0x80008000u;
     const uint32_t xs[4] = {c.x, c.y, c.z, c.w};
-    uint32_t f1, f2 = 0;
-    if (sc <= 128) {
-        f1 = bf16x2_pow2(sc - 1);
-    } else {
-        f1 = bf16x2_pow2(126);
-        f2 = bf16x2_pow2(sc - 127);
-    }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t x = xs[j];
-        uint32_t p[4];
-        p[0] = ((x << 6) & MAG) | ((x << 12) & SGN);
-        p[1] = ((x << 2) & MAG) | ((x << 8) & SGN);
-        p[2] = ((x >> 2) & MAG) | ((x << 4) & SGN);
-        p[3] = ((x >> 6) & MAG) | (x & SGN);
+        out[4 * j + 0] = ((x << 6) & MAG) | ((x << 12) & SGN);
+        out[4 * j + 1] = ((x << 2) & MAG) | ((x << 8) & SGN);
+        out[4 * j + 2] = ((x >> 2) & MAG) | ((x << 4) & SGN);
+        out[4 * j + 3] = ((x >> 6) & MAG) | (x & SGN);
+    }
+}
+
+__device__ __forceinline__ void mxfp4_decode_unit(const uint4 c, int sc, uint32_t* out) {
+    mxfp4_decode_patterns(c, out);
+    if (sc <= 128) {  // one branch per 32 weights, uniform across the warp for realistic scales
+        const uint32_t f1 = bf16x2_pow2(sc - 1);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t r = bf16x2_mul(p[i], f1);
-            if (sc > 128) r = bf16x2_mul(r, f2);
-            out[4 * j + i] = r;
-        }
+        for (int i = 0; i < 16; ++i) out[i] = bf16x2_mul(out[i], f1);
+    } else {
+        const uint32_t f1 = bf16x2_pow2(126), f2 = bf16x2_pow2(sc - 127);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) out[i] = bf16x2_mul(bf16x2_mul(out[i], f1), f2);
     }
 }
 
@@ -307,7 +306,7 @@ __global__ void __launch_bounds__(GF_THREADS, 1)
             const int row0 = s_off[g] + tb * NT;
             const int wrow = wb * GF_BM;
             for (int ks = 0; ks < KS; ++ks) {
-                if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
+                if (lane == 0) ok = mbar_wait_backoff(&empty_bar[stage], phase ^ 1u, abort_flag, 64);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 if (lane == 0) {
@@ -345,7 +344,7 @@ __global__ void __launch_bounds__(GF_THREADS, 1)
         uint32_t phase = 0, slot_phase = 0, acc_phase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-            if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, abort_flag);
+            if (lane == 0) ok = mbar_wait_backoff(&tempty_bar[acc], acc_phase ^ 1u, abort_flag, 64);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
@@ -465,7 +464,7 @@ __global__ void __launch_bounds__(GF_THREADS, 1)
             const int row0 = s_off[g] + tb * NT;
             const int rows = min(NT, s_off[g + 1] - row0);
             const int n = wb * GF_BM + r;  // output column of this thread
-            if (lane == 0) ok = mbar_wait_bounded(&tfull_bar[acc], acc_phase, abort_flag);
+            if (lane == 0) ok = mbar_wait_backoff(&tfull_bar[acc], acc_phase, abort_flag, 256);
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after_sync();
