@@ -25,6 +25,11 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
                  a hand-packed word of the documented nibble layout
   mxfp4_dequantize pinned: inverse of the above on every code and scale range;
                  numpy decode of the documented layout
+  moe_backward   pinned: torch fp64 autograd of the same per-token loop (dx, every
+                 weight gradient, routing-weight gradients, shared expert); central
+                 differences of moe_tokens in the routing weights; linearity in dy
+  router_backward pinned: torch fp64 autograd of each mode's weight formula and of the
+                 router projection; central differences of topk's weights in the logits
 """
 from __future__ import annotations
 
@@ -67,6 +72,10 @@ def load(path: str | None = None):
     lib.oracle_mxfp4_quantize.restype = ci
     lib.oracle_mxfp4_dequantize.argtypes = [vp, vp, ci, ci, ci, vp, ci]
     lib.oracle_mxfp4_dequantize.restype = ci
+    lib.oracle_moe_backward.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, ci, vp, vp, vp, vp, vp, vp]
+    lib.oracle_moe_backward.restype = ci
+    lib.oracle_router_backward.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
+    lib.oracle_router_backward.restype = ci
     return lib
 
 
@@ -234,6 +243,75 @@ def mxfp4_round_trip(w_bits: np.ndarray, lib=None) -> np.ndarray:
     """The weights an MXFP4 layer computes with: bf16 weights encoded, then decoded."""
     q, s = mxfp4_quantize(w_bits, lib=lib)
     return mxfp4_dequantize(q, s, lib=lib)
+
+
+def moe_backward(x_bits, expert_gateup, expert_down, idx, w, dy, shared_gateup=None, shared_down=None, lib=None):
+    """Gradients of the expert part of the layer (section "Training MoEs with Transformers" trains through the
+    same expert backend): given dy = d loss / d out for every token, returns a dict with dx [T, d], dw_gateup
+    [E, 2f, d], dw_down [E, d, f], dw [T, k] (routing weights) and, with a shared expert, its two weight
+    gradients. Weights as for moe_tokens (bf16 bits, every expert that a token selects must be given). fp64."""
+    lib = lib or _L()
+    x = _c(x_bits, np.uint16)
+    T, d = x.shape
+    E = len(expert_gateup)
+    ix = _c(idx, np.int32)
+    k = ix.shape[1]
+    ww = _c(w, np.float64)
+    g = _c(dy, np.float64)
+    f = next(a.shape[0] // 2 for a in expert_gateup if a is not None)
+    keep = []
+    gu_p, dn_p = (ctypes.c_void_p * E)(), (ctypes.c_void_p * E)()
+    dgu_p, ddn_p = (ctypes.c_void_p * E)(), (ctypes.c_void_p * E)()
+    dgu = np.zeros((E, 2 * f, d))
+    ddn = np.zeros((E, d, f))
+    for e in range(E):
+        if expert_gateup[e] is None or expert_down[e] is None:
+            continue
+        gu, dn = _c(expert_gateup[e], np.uint16), _c(expert_down[e], np.uint16)
+        keep += [gu, dn]
+        gu_p[e], dn_p[e] = gu.ctypes.data, dn.ctypes.data
+        dgu_p[e], ddn_p[e] = dgu[e].ctypes.data, ddn[e].ctypes.data
+    sgu = _c(shared_gateup, np.uint16) if shared_gateup is not None else None
+    sdn = _c(shared_down, np.uint16) if shared_down is not None else None
+    fs = sgu.shape[0] // 2 if sgu is not None else 0
+    dsgu = np.zeros((2 * fs, d)) if fs else None
+    dsdn = np.zeros((d, fs)) if fs else None
+    dx = np.empty((T, d))
+    dw = np.empty((T, k))
+    rc = lib.oracle_moe_backward(x.ctypes.data, T, d, f, E, k, gu_p, dn_p, ix.ctypes.data, ww.ctypes.data, g.ctypes.data,
+                                 sgu.ctypes.data if fs else None, sdn.ctypes.data if fs else None, fs,
+                                 dx.ctypes.data, dgu_p, ddn_p, dw.ctypes.data,
+                                 dsgu.ctypes.data if fs else None, dsdn.ctypes.data if fs else None)
+    if rc:
+        raise ValueError(f"oracle_moe_backward failed ({rc})")
+    out = {"dx": dx, "dw_gateup": dgu, "dw_down": ddn, "dw": dw}
+    if fs:
+        out["dw_gateup_shared"], out["dw_down_shared"] = dsgu, dsdn
+    return out
+
+
+def router_backward(x_bits, w_router, logits_f32, idx, w, dw, mode: str, lib=None):
+    """Router gradients with the top-k selection held fixed: from dw = d loss / d w (routing weights computed by
+    topk from these fp32 logits), returns dlogits [T, E], dw_router [E, d], dbias [E] and the router's share of
+    dx [T, d]. fp64."""
+    lib = lib or _L()
+    x = _c(x_bits, np.uint16)
+    T, d = x.shape
+    wr = _c(w_router, np.float32)
+    E = wr.shape[0]
+    l = _c(logits_f32, np.float32)
+    ix = _c(idx, np.int32)
+    k = ix.shape[1]
+    dl = np.empty((T, E))
+    dwr = np.empty((E, d))
+    db = np.empty(E)
+    dx = np.empty((T, d))
+    rc = lib.oracle_router_backward(x.ctypes.data, wr.ctypes.data, l.ctypes.data, T, d, E, k, ROUTE_MODES[mode],
+                                    ix.ctypes.data, _c(w, np.float64).ctypes.data, _c(dw, np.float64).ctypes.data,
+                                    dl.ctypes.data, dwr.ctypes.data, db.ctypes.data, dx.ctypes.data)
+    if rc:
+        raise ValueError(f"oracle_router_backward failed ({rc})")
+    return {"dlogits": dl, "dw_router": dwr, "dbias": db, "dx": dx}
 
 
 class LayerReference:

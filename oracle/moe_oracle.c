@@ -436,3 +436,166 @@ int oracle_mxfp4_dequantize(const uint8_t* q, const uint8_t* s, int G, int N, in
     J.qin = q; J.sin = s; J.w_out = w; J.N = N; J.K = K;
     return mx_run(mx_dequantize_rows, J, (long)G * N, nthreads);
 }
+
+/*
+ * Backward pass (training). The blog post's section "Training MoEs with Transformers" trains through the same
+ * grouped_mm expert backend; the gradients below are those of the per-token eager loop above, differentiated by
+ * hand, in fp64. Given dy[t] = d loss / d out[t]:
+ *   for each selected expert e of token t, routing weight w_tj:
+ *     g = Wg x, u = Wu x, a = silu(g), h = a * u, y_e = Wd h
+ *     dw[t][j]      = <dy[t], y_e>
+ *     dye           = w_tj * dy[t]
+ *     dh[n]         = sum_c dye[c] * Wd[c][n]
+ *     dWd[e][c][n] += dye[c] * h[n]
+ *     dg[n]         = dh[n] * u[n] * silu'(g[n]),  silu'(g) = s * (1 + g * (1 - s)),  s = 1 / (1 + e^-g)
+ *     du[n]         = dh[n] * a[n]
+ *     dx[t][i]     += sum_n dg[n] * Wg[n][i] + du[n] * Wu[n][i]
+ *     dWg[e][n][i] += dg[n] * x[i];  dWu[e][n][i] += du[n] * x[i]
+ *   the shared expert the same with weight 1 and no routing-weight gradient.
+ * Single-threaded (weight gradients accumulate over tokens); meant for small problems.
+ */
+static void swiglu_expert_backward(const uint16_t* xt, int d, int f, const uint16_t* wgu, const uint16_t* wd,
+                                   double scale, const double* dyt, double* dxt, double* dwgu, double* dwd,
+                                   double* dwt, double* g, double* u, double* h, double* dh) {
+    for (int n = 0; n < f; ++n) {
+        const uint16_t* gr = wgu + (size_t)n * d;
+        const uint16_t* ur = wgu + (size_t)(f + n) * d;
+        double gs = 0.0, us = 0.0;
+        for (int i = 0; i < d; ++i) {
+            const double xi = bf16_to_double(xt[i]);
+            gs += xi * bf16_to_double(gr[i]);
+            us += xi * bf16_to_double(ur[i]);
+        }
+        g[n] = gs;
+        u[n] = us;
+        h[n] = gs / (1.0 + exp(-gs)) * us;
+    }
+    if (dwt) { /* <dy, y_e>, y_e = Wd h */
+        double s = 0.0;
+        for (int c = 0; c < d; ++c) {
+            const uint16_t* dr = wd + (size_t)c * f;
+            double yc = 0.0;
+            for (int n = 0; n < f; ++n) yc += bf16_to_double(dr[n]) * h[n];
+            s += dyt[c] * yc;
+        }
+        *dwt = s;
+    }
+    for (int n = 0; n < f; ++n) dh[n] = 0.0;
+    for (int c = 0; c < d; ++c) {
+        const uint16_t* dr = wd + (size_t)c * f;
+        const double dyc = scale * dyt[c];
+        for (int n = 0; n < f; ++n) {
+            dh[n] += dyc * bf16_to_double(dr[n]);
+            dwd[(size_t)c * f + n] += dyc * h[n];
+        }
+    }
+    for (int n = 0; n < f; ++n) {
+        const double s = 1.0 / (1.0 + exp(-g[n]));
+        const double a = g[n] * s;
+        const double dg = dh[n] * u[n] * (s * (1.0 + g[n] * (1.0 - s)));
+        const double du = dh[n] * a;
+        const uint16_t* gr = wgu + (size_t)n * d;
+        const uint16_t* ur = wgu + (size_t)(f + n) * d;
+        double* dgr = dwgu + (size_t)n * d;
+        double* dur = dwgu + (size_t)(f + n) * d;
+        for (int i = 0; i < d; ++i) {
+            const double xi = bf16_to_double(xt[i]);
+            dxt[i] += dg * bf16_to_double(gr[i]) + du * bf16_to_double(ur[i]);
+            dgr[i] += dg * xi;
+            dur[i] += du * xi;
+        }
+    }
+}
+
+/* dx [T][d], dwgu: E pointers to [2f][d], dwd: E pointers to [d][f] (all fp64, zeroed here; NULL pointers for
+   experts no token selects), dw [T][k]; shared-expert gradients dwgu_s [2fs][d], dwd_s [d][fs] when given.
+   Returns 0, -1 on a bad argument or allocation failure, -2 when a selected expert has no weights. */
+int oracle_moe_backward(const uint16_t* x, int T, int d, int f, int E, int k, const uint16_t* const* wgu,
+                        const uint16_t* const* wd, const int32_t* idx, const double* w, const double* dy,
+                        const uint16_t* wgu_s, const uint16_t* wd_s, int fs, double* dx, double* const* dwgu,
+                        double* const* dwd, double* dw, double* dwgu_s, double* dwd_s) {
+    if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0 || k > E) return -1;
+    const int hf = f > fs ? f : fs;
+    double* g = (double*)malloc(sizeof(double) * (size_t)hf);
+    double* u = (double*)malloc(sizeof(double) * (size_t)hf);
+    double* h = (double*)malloc(sizeof(double) * (size_t)hf);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)hf);
+    if (!g || !u || !h || !dh) { free(g); free(u); free(h); free(dh); return -1; }
+    memset(dx, 0, sizeof(double) * (size_t)T * d);
+    for (int e = 0; e < E; ++e) {
+        if (dwgu[e]) memset(dwgu[e], 0, sizeof(double) * (size_t)2 * f * d);
+        if (dwd[e]) memset(dwd[e], 0, sizeof(double) * (size_t)d * f);
+    }
+    const int shared = wgu_s && wd_s && dwgu_s && dwd_s && fs > 0;
+    if (shared) {
+        memset(dwgu_s, 0, sizeof(double) * (size_t)2 * fs * d);
+        memset(dwd_s, 0, sizeof(double) * (size_t)d * fs);
+    }
+    int status = 0;
+    for (int t = 0; t < T && !status; ++t) {
+        const uint16_t* xt = x + (size_t)t * d;
+        const double* dyt = dy + (size_t)t * d;
+        double* dxt = dx + (size_t)t * d;
+        for (int j = 0; j < k; ++j) {
+            const int e = idx[(size_t)t * k + j];
+            if (e < 0 || e >= E || !wgu[e] || !wd[e] || !dwgu[e] || !dwd[e]) { status = -2; break; }
+            swiglu_expert_backward(xt, d, f, wgu[e], wd[e], w[(size_t)t * k + j], dyt, dxt, dwgu[e], dwd[e],
+                                   &dw[(size_t)t * k + j], g, u, h, dh);
+        }
+        if (shared && !status)
+            swiglu_expert_backward(xt, d, fs, wgu_s, wd_s, 1.0, dyt, dxt, dwgu_s, dwd_s, NULL, g, u, h, dh);
+    }
+    free(g); free(u); free(h); free(dh);
+    return status;
+}
+
+/* Router backward, the selection held fixed (top-k is piecewise constant in the logits, so no gradient flows
+   through it). From dw[t][j] = d loss / d w[t][j], with the weights w the forward computed from the fp32 logits:
+     top-k softmax and softmax -> top-k -> renorm (the same function of the selected logits):
+         dl[t][e_j] = w_j * (dw_j - sum_i w_i dw_i)
+     sigmoid -> top-k -> norm, s_j = sigmoid(l_j), S = sum_i s_i:
+         dl[t][e_j] = s_j * (1 - s_j) / S * (dw_j - sum_i w_i dw_i)
+     unselected experts: 0.
+   Then through l = x W_r^T + b: dW_r[e][i] = sum_t dl[t][e] x[t][i], dbias[e] = sum_t dl[t][e],
+   dx[t][i] = sum_e dl[t][e] W_r[e][i]. Outputs fp64, zeroed here. */
+int oracle_router_backward(const uint16_t* x, const float* w_router, const float* logits, int T, int d, int E, int k,
+                           int mode, const int32_t* idx, const double* w, const double* dw, double* dlogits,
+                           double* dw_router, double* dbias, double* dx) {
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || mode < 0 || mode > 2) return -1;
+    memset(dlogits, 0, sizeof(double) * (size_t)T * E);
+    memset(dw_router, 0, sizeof(double) * (size_t)E * d);
+    memset(dbias, 0, sizeof(double) * (size_t)E);
+    memset(dx, 0, sizeof(double) * (size_t)T * d);
+    for (int t = 0; t < T; ++t) {
+        const int32_t* it = idx + (size_t)t * k;
+        const double* wt = w + (size_t)t * k;
+        const double* dwt = dw + (size_t)t * k;
+        double dot = 0.0;
+        for (int j = 0; j < k; ++j) dot += wt[j] * dwt[j];
+        double S = 0.0;
+        if (mode == ORACLE_SIGMOID_TOPK_NORM)
+            for (int j = 0; j < k; ++j) S += 1.0 / (1.0 + exp(-(double)logits[(size_t)t * E + it[j]]));
+        for (int j = 0; j < k; ++j) {
+            const int e = it[j];
+            if (e < 0 || e >= E) return -2;
+            double g;
+            if (mode == ORACLE_SIGMOID_TOPK_NORM) {
+                const double s = 1.0 / (1.0 + exp(-(double)logits[(size_t)t * E + e]));
+                g = s * (1.0 - s) / S * (dwt[j] - dot);
+            } else {
+                g = wt[j] * (dwt[j] - dot);
+            }
+            dlogits[(size_t)t * E + e] = g;
+        }
+        for (int e = 0; e < E; ++e) {
+            const double g = dlogits[(size_t)t * E + e];
+            if (g == 0.0) continue;
+            dbias[e] += g;
+            for (int i = 0; i < d; ++i) {
+                dw_router[(size_t)e * d + i] += g * bf16_to_double(x[(size_t)t * d + i]);
+                dx[(size_t)t * d + i] += g * (double)w_router[(size_t)e * d + i];
+            }
+        }
+    }
+    return 0;
+}

@@ -401,6 +401,152 @@ def pin_mxfp4_error_bound(lib):
     assert (np.signbit(dq) == np.signbit(v)).all()
 
 
+# ---- backward (training) ---------------------------------------------------------------------------------
+
+def _torch_expert_grads(x_bits, gu, dn, idx, w, dy, sgu=None, sdn=None):
+    """Gradients of sum(dy * out) through the per-token layer, by torch fp64 autograd (an independent
+    derivation of what the oracle's hand-written backward computes)."""
+    import torch
+
+    X = torch.tensor(_f64(x_bits), requires_grad=True)
+    GU = [torch.tensor(_f64(m), requires_grad=True) for m in gu]
+    DN = [torch.tensor(_f64(m), requires_grad=True) for m in dn]
+    W = torch.tensor(np.asarray(w, np.float64), requires_grad=True)
+    SG = torch.tensor(_f64(sgu), requires_grad=True) if sgu is not None else None
+    SD = torch.tensor(_f64(sdn), requires_grad=True) if sdn is not None else None
+    T, k = idx.shape
+    f = gu[0].shape[0] // 2
+
+    def mlp(gum, dnm, xt, ff):
+        return dnm @ (torch.nn.functional.silu(gum[:ff] @ xt) * (gum[ff:] @ xt))
+
+    rows = []
+    for t in range(T):
+        acc = sum(W[t, j] * mlp(GU[idx[t, j]], DN[idx[t, j]], X[t], f) for j in range(k))
+        if SG is not None:
+            acc = acc + mlp(SG, SD, X[t], SG.shape[0] // 2)
+        rows.append(acc)
+    (torch.stack(rows) * torch.tensor(np.asarray(dy, np.float64))).sum().backward()
+    z = lambda P, ref: np.zeros(ref.shape) if P.grad is None else P.grad.numpy()
+    out = {"dx": X.grad.numpy(), "dw_gateup": np.stack([z(P, m) for P, m in zip(GU, gu)]),
+           "dw_down": np.stack([z(P, m) for P, m in zip(DN, dn)]), "dw": W.grad.numpy()}
+    if SG is not None:
+        out["dw_gateup_shared"], out["dw_down_shared"] = SG.grad.numpy(), SD.grad.numpy()
+    return out
+
+
+def pin_backward_autograd(lib):
+    rng = _rng(40)
+    T, d, f, E, k, fs = 6, 12, 8, 5, 2, 6
+    x, gu, dn, idx, w = _random_layer(rng, T, d, f, E, k)
+    sgu = _random_bf16(rng, (2 * fs, d), 0.3)
+    sdn = _random_bf16(rng, (d, fs), 0.3)
+    dy = rng.standard_normal((T, d))
+    got = oracle.moe_backward(x, gu, dn, idx, w, dy, sgu, sdn, lib=lib)
+    want = _torch_expert_grads(x, gu, dn, idx, w, dy, sgu, sdn)
+    for key in want:
+        np.testing.assert_allclose(got[key], want[key], rtol=1e-10, atol=1e-12, err_msg=key)
+
+
+def pin_backward_routing_weights_finite_difference(lib):
+    """The layer is linear in each routing weight, so a central difference of the forward oracle gives
+    d sum(dy * out) / d w[t, j] up to rounding."""
+    rng = _rng(41)
+    T, d, f, E, k = 5, 10, 6, 4, 3
+    x, gu, dn, idx, w = _random_layer(rng, T, d, f, E, k)
+    dy = rng.standard_normal((T, d))
+    got = oracle.moe_backward(x, gu, dn, idx, w, dy, lib=lib)["dw"]
+    h = 1e-3
+    for t in range(T):
+        for j in range(k):
+            wp, wm = w.copy(), w.copy()
+            wp[t, j] += h
+            wm[t, j] -= h
+            fp = oracle.moe_tokens(x, gu, dn, idx, wp, np.arange(T), lib=lib)
+            fm = oracle.moe_tokens(x, gu, dn, idx, wm, np.arange(T), lib=lib)
+            num = ((fp - fm) * dy).sum() / (2 * h)
+            assert abs(num - got[t, j]) <= 1e-9 * max(1.0, abs(num)), (t, j, num, got[t, j])
+
+
+def pin_backward_linear_in_dy(lib):
+    rng = _rng(42)
+    x, gu, dn, idx, w = _random_layer(rng, 4, 8, 8, 3, 2)
+    a, b = rng.standard_normal((4, 8)), rng.standard_normal((4, 8))
+    ga = oracle.moe_backward(x, gu, dn, idx, w, a, lib=lib)
+    gb = oracle.moe_backward(x, gu, dn, idx, w, b, lib=lib)
+    gab = oracle.moe_backward(x, gu, dn, idx, w, a + 2 * b, lib=lib)
+    for key in ga:
+        np.testing.assert_allclose(gab[key], ga[key] + 2 * gb[key], rtol=1e-10, atol=1e-12, err_msg=key)
+
+
+def _router_case(rng, T, E, k):
+    """fp32 logits whose k-th and (k+1)-th values are well apart (the selection survives small steps)."""
+    l = np.empty((T, E), dtype=np.float32)
+    for t in range(T):
+        v = rng.permutation(E).astype(np.float64) * 0.37 + rng.uniform(-0.05, 0.05, E)
+        l[t] = (v - v.mean()).astype(np.float32)
+    return l
+
+
+def pin_router_backward_autograd(lib):
+    import torch
+
+    rng = _rng(43)
+    T, d, E, k = 7, 16, 9, 3
+    x = _random_bf16(rng, (T, d), 1.0)
+    wr = (rng.standard_normal((E, d)) * 0.3).astype(np.float32)
+    bias = (rng.standard_normal(E) * 0.2).astype(np.float32)
+    for mode in ("topk_softmax", "softmax_topk_renorm", "sigmoid_topk_norm"):
+        X = torch.tensor(_f64(x), requires_grad=True)
+        WR = torch.tensor(wr.astype(np.float64), requires_grad=True)
+        B = torch.tensor(bias.astype(np.float64), requires_grad=True)
+        L = X @ WR.T + B
+        l32 = L.detach().numpy().astype(np.float32)
+        idx, w = oracle.topk(l32, k, mode, lib=lib)
+        dw = rng.standard_normal((T, k))
+        sel = L.gather(1, torch.tensor(idx, dtype=torch.int64))
+        if mode == "topk_softmax":
+            ww = torch.softmax(sel, dim=1)
+        elif mode == "softmax_topk_renorm":
+            p = torch.softmax(L, dim=1).gather(1, torch.tensor(idx, dtype=torch.int64))
+            ww = p / p.sum(1, keepdim=True)
+        else:
+            s = torch.sigmoid(sel)
+            ww = s / s.sum(1, keepdim=True)
+        L.retain_grad()
+        (ww * torch.tensor(dw)).sum().backward()
+        got = oracle.router_backward(x, wr, l32, idx, w, dw, mode, lib=lib)
+        # the oracle works from the fp32-rounded logits; autograd from the fp64 ones
+        np.testing.assert_allclose(got["dlogits"], L.grad.numpy(), rtol=1e-5, atol=1e-7, err_msg=mode)
+        np.testing.assert_allclose(got["dw_router"], WR.grad.numpy(), rtol=1e-5, atol=1e-6, err_msg=mode)
+        np.testing.assert_allclose(got["dbias"], B.grad.numpy(), rtol=1e-5, atol=1e-7, err_msg=mode)
+        np.testing.assert_allclose(got["dx"], X.grad.numpy(), rtol=1e-5, atol=1e-7, err_msg=mode)
+
+
+def pin_router_backward_finite_difference(lib):
+    """Central differences of topk's routing weights in each logit (selection unchanged by the step)."""
+    rng = _rng(44)
+    T, E, k = 5, 8, 3
+    l = _router_case(rng, T, E, k)
+    x = _random_bf16(rng, (T, 4), 1.0)
+    wr = np.zeros((E, 4), dtype=np.float32)
+    for mode in ("topk_softmax", "softmax_topk_renorm", "sigmoid_topk_norm"):
+        idx, w = oracle.topk(l, k, mode, lib=lib)
+        dw = rng.standard_normal((T, k))
+        got = oracle.router_backward(x, wr, l, idx, w, dw, mode, lib=lib)["dlogits"]
+        for t in range(T):
+            for e in range(E):
+                lp, lm = l.copy(), l.copy()
+                lp[t, e] += np.float32(1e-2)
+                lm[t, e] -= np.float32(1e-2)
+                ip, wp = oracle.topk(lp, k, mode, lib=lib)
+                im, wm = oracle.topk(lm, k, mode, lib=lib)
+                assert (ip == idx).all() and (im == idx).all()
+                step = float(lp[t, e]) - float(lm[t, e])
+                num = ((wp - wm) * dw).sum() / step
+                assert abs(num - got[t, e]) <= 2e-4 * max(1.0, abs(num)), (mode, t, e, num, got[t, e])
+
+
 PINS = [
     pin_router_logits_numpy,
     pin_topk_golden,
@@ -422,4 +568,9 @@ PINS = [
     pin_mxfp4_round_trip,
     pin_mxfp4_scale_closed_form,
     pin_mxfp4_error_bound,
+    pin_backward_autograd,
+    pin_backward_routing_weights_finite_difference,
+    pin_backward_linear_in_dy,
+    pin_router_backward_autograd,
+    pin_router_backward_finite_difference,
 ]

@@ -51,6 +51,19 @@ MUTATIONS = {
     "mxfp4_zero_block_scale_max": ("int shared = -127;", "int shared = 127;"),
     "mxfp4_decode_odd_even_swapped": ("const int nib = (e % 2 == 0) ? e / 2 : 4 + e / 2;",
                                       "const int nib = (e % 2 == 1) ? e / 2 : 4 + e / 2;"),
+    "backward_silu_prime_missing_term": ("(s * (1.0 + g[n] * (1.0 - s)))", "s"),
+    "backward_du_uses_gate": ("const double du = dh[n] * a;", "const double du = dh[n] * g[n];"),
+    "backward_routing_weight_dropped": ("const double dyc = scale * dyt[c];", "const double dyc = dyt[c];"),
+    "backward_dwd_transposed": ("dwd[(size_t)c * f + n] += dyc * h[n];", "dwd[(size_t)n * d + c] += dyc * h[n];"),
+    "backward_dx_missing_up_path": ("dxt[i] += dg * bf16_to_double(gr[i]) + du * bf16_to_double(ur[i]);",
+                                    "dxt[i] += dg * bf16_to_double(gr[i]);"),
+    "backward_dw_scaled_by_w": ("*dwt = s;", "*dwt = scale * s;"),
+    "backward_shared_expert_skipped": ("if (shared && !status)\n            swiglu_expert_backward(",
+                                       "if (0)\n            swiglu_expert_backward("),
+    "router_backward_softmax_not_centred": ("g = wt[j] * (dwt[j] - dot);", "g = wt[j] * dwt[j];"),
+    "router_backward_sigmoid_derivative_dropped": ("g = s * (1.0 - s) / S * (dwt[j] - dot);", "g = s / S * (dwt[j] - dot);"),
+    "router_backward_dx_uses_x": ("dx[(size_t)t * d + i] += g * (double)w_router[(size_t)e * d + i];",
+                                  "dx[(size_t)t * d + i] += g * bf16_to_double(x[(size_t)t * d + i]);"),
     "mxfp4_decode_scale_bias": ("oracle_e2m1_value(code) * ldexp(1.0, sc - 127)", "oracle_e2m1_value(code) * ldexp(1.0, sc - 126)"),
 }
 
