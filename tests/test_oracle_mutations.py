@@ -14,7 +14,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
 
 MUTATIONS = {
     "router_bias_dropped": ("if (bias) s += (double)bias[e];", ""),
-    "router_weight_transposed": ("(double)w_router[(size_t)e * d + i]", "(double)w_router[(size_t)i * E + e]"),
+    "router_weight_transposed": ("s += bf16_to_double(x[(size_t)t * d + i]) * (double)w_router[(size_t)e * d + i]",
+                                 "s += bf16_to_double(x[(size_t)t * d + i]) * (double)w_router[(size_t)i * E + e]"),
     "topk_tie_prefers_higher_id": ("l[e] > l[best]", "l[e] >= l[best]"),
     "softmax_missing_normalisation": ("for (int j = 0; j < k; ++j) wt[j] /= z;\n        } else if",
                                       "\n        } else if"),
@@ -28,10 +29,13 @@ MUTATIONS = {
                          "for (long a = R - 1; a >= 0; --a) {\n        int32_t r"),
     "silu_sign_flipped": ("h[n] = g / (1.0 + exp(-g)) * u;", "h[n] = g / (1.0 + exp(g)) * u;"),
     "silu_on_up_not_gate": ("h[n] = g / (1.0 + exp(-g)) * u;", "h[n] = u / (1.0 + exp(-u)) * g;"),
-    "gate_up_rows_swapped": ("const uint16_t* gr = wgu + (size_t)n * d;\n        const uint16_t* ur = wgu + (size_t)(f + n) * d;",
-                             "const uint16_t* gr = wgu + (size_t)(f + n) * d;\n        const uint16_t* ur = wgu + (size_t)n * d;"),
-    "gate_up_interleaved": ("const uint16_t* gr = wgu + (size_t)n * d;\n        const uint16_t* ur = wgu + (size_t)(f + n) * d;",
-                            "const uint16_t* gr = wgu + (size_t)(2 * n) * d;\n        const uint16_t* ur = wgu + (size_t)(2 * n + 1) * d;"),
+    # the forward loop's gate/up rows (the anchor runs into its accumulator declaration, which is unique)
+    "gate_up_rows_swapped": ("const uint16_t* gr = wgu + (size_t)n * d;\n        const uint16_t* ur = wgu + (size_t)(f + n) * d;\n        double g = 0.0, u = 0.0;",
+                             "const uint16_t* gr = wgu + (size_t)(f + n) * d;\n        const uint16_t* ur = wgu + (size_t)n * d;\n        double g = 0.0, u = 0.0;"),
+    "gate_up_interleaved": ("const uint16_t* gr = wgu + (size_t)n * d;\n        const uint16_t* ur = wgu + (size_t)(f + n) * d;\n        double g = 0.0, u = 0.0;",
+                            "const uint16_t* gr = wgu + (size_t)(2 * n) * d;\n        const uint16_t* ur = wgu + (size_t)(2 * n + 1) * d;\n        double g = 0.0, u = 0.0;"),
+    "backward_gate_up_rows_swapped": ("const uint16_t* gr = wgu + (size_t)n * d;\n        const uint16_t* ur = wgu + (size_t)(f + n) * d;\n        double* dgr",
+                                      "const uint16_t* gr = wgu + (size_t)(f + n) * d;\n        const uint16_t* ur = wgu + (size_t)n * d;\n        double* dgr"),
     "down_transposed": ("s += h[n] * bf16_to_double(dr[n]);", "s += h[n] * bf16_to_double(wd[(size_t)n * d + c]);"),
     "routing_weight_dropped": ("acc[c] += scale * s;", "acc[c] += s;"),
     "last_expert_dropped": ("for (int j = 0; j < J->k; ++j) {", "for (int j = 0; j < J->k - 1; ++j) {"),
