@@ -245,11 +245,12 @@ def mxfp4_round_trip(w_bits: np.ndarray, lib=None) -> np.ndarray:
     return mxfp4_dequantize(q, s, lib=lib)
 
 
-def moe_backward(x_bits, expert_gateup, expert_down, idx, w, dy, shared_gateup=None, shared_down=None, lib=None):
+def moe_backward(x_bits, expert_gateup, expert_down, idx, w, dy, shared_gateup=None, shared_down=None, lib=None,
+                 weight_grads: bool = True):
     """Gradients of the expert part of the layer (section "Training MoEs with Transformers" trains through the
-    same expert backend): given dy = d loss / d out for every token, returns a dict with dx [T, d], dw_gateup
-    [E, 2f, d], dw_down [E, d, f], dw [T, k] (routing weights) and, with a shared expert, its two weight
-    gradients. Weights as for moe_tokens (bf16 bits, every expert that a token selects must be given). fp64."""
+    same expert backend): given dy = d loss / d out for every token, returns a dict with dx [T, d], dw [T, k]
+    (routing weights) and, with weight_grads, dw_gateup [E, 2f, d], dw_down [E, d, f] and the shared expert's two
+    weight gradients. Weights as for moe_tokens (bf16 bits, every expert that a token selects must be given). fp64."""
     lib = lib or _L()
     x = _c(x_bits, np.uint16)
     T, d = x.shape
@@ -262,31 +263,35 @@ def moe_backward(x_bits, expert_gateup, expert_down, idx, w, dy, shared_gateup=N
     keep = []
     gu_p, dn_p = (ctypes.c_void_p * E)(), (ctypes.c_void_p * E)()
     dgu_p, ddn_p = (ctypes.c_void_p * E)(), (ctypes.c_void_p * E)()
-    dgu = np.zeros((E, 2 * f, d))
-    ddn = np.zeros((E, d, f))
+    dgu = np.zeros((E, 2 * f, d)) if weight_grads else None
+    ddn = np.zeros((E, d, f)) if weight_grads else None
     for e in range(E):
         if expert_gateup[e] is None or expert_down[e] is None:
             continue
         gu, dn = _c(expert_gateup[e], np.uint16), _c(expert_down[e], np.uint16)
         keep += [gu, dn]
         gu_p[e], dn_p[e] = gu.ctypes.data, dn.ctypes.data
-        dgu_p[e], ddn_p[e] = dgu[e].ctypes.data, ddn[e].ctypes.data
+        if weight_grads:
+            dgu_p[e], ddn_p[e] = dgu[e].ctypes.data, ddn[e].ctypes.data
     sgu = _c(shared_gateup, np.uint16) if shared_gateup is not None else None
     sdn = _c(shared_down, np.uint16) if shared_down is not None else None
     fs = sgu.shape[0] // 2 if sgu is not None else 0
-    dsgu = np.zeros((2 * fs, d)) if fs else None
-    dsdn = np.zeros((d, fs)) if fs else None
+    dsgu = np.zeros((2 * fs, d)) if fs and weight_grads else None
+    dsdn = np.zeros((d, fs)) if fs and weight_grads else None
     dx = np.empty((T, d))
     dw = np.empty((T, k))
     rc = lib.oracle_moe_backward(x.ctypes.data, T, d, f, E, k, gu_p, dn_p, ix.ctypes.data, ww.ctypes.data, g.ctypes.data,
                                  sgu.ctypes.data if fs else None, sdn.ctypes.data if fs else None, fs,
-                                 dx.ctypes.data, dgu_p, ddn_p, dw.ctypes.data,
-                                 dsgu.ctypes.data if fs else None, dsdn.ctypes.data if fs else None)
+                                 dx.ctypes.data, dgu_p if weight_grads else None, ddn_p if weight_grads else None,
+                                 dw.ctypes.data, dsgu.ctypes.data if dsgu is not None else None,
+                                 dsdn.ctypes.data if dsdn is not None else None)
     if rc:
         raise ValueError(f"oracle_moe_backward failed ({rc})")
-    out = {"dx": dx, "dw_gateup": dgu, "dw_down": ddn, "dw": dw}
-    if fs:
-        out["dw_gateup_shared"], out["dw_down_shared"] = dsgu, dsdn
+    out = {"dx": dx, "dw": dw}
+    if weight_grads:
+        out["dw_gateup"], out["dw_down"] = dgu, ddn
+        if fs:
+            out["dw_gateup_shared"], out["dw_down_shared"] = dsgu, dsdn
     return out
 
 
@@ -338,14 +343,31 @@ class LayerReference:
         self._dn = [None] * wl.E
         self._shared = None
 
-    def near_ties(self, eps: float = 1e-5) -> np.ndarray:
-        return np.nonzero(self.margin < eps)[0]
-
-    def outputs(self, tokens, nthreads: int | None = None) -> np.ndarray:
+    def input_grad(self, dy_bits, tokens, nthreads: int | None = None) -> np.ndarray:
+        """d loss / d x for the given tokens (rows of dy = d loss / d y as bf16 bits [T, d]): the experts' share
+        (moe_backward) plus the router's (router_backward), the top-k selection held fixed. A token's input
+        gradient depends only on that token, so a sample of tokens is computed alone. fp64."""
         import synth
 
         wl = self.wl
         tokens = np.asarray(tokens, dtype=np.int32)
+        sgu, sdn = self._load_weights(tokens)
+        dy = synth.bf16_bits_to_f32(np.asarray(dy_bits)[tokens]).astype(np.float64)
+        xs = self.x[tokens]
+        exp = moe_backward(xs, self._gu, self._dn, self.idx[tokens], self.w[tokens], dy, sgu, sdn, lib=self.lib,
+                           weight_grads=False)
+        rt = router_backward(xs, self.w_router, self.logits32[tokens], self.idx[tokens], self.w[tokens], exp["dw"],
+                             wl.route, lib=self.lib)
+        return exp["dx"] + rt["dx"]
+
+    def near_ties(self, eps: float = 1e-5) -> np.ndarray:
+        return np.nonzero(self.margin < eps)[0]
+
+    def _load_weights(self, tokens):
+        """Generate (once) the weights of the experts these tokens select, and the shared expert's."""
+        import synth
+
+        wl = self.wl
         need = np.unique(self.idx[tokens].ravel()) if len(tokens) else np.zeros(0, np.int32)
         # MXFP4 workloads compute with the weights their encoding represents
         enc = (lambda a: mxfp4_round_trip(a, lib=self.lib)) if wl.weights == "mxfp4" else (lambda a: a)
@@ -355,7 +377,12 @@ class LayerReference:
                 self._dn[e] = enc(synth.w_down_expert_host(wl, int(e)))
         if wl.shared_f and self._shared is None:
             self._shared = tuple(enc(a) for a in synth.shared_host(wl))
-        sgu, sdn = self._shared if self._shared else (None, None)
+        return self._shared if self._shared else (None, None)
+
+    def outputs(self, tokens, nthreads: int | None = None) -> np.ndarray:
+        wl = self.wl
+        tokens = np.asarray(tokens, dtype=np.int32)
+        sgu, sdn = self._load_weights(tokens)
         if len(tokens) == 0:
             return np.zeros((0, wl.d))
         return moe_tokens(self.x, self._gu, self._dn, self.idx, self.w, tokens, sgu, sdn, nthreads=nthreads,

@@ -486,7 +486,7 @@ static void swiglu_expert_backward(const uint16_t* xt, int d, int f, const uint1
         const double dyc = scale * dyt[c];
         for (int n = 0; n < f; ++n) {
             dh[n] += dyc * bf16_to_double(dr[n]);
-            dwd[(size_t)c * f + n] += dyc * h[n];
+            if (dwd) dwd[(size_t)c * f + n] += dyc * h[n];
         }
     }
     for (int n = 0; n < f; ++n) {
@@ -496,20 +496,23 @@ static void swiglu_expert_backward(const uint16_t* xt, int d, int f, const uint1
         const double du = dh[n] * a;
         const uint16_t* gr = wgu + (size_t)n * d;
         const uint16_t* ur = wgu + (size_t)(f + n) * d;
-        double* dgr = dwgu + (size_t)n * d;
-        double* dur = dwgu + (size_t)(f + n) * d;
+        double* dgr = dwgu ? dwgu + (size_t)n * d : NULL;
+        double* dur = dwgu ? dwgu + (size_t)(f + n) * d : NULL;
         for (int i = 0; i < d; ++i) {
             const double xi = bf16_to_double(xt[i]);
             dxt[i] += dg * bf16_to_double(gr[i]) + du * bf16_to_double(ur[i]);
-            dgr[i] += dg * xi;
-            dur[i] += du * xi;
+            if (dgr) {
+                dgr[i] += dg * xi;
+                dur[i] += du * xi;
+            }
         }
     }
 }
 
 /* dx [T][d], dwgu: E pointers to [2f][d], dwd: E pointers to [d][f] (all fp64, zeroed here; NULL pointers for
-   experts no token selects), dw [T][k]; shared-expert gradients dwgu_s [2fs][d], dwd_s [d][fs] when given.
-   Returns 0, -1 on a bad argument or allocation failure, -2 when a selected expert has no weights. */
+   experts no token selects; dwgu and dwd themselves NULL when no weight gradient is wanted), dw [T][k];
+   shared-expert gradients dwgu_s [2fs][d], dwd_s [d][fs] when given. Returns 0, -1 on a bad argument or
+   allocation failure, -2 when a selected expert has no weights (or no gradient arrays, when they are wanted). */
 int oracle_moe_backward(const uint16_t* x, int T, int d, int f, int E, int k, const uint16_t* const* wgu,
                         const uint16_t* const* wd, const int32_t* idx, const double* w, const double* dy,
                         const uint16_t* wgu_s, const uint16_t* wd_s, int fs, double* dx, double* const* dwgu,
@@ -522,12 +525,14 @@ int oracle_moe_backward(const uint16_t* x, int T, int d, int f, int E, int k, co
     double* dh = (double*)malloc(sizeof(double) * (size_t)hf);
     if (!g || !u || !h || !dh) { free(g); free(u); free(h); free(dh); return -1; }
     memset(dx, 0, sizeof(double) * (size_t)T * d);
-    for (int e = 0; e < E; ++e) {
-        if (dwgu[e]) memset(dwgu[e], 0, sizeof(double) * (size_t)2 * f * d);
-        if (dwd[e]) memset(dwd[e], 0, sizeof(double) * (size_t)d * f);
-    }
-    const int shared = wgu_s && wd_s && dwgu_s && dwd_s && fs > 0;
-    if (shared) {
+    const int wgrad = dwgu != NULL && dwd != NULL;
+    if (wgrad)
+        for (int e = 0; e < E; ++e) {
+            if (dwgu[e]) memset(dwgu[e], 0, sizeof(double) * (size_t)2 * f * d);
+            if (dwd[e]) memset(dwd[e], 0, sizeof(double) * (size_t)d * f);
+        }
+    const int shared = wgu_s && wd_s && fs > 0;
+    if (shared && dwgu_s && dwd_s) {
         memset(dwgu_s, 0, sizeof(double) * (size_t)2 * fs * d);
         memset(dwd_s, 0, sizeof(double) * (size_t)d * fs);
     }
@@ -538,9 +543,9 @@ int oracle_moe_backward(const uint16_t* x, int T, int d, int f, int E, int k, co
         double* dxt = dx + (size_t)t * d;
         for (int j = 0; j < k; ++j) {
             const int e = idx[(size_t)t * k + j];
-            if (e < 0 || e >= E || !wgu[e] || !wd[e] || !dwgu[e] || !dwd[e]) { status = -2; break; }
-            swiglu_expert_backward(xt, d, f, wgu[e], wd[e], w[(size_t)t * k + j], dyt, dxt, dwgu[e], dwd[e],
-                                   &dw[(size_t)t * k + j], g, u, h, dh);
+            if (e < 0 || e >= E || !wgu[e] || !wd[e] || (wgrad && (!dwgu[e] || !dwd[e]))) { status = -2; break; }
+            swiglu_expert_backward(xt, d, f, wgu[e], wd[e], w[(size_t)t * k + j], dyt, dxt,
+                                   wgrad ? dwgu[e] : NULL, wgrad ? dwd[e] : NULL, &dw[(size_t)t * k + j], g, u, h, dh);
         }
         if (shared && !status)
             swiglu_expert_backward(xt, d, fs, wgu_s, wd_s, 1.0, dyt, dxt, dwgu_s, dwd_s, NULL, g, u, h, dh);

@@ -14,7 +14,8 @@ Mixtral-8x7B) plus a tiny case, a Zipf-skewed 128-expert case and a
 are involved; everything is drawn from the generator.
 
 Tensor ids within one seed: 0 x, 1 router weight, 2 gate|up weight,
-3 down weight, 4 router-bias permutation, 5 shared gate|up, 6 shared down.
+3 down weight, 4 router-bias permutation, 5 shared gate|up, 6 shared down,
+7 upstream gradient dy (for the backward pass).
 """
 from __future__ import annotations
 
@@ -30,7 +31,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _HOST_SO = os.path.join(_HERE, "_gen.so")
 _CUDA_SO = os.path.join(_HERE, "_gen_cuda.so")
 
-TID_X, TID_WR, TID_WGU, TID_WD, TID_BIAS_PERM, TID_WGU_SHARED, TID_WD_SHARED = range(7)
+TID_X, TID_WR, TID_WGU, TID_WD, TID_BIAS_PERM, TID_WGU_SHARED, TID_WD_SHARED, TID_DY = range(8)
 
 X_SIGMA = 1.0
 W_SIGMA = 0.02
@@ -200,6 +201,11 @@ def zipf_bias(w: Workload) -> np.ndarray | None:
 
 def x_host(w: Workload) -> np.ndarray:
     return normal_bf16(w.seed, TID_X, 0, w.T * w.d, X_SIGMA).reshape(w.T, w.d)
+
+
+def dy_host(w: Workload) -> np.ndarray:
+    """Upstream gradient d loss / d y for the backward pass: [T, d] bf16 bits, N(0, 1)."""
+    return normal_bf16(w.seed, TID_DY, 0, w.T * w.d, X_SIGMA).reshape(w.T, w.d)
 
 
 def w_router_host(w: Workload) -> np.ndarray:

@@ -547,6 +547,38 @@ def pin_router_backward_finite_difference(lib):
                 assert abs(num - got[t, e]) <= 2e-4 * max(1.0, abs(num)), (mode, t, e, num, got[t, e])
 
 
+def pin_layer_input_grad_autograd(lib):
+    """The whole layer's input gradient (experts + router, selection held fixed) on the tiny workload equals torch
+    fp64 autograd through the router projection, the routing-weight formula and the experts."""
+    import torch
+
+    wl = synth.workload("tiny")
+    ref = oracle.LayerReference(wl, lib=lib)
+    dy_bits = synth.dy_host(wl)
+    toks = np.arange(wl.T)
+    got = ref.input_grad(dy_bits, toks)
+    X = torch.tensor(_f64(ref.x), requires_grad=True)
+    L = X @ torch.tensor(ref.w_router.astype(np.float64)).T
+    sel = torch.tensor(ref.idx, dtype=torch.int64)
+    w = torch.softmax(L.gather(1, sel), dim=1)  # the tiny workload routes by softmax over the selected logits
+    assert wl.route == "topk_softmax"
+    gus = {e: torch.tensor(_f64(synth.w_gateup_expert_host(wl, e))) for e in np.unique(ref.idx)}
+    dns = {e: torch.tensor(_f64(synth.w_down_expert_host(wl, e))) for e in np.unique(ref.idx)}
+    f = wl.f
+    rows = []
+    for t in range(wl.T):
+        acc = 0
+        for j in range(wl.k):
+            e = int(ref.idx[t, j])
+            hh = torch.nn.functional.silu(gus[e][:f] @ X[t]) * (gus[e][f:] @ X[t])
+            acc = acc + w[t, j] * (dns[e] @ hh)
+        rows.append(acc)
+    (torch.stack(rows) * torch.tensor(_f64(dy_bits))).sum().backward()
+    want = X.grad.numpy()
+    # the oracle takes its routing weights from the fp32-rounded logits; autograd from the fp64 ones
+    np.testing.assert_allclose(got, want, rtol=1e-4, atol=1e-5 * np.abs(want).max())
+
+
 PINS = [
     pin_router_logits_numpy,
     pin_topk_golden,
@@ -573,4 +605,5 @@ PINS = [
     pin_backward_linear_in_dy,
     pin_router_backward_autograd,
     pin_router_backward_finite_difference,
+    pin_layer_input_grad_autograd,
 ]
