@@ -76,6 +76,8 @@ def load(path: str | None = None):
     lib.oracle_moe_backward.restype = ci
     lib.oracle_router_backward.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp]
     lib.oracle_router_backward.restype = ci
+    lib.oracle_weight_grad_entries.argtypes = [vp, ci, ci, ci, ci, vp, vp, ci, vp, vp, vp, ci, vp, vp, ci, vp]
+    lib.oracle_weight_grad_entries.restype = ci
     return lib
 
 
@@ -292,6 +294,27 @@ def moe_backward(x_bits, expert_gateup, expert_down, idx, w, dy, shared_gateup=N
         out["dw_gateup"], out["dw_down"] = dgu, ddn
         if fs:
             out["dw_gateup_shared"], out["dw_down_shared"] = dsgu, dsdn
+    return out
+
+
+def weight_grad_entries(x_bits, w_gateup_e, w_down_e, e: int, idx, w, dy, which: str, rows, cols, lib=None):
+    """Entries (rows[q], cols[q]) of expert e's weight gradient, summed over every token that selects e:
+    which = "down" -> dW_down[e] [d, f]; which = "gateup" -> dW_gateup[e] [2f, d]. fp64. The same sums as
+    moe_backward, for a sample of entries (full-size layers)."""
+    lib = lib or _L()
+    x = _c(x_bits, np.uint16)
+    T, d = x.shape
+    gu, dn = _c(w_gateup_e, np.uint16), _c(w_down_e, np.uint16)
+    f = gu.shape[0] // 2
+    ix = _c(idx, np.int32)
+    a, b = _c(rows, np.int32), _c(cols, np.int32)
+    out = np.empty(len(a))
+    rc = lib.oracle_weight_grad_entries(x.ctypes.data, T, d, f, ix.shape[1], gu.ctypes.data, dn.ctypes.data, int(e),
+                                        ix.ctypes.data, _c(w, np.float64).ctypes.data, _c(dy, np.float64).ctypes.data,
+                                        0 if which == "down" else 1, a.ctypes.data, b.ctypes.data, len(a),
+                                        out.ctypes.data)
+    if rc:
+        raise ValueError(f"oracle_weight_grad_entries failed ({rc})")
     return out
 
 

@@ -604,3 +604,61 @@ int oracle_router_backward(const uint16_t* x, const float* w_router, const float
     }
     return 0;
 }
+
+/* Selected entries of one expert's weight gradients, summed over every (token, slot) that selects expert e: the
+   sums oracle_moe_backward accumulates, restricted to the asked entries so that full-size layers stay cheap.
+     kind 0 (down):    out[q] = dWd[a[q]][b[q]] = sum w_tj * dy[t][c] * h_t[n],          c = a[q], n = b[q]
+     kind 1 (gate|up): out[q] = dWgu[a[q]][b[q]], row m = a[q] in [0, 2f), column i = b[q]:
+                       sum dg_t[m] * x_t[i] for m < f,  sum du_t[m - f] * x_t[i] for m >= f
+   with h, dg, du as in oracle_moe_backward. Returns 0, or -1 on a bad argument or allocation failure. */
+int oracle_weight_grad_entries(const uint16_t* x, int T, int d, int f, int k, const uint16_t* wgu, const uint16_t* wd,
+                               int e, const int32_t* idx, const double* w, const double* dy, int kind,
+                               const int32_t* a, const int32_t* b, int n_entries, double* out) {
+    if (T < 0 || d <= 0 || f <= 0 || k <= 0 || (kind != 0 && kind != 1)) return -1;
+    for (int q = 0; q < n_entries; ++q) {
+        if (kind == 0 && (a[q] < 0 || a[q] >= d || b[q] < 0 || b[q] >= f)) return -1;
+        if (kind == 1 && (a[q] < 0 || a[q] >= 2 * f || b[q] < 0 || b[q] >= d)) return -1;
+        out[q] = 0.0;
+    }
+    double* g = (double*)malloc(sizeof(double) * (size_t)f);
+    double* u = (double*)malloc(sizeof(double) * (size_t)f);
+    double* h = (double*)malloc(sizeof(double) * (size_t)f);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)f);
+    if (!g || !u || !h || !dh) { free(g); free(u); free(h); free(dh); return -1; }
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            if (idx[(size_t)t * k + j] != e) continue;
+            const uint16_t* xt = x + (size_t)t * d;
+            const double wt = w[(size_t)t * k + j];
+            const double* dyt = dy + (size_t)t * d;
+            for (int n = 0; n < f; ++n) {
+                double gs = 0.0, us = 0.0;
+                for (int i = 0; i < d; ++i) {
+                    const double xi = bf16_to_double(xt[i]);
+                    gs += xi * bf16_to_double(wgu[(size_t)n * d + i]);
+                    us += xi * bf16_to_double(wgu[(size_t)(f + n) * d + i]);
+                }
+                g[n] = gs;
+                u[n] = us;
+                h[n] = gs / (1.0 + exp(-gs)) * us;
+            }
+            if (kind == 0) {
+                for (int q = 0; q < n_entries; ++q) out[q] += wt * dyt[a[q]] * h[b[q]];
+                continue;
+            }
+            for (int n = 0; n < f; ++n) {
+                double s = 0.0;
+                for (int c = 0; c < d; ++c) s += wt * dyt[c] * bf16_to_double(wd[(size_t)c * f + n]);
+                dh[n] = s;
+            }
+            for (int q = 0; q < n_entries; ++q) {
+                const int m = a[q], i = b[q];
+                const int n = m < f ? m : m - f;
+                const double sg = 1.0 / (1.0 + exp(-g[n]));
+                const double coef = m < f ? dh[n] * u[n] * (sg * (1.0 + g[n] * (1.0 - sg))) : dh[n] * g[n] * sg;
+                out[q] += coef * bf16_to_double(xt[i]);
+            }
+        }
+    free(g); free(u); free(h); free(dh);
+    return 0;
+}

@@ -547,6 +547,22 @@ def pin_router_backward_finite_difference(lib):
                 assert abs(num - got[t, e]) <= 2e-4 * max(1.0, abs(num)), (mode, t, e, num, got[t, e])
 
 
+def pin_weight_grad_entries(lib):
+    """Sampled weight-gradient entries equal the corresponding entries of the full backward (which autograd pins)."""
+    rng = _rng(45)
+    T, d, f, E, k = 9, 16, 12, 4, 2
+    x, gu, dn, idx, w = _random_layer(rng, T, d, f, E, k)
+    dy = rng.standard_normal((T, d))
+    full = oracle.moe_backward(x, gu, dn, idx, w, dy, lib=lib)
+    for e in range(E):
+        rows, cols = rng.integers(0, d, 20), rng.integers(0, f, 20)
+        got = oracle.weight_grad_entries(x, gu[e], dn[e], e, idx, w, dy, "down", rows, cols, lib=lib)
+        np.testing.assert_allclose(got, full["dw_down"][e][rows, cols], rtol=1e-12, atol=1e-14)
+        rows, cols = rng.integers(0, 2 * f, 20), rng.integers(0, d, 20)
+        got = oracle.weight_grad_entries(x, gu[e], dn[e], e, idx, w, dy, "gateup", rows, cols, lib=lib)
+        np.testing.assert_allclose(got, full["dw_gateup"][e][rows, cols], rtol=1e-12, atol=1e-14)
+
+
 def pin_layer_input_grad_autograd(lib):
     """The whole layer's input gradient (experts + router, selection held fixed) on the tiny workload equals torch
     fp64 autograd through the router projection, the routing-weight formula and the experts."""
@@ -606,4 +622,5 @@ PINS = [
     pin_router_backward_autograd,
     pin_router_backward_finite_difference,
     pin_layer_input_grad_autograd,
+    pin_weight_grad_entries,
 ]

@@ -68,6 +68,9 @@ MUTATIONS = {
     "router_backward_sigmoid_derivative_dropped": ("g = s * (1.0 - s) / S * (dwt[j] - dot);", "g = s / S * (dwt[j] - dot);"),
     "router_backward_dx_uses_x": ("dx[(size_t)t * d + i] += g * (double)w_router[(size_t)e * d + i];",
                                   "dx[(size_t)t * d + i] += g * bf16_to_double(x[(size_t)t * d + i]);"),
+    "grad_entries_routing_weight_dropped": ("for (int q = 0; q < n_entries; ++q) out[q] += wt * dyt[a[q]] * h[b[q]];",
+                                            "for (int q = 0; q < n_entries; ++q) out[q] += dyt[a[q]] * h[b[q]];"),
+    "grad_entries_up_uses_silu_prime": (": dh[n] * g[n] * sg;", ": dh[n] * u[n] * sg;"),
     "mxfp4_decode_scale_bias": ("oracle_e2m1_value(code) * ldexp(1.0, sc - 127)", "oracle_e2m1_value(code) * ldexp(1.0, sc - 126)"),
 }
 
