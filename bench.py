@@ -5,12 +5,16 @@ One step = one pass of the whole layer (route -> permute -> gate|up grouped GEMM
 GEMM -> weighted combine) over one batch of seeded synthetic tokens, through the library's public API.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py --kernel gateup|down [--workload NAME] [--shape T=..,E=..] [--gemm FAMILY]
 
-Prints one JSON line (rank 0). Device timing: CUDA events on the launching stream around each step, L2
-flushed (256 MiB write) before every step outside the events, max over ranks. `e2e` repeats the step with
-the input copied from pinned host memory and the output copied back inside the timed region. Multi-GPU
-runs are independent replicas (the layer has no cross-GPU exchange): weak scaling, value = all tokens / time.
+Prints one JSON line (rank 0). Device timing: CUDA events on the launching stream around each step (no events
+inside a step), L2 flushed (256 MiB write) before every step outside the events, max over ranks. The per-stage
+split comes from a second, separate pass with events between the stages. `e2e` repeats the step with the input
+copied from pinned host memory and the output copied back inside the timed region. Multi-GPU runs are
+independent replicas (the layer has no cross-GPU exchange): weak scaling, value = all tokens / time.
 `--impl reference` times the CPU oracle (plain fp64 C, all host cores) on a bounded token sample.
+`--kernel` times one grouped GEMM alone on the workload's realised routing (for profilers); `--shape` shrinks the
+workload for such captures and `--gemm` forces a kernel family (single, pair, wide, swap).
 """
 from __future__ import annotations
 
@@ -55,7 +59,8 @@ TRAFFIC = {
     ("grouped_gemm_down", "decode-256e-shared", "b23bf8a046918afc"): 6464814848,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
-                  ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "sm100.cuh", "common.cuh", "moe.cu")]
+                  ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "sm100.cuh", "common.cuh",
+                   "moe.cu")]
 
 
 def kernel_source_hash() -> str:
@@ -92,6 +97,11 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--settle-seconds", type=float, default=2.0,
                     help="extra untimed load after the warm-up so clocks and power settle")
+    ap.add_argument("--kernel", choices=["gateup", "down"], default=None,
+                    help="time one grouped GEMM alone (kernel-only mode, for profilers)")
+    ap.add_argument("--gemm", choices=["auto", "single", "pair", "wide", "swap"], default="auto",
+                    help="force a grouped-GEMM kernel family")
+    ap.add_argument("--shape", default="", help="comma-separated workload overrides, e.g. T=1024,E=64 (profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -341,19 +351,30 @@ def run_reference(args):
 
 # ---- our arm --------------------------------------------------------------------------------------------
 
-def run_ours(args):
-    import numpy as np
+def bench_workload(args):
+    """The workload named by --workload, with any --shape overrides (a renamed copy, never the headline)."""
+    import synth
+
+    wl = synth.workload(args.workload)
+    if args.shape:
+        over = {}
+        for item in args.shape.split(","):
+            key, val = item.split("=")
+            if key not in ("T", "d", "f", "E", "k", "shared_f"):
+                raise SystemExit(f"--shape: {key} cannot be overridden")
+            over[key] = int(val)
+        tag = ",".join(f"{k}={v}" for k, v in over.items())
+        wl = synth.workload(args.workload, **over, name=f"{wl.name}[{tag}]")
+    return wl
+
+
+def setup_layer(args, dev):
     import torch
 
     import synth
-    from mixture_experts_ffn_11_b200 import MoEFFN, get_device_error
+    from mixture_experts_ffn_11_b200 import MoEFFN
 
-    rank, local, world = dist_init("nccl")
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU (there is no CPU fallback)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    wl = synth.workload(args.workload)
+    wl = bench_workload(args)
     synth.build_cuda()
     inp = synth.device_inputs(wl, dev)
     layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
@@ -362,6 +383,66 @@ def run_ours(args):
         for key in ("w_gateup", "w_down", "w_gateup_shared", "w_down_shared"):
             inp[key] = None
         torch.cuda.empty_cache()
+    return wl, inp, layer
+
+
+def run_kernel(args):
+    """One grouped GEMM alone, on the routing the layer realises: W warm-up launches, then K launches each after
+    an L2 flush, CUDA events around each launch. For profilers (select the kernel with -k and skip the warm-up
+    launches) and for comparing kernel families."""
+    import torch
+
+    from mixture_experts_ffn_11_b200 import _native as N
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    N.set_gemm_kernel(args.gemm)
+    wl, inp, layer = setup_layer(args, dev)
+    layer.forward(inp["x"])
+    b = layer.buf
+    s = torch.cuda.current_stream(dev)
+    if args.kernel == "gateup":
+        launch = lambda: layer._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)  # noqa: E731
+    else:
+        launch = lambda: layer._down(b["h"], "routed", b["offsets"], b["y_perm"], s)  # noqa: E731
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        launch()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, c in ev:
+        flush.zero_()
+        a.record(s)
+        launch()
+        c.record(s)
+    torch.cuda.synchronize(dev)
+    if N.get_device_error():
+        raise SystemExit("device error word set")
+    ms = statistics.mean(a.elapsed_time(c) for a, c in ev)
+    counts = b["counts"].cpu().numpy()
+    active, fig_gu, fig_dn = gemm_figures(wl, counts)
+    peaks, src = load_peaks()
+    fig = fig_gu if args.kernel == "gateup" else fig_dn
+    roof = roofline_entry(f"grouped_gemm_{args.kernel}", fig, ms, peaks, "bf16_tflops", None)
+    roof["peak_source"] = f"{src} {'hbm_gbs' if roof['bound'] == 'hbm' else 'bf16_tflops'}"
+    print(json.dumps({"kernel_only": args.kernel, "gemm_family": args.gemm, "ms": round(ms, 5), "launches": args.steps,
+                      "config": workload_config(wl), "active_experts": active, "roofline": roof}), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+
+    from mixture_experts_ffn_11_b200 import _native as N
+    from mixture_experts_ffn_11_b200 import get_device_error
+
+    rank, local, world = dist_init("nccl")
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    N.set_gemm_kernel(args.gemm)
+    wl, inp, layer = setup_layer(args, dev)
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -385,29 +466,39 @@ def run_ours(args):
     if get_device_error():
         raise SystemExit("device error word set during warm-up")
 
+    def timed_pass(stage_events: bool):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        stage_ev = [dict() for _ in range(K)]
+        barrier(dev)
+        torch.cuda.synchronize(dev)
+        t_a = time.time()
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step(timing=stage_ev[i] if stage_events else None)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dev)
+        t_b = time.time()
+        step_ms = [a.elapsed_time(b) for a, b in ev]
+        stages = {}
+        if stage_events:
+            for name in stage_ev[0]:
+                stages[name] = statistics.mean(a.elapsed_time(b) for a, b in (s[name] for s in stage_ev))
+        return step_ms, stages, t_a, t_b
+
+    # headline: K steps with events only around each whole step
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    stage_ev = [dict() for _ in range(K)]
-    barrier(dev)
-    torch.cuda.synchronize(dev)
-    t0 = time.time()
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step(timing=stage_ev[i])
-        ev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dev)
-    t1 = time.time()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
+    step_ms, _, t0, t1 = timed_pass(False)
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / K
-    stages = {}
-    for name in stage_ev[0]:
-        stages[name] = statistics.mean(a.elapsed_time(b) for a, b in (s[name] for s in stage_ev))
     err = get_device_error()
     if err:
         raise SystemExit(f"device error word {err:#x} set during the timed region")
+    # breakdown: a second pass of K steps with events between the stages (they split the programmatic launch
+    # overlap between kernels, so this pass runs a little slower than the headline; both are reported)
+    staged_ms, stages, _, _ = timed_pass(True)
+    staged_ms_per_step = max_over_ranks(sum(staged_ms), dev) / K
 
     # end to end, as a server would run it: every step copies its input from pinned host memory and its
     # output back to pinned host memory, on their own streams, so step i's copies overlap the layer of the
@@ -463,7 +554,8 @@ def run_ours(args):
                        "pinned host on a second copy stream; two buffer sets, copies of one step overlap the layer "
                        "of the next",
                "l2": "not flushed (steps overlap); each step streams its expert weights (larger than L2) and a "
-                     "fresh input from the host"}
+                     "fresh input from the host",
+               "comparable_with_value": False}
     sampler.stop()
     clocks = sampler.summary(t0, t1)
 
@@ -475,6 +567,7 @@ def run_ours(args):
     tr = TRAFFIC.get(("grouped_gemm_gateup", wl.name, src_hash))
     roof = roofline_entry("grouped_gemm_gateup", fig_gu, stages["gateup"], peaks, peak_kind, tr)
     roof["peak_source"] = f"{peak_src} {'hbm_gbs' if roof['bound'] == 'hbm' else peak_kind}"
+    roof["launch_ms_source"] = "CUDA events around the kernel in the breakdown pass (not the headline pass)"
     roof_dn = roofline_entry("grouped_gemm_down", fig_dn, stages["down"], peaks, peak_kind,
                              TRAFFIC.get(("grouped_gemm_down", wl.name, src_hash)))
     lflop, lbytes = layer_figures(wl, active)
@@ -488,8 +581,11 @@ def run_ours(args):
                                "frac": round(t_roof * 1e3 / ms_per_step, 4),
                                "achieved_tflops": round(lflop / (ms_per_step * 1e-3) / 1e12, 2)},
             "breakdown_ms": {k: round(v, 5) for k, v in stages.items()},
+            "breakdown_pass_ms_per_step": round(staged_ms_per_step, 5),
             "gpu_launches": K * launches_per_step, "clocks": clocks, "e2e": e2e,
             "parallelism": "replicas" if world > 1 else "single GPU"}
+    if args.gemm != "auto":
+        line["gemm_family"] = args.gemm
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     if rank == 0:
@@ -505,6 +601,8 @@ def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.kernel:
+        return run_kernel(args)
     return run_ours(args)
 
 

@@ -99,7 +99,8 @@ typedef enum {
  *   logits_out [T][E] fp32, written (required: the selection reads it back)
  *   topk_idx   [T][k] int32, expert ids, descending logit order
  *   topk_w     [T][k] fp32, routing weights per `mode`
- * Limits: 1 <= k <= E <= 1024, T >= 0 (T == 0 launches nothing). */
+ * Limits: 1 <= E <= 1024, 1 <= k <= min(E, 32), T >= 0 (T == 0 launches
+ * nothing). */
 moe_status_t moe_route_topk(const moe_bf16_t* x, const float* w_router, const float* bias, int T, int d, int E,
                             int k, moe_route_mode_t mode, float* logits_out, int32_t* topk_idx, float* topk_w,
                             cudaStream_t stream);
@@ -151,7 +152,8 @@ size_t moe_permute_workspace_size(int T, int E, int k);
  *                  bytes, 256-byte aligned; its contents need not be
  *                  initialised and are scratch after the call.
  * Expert ids outside [0,E) are skipped and flagged (MOE_DEVERR_EXPERT_RANGE);
- * the outputs are then incomplete. Limits: 1 <= k <= E <= 1024. */
+ * the outputs are then incomplete. Limits: 1 <= E <= 1024,
+ * 1 <= k <= min(E, 32). */
 moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, int d, int E, int k,
                          int32_t* expert_counts, int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
                          moe_bf16_t* x_perm, void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -173,7 +175,9 @@ moe_status_t moe_permute(const moe_bf16_t* x, const int32_t* topk_idx, int T, in
  *    E = 1024 up to 262,144).
  *  - The first call on a device looks up the array's device address (a
  *    one-time set-up per device); make that first call before capturing a
- *    stream.
+ *    stream. The address is kept for the life of the process: a device
+ *    reset (cudaDeviceReset, or tearing down the primary context) is not
+ *    supported while the library stays loaded.
  *  - All calls on a device share the one array. Its contents persist between
  *    calls, and each call rewrites every byte it reads before reading it, so
  *    nothing has to be cleared. Calls that can overlap on the GPU (different
@@ -271,6 +275,44 @@ moe_status_t moe_grouped_gemm_down_mxfp4(const moe_bf16_t* h, const uint8_t* wq_
 moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_perm, const float* topk_w,
                                    const moe_bf16_t* shared, int T, int d, int k, moe_bf16_t* y,
                                    cudaStream_t stream);
+
+/* ---- Measurement and test hook ----
+ * The bf16 grouped GEMMs (moe_grouped_gemm_gateup / _down) pick one of
+ * several kernel families from the problem's shape. All of them compute the
+ * same sums in the same order per output element (bf16 products, fp32
+ * accumulation over K in ascending 16-element steps), so their results are
+ * identical; they differ in tile shape and speed:
+ *   MOE_GEMM_SINGLE  one CTA per 128-row tile (few rows per expert)
+ *   MOE_GEMM_PAIR    CTA pairs, 256 token rows per tile
+ *   MOE_GEMM_WIDE    CTA pairs, 256 token rows x two accumulators per tile
+ *   MOE_GEMM_SWAP    CTA pairs, the weight rows as the MMA's M dimension
+ *                    and tiles of any multiple of 16 token rows
+ * moe_set_gemm_kernel forces one family for every later call in the process
+ * (on every device), so that a test can reach each of them and a benchmark
+ * can compare them; MOE_GEMM_AUTO restores the library's own choice. The
+ * setting is process-wide and not tied to a stream: do not change it while
+ * another thread is calling the GEMMs. Not needed for normal use. */
+typedef enum {
+    MOE_GEMM_AUTO = 0,
+    MOE_GEMM_SINGLE = 1,
+    MOE_GEMM_PAIR = 2,
+    MOE_GEMM_WIDE = 3,
+    MOE_GEMM_SWAP = 4
+} moe_gemm_kernel_t;
+moe_status_t moe_set_gemm_kernel(moe_gemm_kernel_t kind);
+
+/* Test hook for the kernels' failure path. Every pipeline wait inside the
+ * grouped GEMMs is bounded: when it runs out, the kernel sets
+ * MOE_DEVERR_WAIT_TIMEOUT, every role leaves its loop, copies and MMAs still
+ * in flight are waited for (each wait bounded again), tensor memory is freed
+ * and the kernel returns; the CUDA context stays usable. This call sets, on
+ * the current device, the wait limit in nanoseconds (0 restores the default
+ * of 2 s) and, with stall != 0, makes the MMA-issuing warp of every bf16
+ * grouped GEMM first wait on a barrier that nothing arrives on, so that a
+ * test can run the timeout path on purpose. It synchronises the device first.
+ * Results of GEMMs launched while stall is set are undefined; the device
+ * error word reports the timeout. Not for normal use. */
+moe_status_t moe_test_set_wait(unsigned long long limit_ns, int stall);
 
 /* Synchronise `stream`, copy the device error word of the current device to
  * *out (0 = no anomaly) and clear it. Returns MOE_OK when the word was 0,

@@ -25,7 +25,9 @@ ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm":
 EXPORTS = ("moe_route_topk", "moe_router_split_weights", "moe_route_topk_split", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
            "moe_permute_static_ws",
            "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_mxfp4_quantize", "moe_grouped_gemm_gateup_mxfp4",
-           "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_get_device_error", "moe_last_error_string")
+           "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_set_gemm_kernel", "moe_test_set_wait", "moe_get_device_error",
+           "moe_last_error_string")
+GEMM_KERNELS = {"auto": 0, "single": 1, "pair": 2, "wide": 3, "swap": 4}
 
 
 class MoEError(RuntimeError):
@@ -54,6 +56,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_gemm_gateup_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_down_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_unpermute_combine": [vp, vp, vp, vp, ci, ci, ci, vp, vp],
+        "moe_set_gemm_kernel": [ci],
+        "moe_test_set_wait": [ctypes.c_ulonglong, ci],
         "moe_get_device_error": [ctypes.POINTER(ctypes.c_uint), vp],
         "moe_last_error_string": [],
     }
@@ -256,6 +260,35 @@ def unpermute_combine(y_perm, inv_perm, topk_w, shared, y, stream=None):
     _need(y, torch.bfloat16, (T, d), "y")
     _check(_lib.moe_unpermute_combine(_p(y_perm), _p(inv_perm), _p(topk_w), _p(shared), T, d, k, _p(y),
                                       _stream(stream)), "moe_unpermute_combine")
+
+
+def set_gemm_kernel(name: str) -> None:
+    """Force one bf16 grouped-GEMM kernel family ("single", "pair", "wide", "swap") for every later call in the
+    process, or restore the library's own choice ("auto"). A measurement and test hook."""
+    if name not in GEMM_KERNELS:
+        raise ValueError(f"unknown GEMM kernel family {name!r}")
+    _check(_lib.moe_set_gemm_kernel(GEMM_KERNELS[name]), "moe_set_gemm_kernel")
+
+
+class gemm_kernel:
+    """Context manager: `with gemm_kernel("swap"): ...` forces a family inside the block, then restores "auto"."""
+
+    def __init__(self, name: str):
+        self.name = name
+
+    def __enter__(self):
+        set_gemm_kernel(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        set_gemm_kernel("auto")
+        return False
+
+
+def test_set_wait(limit_ns: int = 0, stall: bool = False) -> None:
+    """Test hook: the bounded waits' limit on the current device (0 = the default 2 s) and, with stall, a wait
+    that nothing ends in every bf16 grouped GEMM, so its timeout path runs."""
+    _check(_lib.moe_test_set_wait(int(limit_ns), 1 if stall else 0), "moe_test_set_wait")
 
 
 def get_device_error(stream=None) -> int:

@@ -113,7 +113,7 @@ struct GemmShape {
     static constexpr int EPI_BYTES = 4 * 2048;  // per-epilogue-warp store staging
     static_assert((STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES) % 128 == 0, "staging buffer alignment");
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES + EPI_BYTES;
-    static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert((2 * STAGES + 6) * 8 + 8 <= BAR_BYTES, "barrier area");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -130,7 +130,8 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
     uint64_t* tfull_bar = empty_bar + STAGES;
     uint64_t* tempty_bar = tfull_bar + 2;
     uint64_t* final_bar = tempty_bar + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    uint64_t* never_bar = final_bar + 1;  // nothing arrives on it (test_stall)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES);
     int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
@@ -150,6 +151,7 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
             mbar_init(&tempty_bar[a], 4);
         }
         mbar_init(final_bar, 1);
+        mbar_init(never_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -265,6 +267,8 @@ __global__ void __launch_bounds__(GG_THREADS, 1)
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         bool ok = true;
+        if (lane == 0) ok = test_stall(never_bar, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, abort_flag);
             ok = __shfl_sync(0xffffffffu, ok, 0);

@@ -47,7 +47,7 @@ struct GemmWideShape {
     static_assert((STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES) % 128 == 0, "staging buffer alignment");
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + TABLE_BYTES + EPI_BYTES;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
-    static_assert((2 * STAGES + 4) * 8 + 8 <= BAR_BYTES, "barrier area");
+    static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
 };
 
 // As store_warp_rows_32cols (gemm.cuh), but each 8-column piece u of the chunk has its own destination column
@@ -87,7 +87,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GW_THREADS, 1)
     uint64_t* tfull_bar = empty_bar + STAGES;  // [1]
     uint64_t* tempty_bar = tfull_bar + 1;      // [1], used in the leader
     uint64_t* final_bar = tempty_bar + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    uint64_t* never_bar = final_bar + 1;  // nothing arrives on it (test_stall)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_off = reinterpret_cast<int32_t*>(smem + STAGES * S::STAGE_BYTES + S::BAR_BYTES);
     int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
@@ -108,6 +109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GW_THREADS, 1)
         mbar_init(tfull_bar, 1);
         mbar_init(tempty_bar, 16);  // 8 epilogue warps x 2 CTAs
         mbar_init(final_bar, 1);
+        mbar_init(never_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmA);
@@ -218,6 +220,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GW_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0, tphase = 0;
             bool ok = true;
+            if (lane == 0) ok = test_stall(never_bar, abort_flag);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
             for (int tile = cluster; tile < total && ok; tile += n_clusters) {
                 if (lane == 0) ok = mbar_wait_bounded(tempty_bar, tphase ^ 1u, abort_flag);
                 ok = __shfl_sync(0xffffffffu, ok, 0);

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -18,6 +19,7 @@
 #include "gemm.cuh"
 #include "gemm_pair.cuh"
 #include "gemm_wide.cuh"
+#include "gemm_swap.cuh"
 #include "gemm_fp4.cuh"
 #include "combine.cuh"
 
@@ -87,6 +89,12 @@ using Wide240DN = GemmWideShape<240, 4, false>;
 // K blocks per stage) -30%, K=14336 +10%; down K=768 -25%, K=2880 +4%, K=14336 +10%.
 constexpr int kWideMinK = 8192;      // gate|up
 constexpr int kWideMinKDown = 2048;  // down
+//   CTA pair with the weights as M and the token rows as N (tiles of any multiple of 16 rows)
+using SwapGU = GemmSwapShape<true, 2, 3>;
+using SwapDN = GemmSwapShape<false, 2, 3>;
+
+// Kernel family forced by moe_set_gemm_kernel (MOE_GEMM_AUTO: the library's choice).
+std::atomic<int> g_gemm_kernel{MOE_GEMM_AUTO};
 
 cudaError_t set_gemm_attributes() {
     const cudaFuncAttribute a = cudaFuncAttributeMaxDynamicSharedMemorySize;
@@ -103,6 +111,8 @@ cudaError_t set_gemm_attributes() {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, true>, a, Wide240GU::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<256, 4, false>, a, Wide256DN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, false>, a, Wide240DN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3>, a, SwapDN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<16, true>, a, GemmFp4Shape<16, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<32, true>, a, GemmFp4Shape<32, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<64, true>, a, GemmFp4Shape<64, true>::SMEM_BYTES);
@@ -297,9 +307,61 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)", e);
 }
 
+template <bool GATEUP, int SUB, int STAGES>
+moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
+    using S = GemmSwapShape<GATEUP, SUB, STAGES>;
+    CUtensorMap tw, to;
+    SwapMaps tx;
+    const cuuint64_t rows = GATEUP ? (cuuint64_t)2 * p.f : (cuuint64_t)p.n_out;
+    const cuuint64_t wdims[3] = {(cuuint64_t)p.K, rows, (cuuint64_t)p.G};
+    const cuuint64_t wstr[2] = {(cuuint64_t)p.K * 2, rows * (cuuint64_t)p.K * 2};
+    const cuuint32_t wbox[3] = {GG_BK, GATEUP ? 64u : 128u, 1};
+    moe_status_t st = make_tmap(&tw, p.w, 3, wdims, wstr, wbox);
+    const cuuint64_t xdims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
+    const cuuint64_t xstr[1] = {(cuuint64_t)p.K * 2};
+    for (int i = 0; i < 5 && st == MOE_OK; ++i) {
+        const cuuint32_t xbox[2] = {GG_BK, (cuuint32_t)(128 >> i)};
+        st = make_tmap(&tx.x[i], p.a, 2, xdims, xstr, xbox);
+    }
+    if (st == MOE_OK) st = make_out_map(p, &to);
+    if (st != MOE_OK) return st;
+    const GemmArgs args = gemm_args(p, S::TILE_W);
+    const long upper = ((long)p.M / GS_MAX_N + p.G) * (long)args.n_tiles;  // >= the real tile count
+    const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
+    const int streamed_once = (long)p.M <= (long)p.G * GS_MAX_N ? 1 : 0;
+    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES>, dim3(2 * clusters),
+                                     dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, args, streamed_once);
+    return check_launch(GATEUP ? "grouped_gemm_gateup (swap pair)" : "grouped_gemm_down (swap pair)", e);
+}
+
+// A kernel family chosen with moe_set_gemm_kernel.
+moe_status_t launch_forced(int kind, const GemmProblem& p, bool gateup, int sms, cudaStream_t stream) {
+    const bool sub2 = p.K >= kSub2MinK;
+    const bool w240 = (long)(p.n_out + 239) / 240 * 240 < (long)(p.n_out + 255) / 256 * 256;
+    switch (kind) {
+        case MOE_GEMM_SINGLE:
+            return gateup ? launch_single<256, 4, true>(p, sms, stream) : launch_single<256, 4, false>(p, sms, stream);
+        case MOE_GEMM_PAIR:
+            if (gateup) return sub2 ? launch_pair<256, 3, true, 2>(p, sms, stream) : launch_pair<256, 6, true>(p, sms, stream);
+            return w240 ? launch_pair<240, 6, false>(p, sms, stream) : launch_pair<256, 6, false>(p, sms, stream);
+        case MOE_GEMM_WIDE: {
+            const long span = gateup ? 1 : 2;
+            const bool wide240 = (long)(p.n_out + 240 * span - 1) / (240 * span) * (240 * span) <
+                                 (long)(p.n_out + 256 * span - 1) / (256 * span) * (256 * span);
+            if (gateup)
+                return wide240 ? launch_wide<240, 4, true>(p, sms, stream) : launch_wide<256, 4, true>(p, sms, stream);
+            return wide240 ? launch_wide<240, 4, false>(p, sms, stream) : launch_wide<256, 4, false>(p, sms, stream);
+        }
+        default:
+            return gateup ? launch_swap<true, 2, 3>(p, sms, stream) : launch_swap<false, 2, 3>(p, sms, stream);
+    }
+}
+
 // Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs. Otherwise a single CTA
 // per tile, 256 wide unless that leaves SMs idle (e.g. one small group), then 64 wide.
 moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cudaStream_t stream) {
+    const int forced = g_gemm_kernel.load(std::memory_order_relaxed);
+    if (forced != MOE_GEMM_AUTO && sms >= 2) return launch_forced(forced, p, gateup, sms, stream);
     if ((long)p.M >= (long)p.G * GG_BM && sms >= 2 && p.K >= (gateup ? kWideMinK : kWideMinKDown)) {
         // columns padded per tile: gate|up NH per tile, down 2*NH per tile; pick the width that pads less
         const long span = gateup ? 1 : 2;
@@ -472,10 +534,6 @@ moe_status_t static_ws_address(void** out) {
     return MOE_OK;
 }
 }  // namespace
-
-extern "C" {
-
-}  // extern "C"
 
 namespace {
 
@@ -778,6 +836,25 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
                                      reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
                                      reinterpret_cast<__nv_bfloat16*>(y));
     return check_launch("unpermute_combine", e);
+}
+
+moe_status_t moe_set_gemm_kernel(moe_gemm_kernel_t kind) {
+    if (kind < MOE_GEMM_AUTO || kind > MOE_GEMM_SWAP) return fail(MOE_ERR_INVALID_ARG, "unknown GEMM kernel %d", (int)kind);
+    g_gemm_kernel.store((int)kind, std::memory_order_relaxed);
+    return MOE_OK;
+}
+
+moe_status_t moe_test_set_wait(unsigned long long limit_ns, int stall) {
+    if (limit_ns == 0) limit_ns = kWaitLimitNs;
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const int flag = stall ? 1 : 0;
+    cudaError_t e = cudaDeviceSynchronize();  // no kernel of this device is waiting while the values change
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_wait_limit_ns, &limit_ns, sizeof limit_ns);
+    if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_wait_stall, &flag, sizeof flag);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "setting the wait limit: %s", cudaGetErrorString(e));
+    return MOE_OK;
 }
 
 moe_status_t moe_get_device_error(unsigned int* out, cudaStream_t stream) {

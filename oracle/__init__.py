@@ -18,7 +18,7 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
                  E=1,k=1 dense SwiGLU (torch fp64); identical experts; linearity
                  in W_down; hand-derived golden values
   e2m1_value     pinned: the FP4 E2M1 value table of the OCP MX v1.0 specification
-                 (tests/golden/e2m1_values.txt)
+                 (tests/golden/mxfp4_e2m1.json, codes 0..15 including -0)
   mxfp4_quantize pinned: round-trip of encodable blocks; the tie and clamp cases of
                  round-to-nearest-even on the E2M1 grid; closed-form scales (zero,
                  subnormal and power-of-two blocks); the error bound of the grid;
@@ -30,6 +30,10 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
                  differences of moe_tokens in the routing weights; linearity in dy
   router_backward pinned: torch fp64 autograd of each mode's weight formula and of the
                  router projection; central differences of topk's weights in the logits
+  weight_grad_entries pinned: equal to the matching entries of moe_backward's full
+                 weight gradients on random small layers
+  LayerReference.input_grad pinned: torch fp64 autograd of the whole layer per token
+                 (router projection, routing weights and experts) on the tiny workload
 """
 from __future__ import annotations
 

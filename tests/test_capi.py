@@ -36,6 +36,17 @@ def test_every_declared_symbol_is_exported(native):
     assert set(_header_functions()) == set(native.EXPORTS)
 
 
+def test_static_scratch_size_matches_header(native):
+    """The binding's copy of MOE_PERMUTE_STATIC_WS_BYTES is the header's value, and the array holds exactly
+    the workspace of 262,144 assignments over 1024 experts (256 segments x 1024 experts x 4 B)."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    m = re.search(r"#define\s+MOE_PERMUTE_STATIC_WS_BYTES\s+\(1u\s*<<\s*(\d+)\)", src)
+    assert m, "MOE_PERMUTE_STATIC_WS_BYTES not found in include/moe.h"
+    assert native.PERMUTE_STATIC_WS_BYTES == 1 << int(m.group(1))
+    assert native.permute_workspace_size(262_144, 1024, 1) == native.PERMUTE_STATIC_WS_BYTES
+    assert native.permute_workspace_size(262_144 + 1, 1024, 1) > native.PERMUTE_STATIC_WS_BYTES
+
+
 def test_workspace_size(native):
     ws = native.permute_workspace_size
     assert ws(0, 8, 2) == 0
