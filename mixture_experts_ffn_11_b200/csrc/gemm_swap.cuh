@@ -4,9 +4,9 @@
 // Why: an expert's rows come in ragged counts (gpt-oss-shaped prefill: 447-569 rows per expert). With token rows
 // as M, a CTA pair computes 256 of them at a time, so a group's last tile is on average half padding (22% of the
 // tensor work on that workload). With token rows as N, a tile takes any multiple of 16 rows up to 256: a group of
-// n rows is cut into ceil(n / 256) tiles of equal size rounded up to 16 rows, and the padding falls to a few rows
-// per group. The weight rows (M = 256 per pair, 128 per CTA) are the expert's output columns, whose count is
-// fixed by the model and mostly a multiple of 128.
+// n rows is cut into full tiles of 256 rows and one last tile of the remaining rows rounded up to 16, so the
+// padding falls to a few rows per group. The weight rows (M = 256 per pair, 128 per CTA) are the expert's output
+// columns, whose count is fixed by the model and mostly a multiple of 128.
 //
 //   out[r][c] = epilogue( sum_k A[r][k] * W[g][c][k] )   for r in [off[g], off[g+1])
 //
@@ -14,17 +14,19 @@
 // token row. Per pair tile (one group g, one block of weight rows, one block of at most 256 token rows):
 //   down   (GATEUP = false): CTA `rank` holds weight rows (= output columns) c0 + 128*rank + [0, 128).
 //   gate|up (GATEUP = true): the tile covers 128 columns j0 + [0, 128) of h; CTA `rank` holds the 64 gate rows
-//          j0 + 64*rank + [0, 64) in TMEM lanes 0-63 and the matching 64 up rows (f + j) in lanes 64-127, so one
-//          accumulator holds both halves of silu(gate) * up for its columns. A CTA may read TMEM only in the lane
-//          quarter of each warp, so the warps of lanes 64-127 pass their up values to the warps of lanes 0-63
-//          through shared memory (bounded mbarrier hand-off), which compute h.
+//          j0 + 64*rank + [0, 64) in TMEM lanes 0-63 and the matching 64 up rows (f + j) in lanes 64-127 (one
+//          TMA box of the weights viewed as [G][2][f][K]), so one accumulator holds both factors of
+//          silu(gate) * up for its columns. A warp may read TMEM only in its own lane quarter, so the warps of
+//          lanes 0-63 (warps 4 and 5, which share their SM sub-partitions with the TMA and MMA issuing warps)
+//          pass their gate values through shared memory (bounded mbarrier hand-off) to the warps of lanes
+//          64-127 (warps 2 and 3), which compute and store h.
 // The token rows of the tile are split between the pair as the MMA's B operand: the leader loads the first N/2,
-// the peer the next N/2, and both accumulators hold all N columns.
+// the peer the next N/2 (one TMA box of 128, 64, 32, 16 or 8 rows, the smallest that holds N/2), and both
+// accumulators hold all N columns.
 //
 // Roles (192 threads per CTA, both CTAs):
-//   warp 0     TMA producer: this CTA's 128 weight rows (one box, or gate and up boxes of 64 rows) and its N/2
-//              token rows (boxes of 128/64/32/16/8 rows, the binary decomposition of N/2) per 64-wide K block,
-//              SUB K blocks per ring stage; completion counted on the leader's full[stage].
+//   warp 0     TMA producer: per 64-wide K block, this CTA's 128 weight rows (one box) and its token rows (one
+//              box), SUB K blocks per ring stage; completion counted on the leader's full[stage].
 //   warp 1     TMEM allocation (512 columns: two accumulators of up to 256 token columns) and, in the leader,
 //              the MMA issuer: tcgen05.mma.cta_group::2 M=256 N=tile rows (runtime instruction descriptor).
 //   warps 2-5  epilogue: tcgen05.ld of the lane quarter, transpose through shared memory (thread = output
@@ -42,31 +44,28 @@ namespace moe {
 constexpr int GS_THREADS = 192;
 constexpr int GS_MAX_N = 256;  // token rows per tile (UMMA N for M = 256, a multiple of 16)
 
+// Stage layout: the SUB K blocks of this CTA's weight rows, then the SUB K blocks of its token rows:
+//   [W k0 | W k1 | ... | X k0 | X k1 | ...], W blocks 16 KB apart, X blocks (rows per CTA) * 128 bytes apart.
+// BIGBOX: the operands are read through tensor maps that view [rows][K] as [K/64][rows][64] (K a multiple of 64),
+// so one TMA box brings the SUB K blocks of a stage at once (a 32 KB box moves faster than two 16 KB ones).
 template <bool GATEUP, int SUB, int STAGES>
 struct GemmSwapShape {
     static constexpr int W_BYTES = 128 * GG_BK * 2;  // this CTA's 128 weight rows of one K block
     static constexpr int X_BYTES = 128 * GG_BK * 2;  // room for this CTA's share of the token rows (<= 128)
     static constexpr int SUB_BYTES = W_BYTES + X_BYTES;
     static constexpr int STAGE_BYTES = SUB * SUB_BYTES;
+    static constexpr int X_OFF = SUB * W_BYTES;  // token blocks start here in a stage
     static constexpr int TILE_W = GATEUP ? 128 : 256;  // output columns per pair tile
     static constexpr int TMEM_COLS = 512;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int TABLE_BYTES = (3 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;
-    // storing warps x two 2 KB staging blocks; gate|up: two storing warps plus two 4 KB up-value buffers
+    static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;
+    // 4 x two 2 KB staging blocks (down); gate|up: two storing warps' staging blocks + two 4 KB hand-off buffers
     static constexpr int EPI_BYTES = 4 * 2 * 2048;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + TABLE_BYTES;
     static_assert(SUB_BYTES % 1024 == 0, "sub-block bases stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((2 * STAGES + 4 + 1 + 4 + 1) * 8 + 8 <= BAR_BYTES, "barrier area");
 };
-
-// Token-row tiles of a group of n rows: ceil(n / 256) tiles of cs rows (the last one shorter), cs the even share
-// rounded up to 16. Returns cs (0 for an empty group); the tile count is ceil(n / cs) <= ceil(n / 256).
-__device__ __forceinline__ int swap_chunk_rows(int n) {
-    if (n <= 0) return 0;
-    const int nt = (n + GS_MAX_N - 1) / GS_MAX_N;
-    return ((n + nt - 1) / nt + 15) / 16 * 16;
-}
 
 // Write one warp's 32 output columns (thread = column) x 32 token rows (v[t], fp32) into a 2 KB staging block in
 // the output's row-major order: row t holds the 32 columns as 64 bytes, its 16-byte units XOR-swizzled by
@@ -111,14 +110,21 @@ __device__ __forceinline__ void flush_staged_block(uint8_t* stage, int lane, con
     __syncwarp();
 }
 
-// tmW: weights [G][rows][K] (rows = 2f for gate|up with box 64, d for down with box 128), K-major, 128-B swizzle.
-// tmX[i]: the token rows [M][K] with boxes of 128 >> i rows (i = 0..4). tmO: the output [M][n_out], 32 x 32 boxes,
-// 64-byte swizzle.
+// tmX[i]: the token rows [M][K] with boxes of 128 >> i rows (i = 0..4).
 struct SwapMaps {
     CUtensorMap x[5];
 };
 
-template <bool GATEUP, int SUB, int STAGES>
+// Map index of the smallest token box holding `half` rows (half a multiple of 8, 8..128).
+__device__ __forceinline__ int swap_box_index(int half) {
+    return half > 64 ? 0 : (half > 32 ? 1 : (half > 16 ? 2 : (half > 8 ? 3 : 4)));
+}
+
+// tmW: the weights, K-major, 128-byte swizzle: gate|up as [G][2][f][K] with box {64, 64, 2, 1} (64 gate rows
+// and the matching 64 up rows), down as [G][d][K] with box {64, 128, 1}; with BIGBOX the same views with a K-block
+// dimension {64, rows.., K/64} boxing SUB K blocks. tmX: the token rows, [M][K] (or [K/64][M][64] with BIGBOX).
+// tmO: the output [M][n_out], 32 x 32 boxes, 64-byte swizzle.
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ SwapMaps tmX,
                              const __grid_constant__ CUtensorMap tmO, const GemmArgs args, int weights_streamed_once) {
@@ -132,14 +138,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
     uint64_t* tfull_bar = empty_bar + STAGES;  // [2]
     uint64_t* tempty_bar = tfull_bar + 2;      // [2], used in the leader
     uint64_t* final_bar = tempty_bar + 2;
-    uint64_t* xfull_bar = final_bar + 1;   // [2] gate|up: up values of a block are in xbuf[p]
+    uint64_t* xfull_bar = final_bar + 1;   // [2] gate|up: gate values of a block are in xbuf[p]
     uint64_t* xempty_bar = xfull_bar + 2;  // [2] gate|up: xbuf[p] has been read
     uint64_t* never_bar = xempty_bar + 2;  // nothing arrives on it (test_stall)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int32_t* s_off = reinterpret_cast<int32_t*>(epi + S::EPI_BYTES + S::BAR_BYTES);
     int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
-    int32_t* s_cs = s_tp + (GG_MAX_GROUPS + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -185,16 +190,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
         s_off[g] = v;
     }
     __syncthreads();
-    if (warp == 0) {  // per group: token-tile rows, and the tile prefix: tiles(g) = ceil(n / cs) * wblocks
+    if (warp == 0) {  // tile prefix over groups: tiles(g) = ceil(rows / 256) * wblocks
         const int per = (G + 31) / 32;
         const int g0 = lane * per, g1 = min(g0 + per, G);
         int local = 0;
         for (int g = g0; g < g1; ++g) {
             const int n = s_off[g + 1] - s_off[g];
             if (n < 0) flag_error(MOE_DEVERR_GROUP_RANGE);
-            const int cs = swap_chunk_rows(n);
-            s_cs[g] = cs;
-            local += cs ? (n + cs - 1) / cs * wblocks : 0;
+            local += (max(n, 0) + GS_MAX_N - 1) / GS_MAX_N * wblocks;
         }
         int incl = local;
 #pragma unroll
@@ -205,8 +208,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
         int run = incl - local;
         for (int g = g0; g < g1; ++g) {
             s_tp[g] = run;
-            const int n = s_off[g + 1] - s_off[g], cs = s_cs[g];
-            run += cs ? (n + cs - 1) / cs * wblocks : 0;
+            run += (max(s_off[g + 1] - s_off[g], 0) + GS_MAX_N - 1) / GS_MAX_N * wblocks;
         }
         if (lane == 31) s_tp[G] = incl;
     }
@@ -217,7 +219,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
     const uint32_t tmem_base = *tmem_slot;
     const int total = s_tp[G];
 
-    // tile -> group g, weight block wb, first token row r0 (absolute), rows in the tile, N (rows rounded to 16)
+    // tile -> group g, weight block wb, first token row r0 (absolute), rows in the tile (<= 256)
     auto locate = [&](int tile, int& g, int& wb, int& r0, int& rows) {
         int lo = 0, hi = G - 1;
         while (lo < hi) {
@@ -228,13 +230,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                 hi = mid - 1;
         }
         g = lo;
-        const int n = s_off[g + 1] - s_off[g], cs = s_cs[g];
-        const int tt = (n + cs - 1) / cs;
+        const int n = s_off[g + 1] - s_off[g];
+        const int tt = (n + GS_MAX_N - 1) / GS_MAX_N;
         const int local = tile - s_tp[g];
         wb = local / tt;
         const int ti = local - wb * tt;
-        r0 = s_off[g] + ti * cs;
-        rows = min(cs, n - ti * cs);
+        r0 = s_off[g] + ti * GS_MAX_N;
+        rows = min(GS_MAX_N, n - ti * GS_MAX_N);
     };
 
     if (warp == 0) {
@@ -249,36 +251,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
             int g, wb, r0, rows;
             locate(tile, g, wb, r0, rows);
             const int half = ((rows + 15) / 16) * 8;  // token rows per CTA (N / 2)
+            const int bi = swap_box_index(half);
             const int xrow0 = r0 + (int)rank * half;
             const int wrow = GATEUP ? wb * 128 + 64 * (int)rank : wb * 256 + 128 * (int)rank;
-            const uint32_t sub_tx = (uint32_t)(S::W_BYTES + half * GG_BK * 2);
+            const uint32_t sub_tx = (uint32_t)(S::W_BYTES + (128 >> bi) * GG_BK * 2);
             for (int kb = 0; kb < KB; ++kb) {
                 if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 if (lane == 0) {
-                    const int nsub = min(SUB, KBS - kb * SUB);
                     uint8_t* sa = stages + stage * S::STAGE_BYTES;
                     const uint32_t bar = mapa_shared(smem_u32(&full_bar[stage]), 0);
-                    if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * (uint32_t)nsub * sub_tx);
-                    for (int sb = 0; sb < nsub; ++sb) {  // K past the end arrives as zeros
-                        const int kc = (kb * SUB + sb) * GG_BK;
-                        uint8_t* sw = sa + sb * S::SUB_BYTES;
-                        if constexpr (GATEUP) {
-                            tma_load_3d_pair(sw, &tmW, bar, kc, wrow, g, pol_w);
-                            tma_load_3d_pair(sw + 64 * GG_BK * 2, &tmW, bar, kc, args.f + wrow, g, pol_w);
-                        } else {
-                            tma_load_3d_pair(sw, &tmW, bar, kc, wrow, g, pol_w);
-                        }
-                        uint8_t* sx = sw + S::W_BYTES;
-                        int done = 0;
-#pragma unroll
-                        for (int i = 0; i < 5; ++i) {
-                            const int box = 128 >> i;
-                            if (half & box) {
-                                tma_load_2d_pair(sx + done * GG_BK * 2, &tmX.x[i], bar, kc, xrow0 + done, pol_x);
-                                done += box;
-                            }
+                    if constexpr (BIGBOX) {  // one box per operand: SUB K blocks (past the end: zeros)
+                        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * (uint32_t)SUB * sub_tx);
+                        if constexpr (GATEUP)
+                            tma_load_5d_pair(sa, &tmW, bar, 0, wrow, 0, kb * SUB, g, pol_w);
+                        else
+                            tma_load_4d_pair(sa, &tmW, bar, 0, wrow, kb * SUB, g, pol_w);
+                        tma_load_3d_pair(sa + S::X_OFF, &tmX.x[bi], bar, 0, xrow0, kb * SUB, pol_x);
+                    } else {
+                        const int nsub = min(SUB, KBS - kb * SUB);
+                        if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2u * (uint32_t)nsub * sub_tx);
+                        for (int sb = 0; sb < nsub; ++sb) {  // K past the end arrives as zeros
+                            const int kc = (kb * SUB + sb) * GG_BK;
+                            uint8_t* sw = sa + sb * S::W_BYTES;
+                            if constexpr (GATEUP)
+                                tma_load_4d_pair(sw, &tmW, bar, kc, wrow, 0, g, pol_w);
+                            else
+                                tma_load_3d_pair(sw, &tmW, bar, kc, wrow, g, pol_w);
+                            tma_load_2d_pair(sa + S::X_OFF + sb * (128 >> bi) * GG_BK * 2, &tmX.x[bi], bar, kc,
+                                             xrow0, pol_x);
                         }
                     }
                 }
@@ -307,6 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                 int g, wb, r0, rows;
                 locate(tile, g, wb, r0, rows);
                 const uint32_t idesc = idesc_bf16_f32(256, (rows + 15) / 16 * 16);
+                const uint32_t xstride = (uint32_t)(128 >> swap_box_index((rows + 15) / 16 * 8)) * GG_BK * 2;
                 if (lane == 0) ok = mbar_wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, abort_flag);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
@@ -320,9 +323,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                     if (lane == 0) {
                         const int nsub = min(SUB, KBS - kb * SUB);
                         for (int sb = 0; sb < nsub; ++sb) {
-                            const uint32_t sa = smem_u32(stages + stage * S::STAGE_BYTES + sb * S::SUB_BYTES);
-                            const uint64_t wdesc = smem_desc_sw128(sa);
-                            const uint64_t xdesc = smem_desc_sw128(sa + S::W_BYTES);
+                            const uint32_t sa = smem_u32(stages + stage * S::STAGE_BYTES);
+                            const uint64_t wdesc = smem_desc_sw128(sa + sb * S::W_BYTES);
+                            const uint64_t xdesc = smem_desc_sw128(sa + S::X_OFF + sb * xstride);
 #pragma unroll
                             for (int k = 0; k < GG_BK / 16; ++k)
                                 umma_bf16_ss_pair(d_tmem, wdesc + 2 * k, xdesc + 2 * k, idesc,
@@ -350,8 +353,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
         const int q = warp & 3;  // TMEM lanes 32q .. 32q+31
         const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
-        // gate|up: warps of lanes 64-127 (q = 2, 3) hand their up values to the warps of lanes 0-63 (q = 0, 1)
-        const bool up_warp = GATEUP && q >= 2;
+        // gate|up: the warps of lanes 0-63 (q = 0, 1: gate rows) hand their values to the warps of lanes 64-127
+        // (q = 2, 3: up rows), which compute and store h
+        const bool ferry = GATEUP && q < 2;
         const int p = q & 1;  // hand-off pair (gate|up)
         uint8_t* xbuf = epi + 8192 + p * 4096;
         uint8_t* stage_base = epi + (GATEUP ? p : (warp - 2)) * 4096;
@@ -377,8 +381,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                 float v[32];
                 if constexpr (GATEUP) {
                     const uint32_t par = blocks & 1u;
-                    if (up_warp) {
-                        // hand off: thread = up row, 32 token values as eight 16-byte units, XOR-swizzled by lane
+                    if (ferry) {
+                        // hand off: thread = gate row, 32 token values as eight 16-byte units, XOR-swizzled by lane
                         if (blocks > 0) {
                             ok = mbar_wait_bounded(&xempty_bar[p], par ^ 1u, abort_flag);
                             ok = __all_sync(0xffffffffu, ok);
@@ -395,18 +399,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                     ok = mbar_wait_bounded(&xfull_bar[p], par, abort_flag);
                     ok = __all_sync(0xffffffffu, ok);
                     if (!ok) break;
-                    uint32_t up[32];
+                    uint32_t gt[32];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const uint4 w4 = *reinterpret_cast<const uint4*>(xbuf + lane * 128 + ((u ^ (lane & 7)) << 4));
-                        up[4 * u] = w4.x;
-                        up[4 * u + 1] = w4.y;
-                        up[4 * u + 2] = w4.z;
-                        up[4 * u + 3] = w4.w;
+                        gt[4 * u] = w4.x;
+                        gt[4 * u + 1] = w4.y;
+                        gt[4 * u + 2] = w4.z;
+                        gt[4 * u + 3] = w4.w;
                     }
                     mbar_arrive(&xempty_bar[p]);
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) v[t] = swiglu(__uint_as_float(raw[t]), __uint_as_float(up[t]));
+                    for (int t = 0; t < 32; ++t) v[t] = swiglu(__uint_as_float(gt[t]), __uint_as_float(raw[t]));
                 } else {
 #pragma unroll
                     for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(raw[t]);
@@ -425,7 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
-        if (up_warp && ok && blocks > 0) {  // the last hand-off has been read before the buffer goes away
+        if (ferry && ok && blocks > 0) {  // the last hand-off has been read before the buffer goes away
             mbar_wait_bounded(&xempty_bar[p], (blocks & 1u) ^ 1u, abort_flag);
         }
         if (lane == 0) bulk_wait_all();  // the output stores have landed before the CTA leaves

@@ -84,11 +84,9 @@ using Wide256GU = GemmWideShape<256, 4, true>;
 using Wide240GU = GemmWideShape<240, 4, true>;
 using Wide256DN = GemmWideShape<256, 4, false>;
 using Wide240DN = GemmWideShape<240, 4, false>;
-// The wide tile's epilogue is not overlapped with the next tile's MMAs, so it pays off on long reductions only:
-// measured (interleaved A/B against the 256-wide pair tile) gate|up K=2880 -8%, K=2048 -23%, K=4096 (against two
-// K blocks per stage) -30%, K=14336 +10%; down K=768 -25%, K=2880 +4%, K=14336 +10%.
-constexpr int kWideMinK = 8192;      // gate|up
-constexpr int kWideMinKDown = 2048;  // down
+// The wide tile's epilogue is not overlapped with the next tile's MMAs, so it paid off on long reductions only
+// (interleaved A/B against the 256-wide pair tile: gate|up K=2880 -8%, K=14336 +10%; down K=768 -25%, K=14336
+// +10%). The pair and wide families are now reached only through moe_set_gemm_kernel.
 //   CTA pair with the weights as M and the token rows as N (tiles of any multiple of 16 rows)
 using SwapGU = GemmSwapShape<true, 2, 3>;
 using SwapDN = GemmSwapShape<false, 2, 3>;
@@ -111,8 +109,10 @@ cudaError_t set_gemm_attributes() {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, true>, a, Wide240GU::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<256, 4, false>, a, Wide256DN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_wide_kernel<240, 4, false>, a, Wide240DN::SMEM_BYTES);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3>, a, SwapGU::SMEM_BYTES);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3>, a, SwapDN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, false>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, false>, a, SwapDN::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, true>, a, SwapDN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<16, true>, a, GemmFp4Shape<16, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<32, true>, a, GemmFp4Shape<32, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<64, true>, a, GemmFp4Shape<64, true>::SMEM_BYTES);
@@ -209,7 +209,7 @@ moe_status_t make_tmap(CUtensorMap* map, const void* base, int rank, const cuuin
                        CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-    const cuuint32_t elem_strides[3] = {1, 1, 1};
+    const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
     const CUresult r = enc(map, dtype, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, elem_strides,
                            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -307,21 +307,50 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)", e);
 }
 
-template <bool GATEUP, int SUB, int STAGES>
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX>
 moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
     using S = GemmSwapShape<GATEUP, SUB, STAGES>;
     CUtensorMap tw, to;
     SwapMaps tx;
-    const cuuint64_t rows = GATEUP ? (cuuint64_t)2 * p.f : (cuuint64_t)p.n_out;
-    const cuuint64_t wdims[3] = {(cuuint64_t)p.K, rows, (cuuint64_t)p.G};
-    const cuuint64_t wstr[2] = {(cuuint64_t)p.K * 2, rows * (cuuint64_t)p.K * 2};
-    const cuuint32_t wbox[3] = {GG_BK, GATEUP ? 64u : 128u, 1};
-    moe_status_t st = make_tmap(&tw, p.w, 3, wdims, wstr, wbox);
-    const cuuint64_t xdims[2] = {(cuuint64_t)p.K, (cuuint64_t)p.M};
-    const cuuint64_t xstr[1] = {(cuuint64_t)p.K * 2};
-    for (int i = 0; i < 5 && st == MOE_OK; ++i) {
-        const cuuint32_t xbox[2] = {GG_BK, (cuuint32_t)(128 >> i)};
-        st = make_tmap(&tx.x[i], p.a, 2, xdims, xstr, xbox);
+    moe_status_t st;
+    const cuuint64_t K = (cuuint64_t)p.K, f = (cuuint64_t)p.f, G = (cuuint64_t)p.G, n_out = (cuuint64_t)p.n_out;
+    const cuuint64_t KBS = (K + GG_BK - 1) / GG_BK;
+    if (BIGBOX) {  // K-block views: [rows][K] read as [K/64][rows][64] (K a multiple of 64), SUB K blocks per box
+        if (GATEUP) {  // [G][K/64][2][f][64]
+            const cuuint64_t wdims[5] = {GG_BK, f, 2, KBS, G};
+            const cuuint64_t wstr[4] = {K * 2, f * K * 2, GG_BK * 2, 2 * f * K * 2};
+            const cuuint32_t wbox[5] = {GG_BK, 64, 2, SUB, 1};
+            st = make_tmap(&tw, p.w, 5, wdims, wstr, wbox);
+        } else {  // [G][K/64][d][64]
+            const cuuint64_t wdims[4] = {GG_BK, n_out, KBS, G};
+            const cuuint64_t wstr[3] = {K * 2, GG_BK * 2, n_out * K * 2};
+            const cuuint32_t wbox[4] = {GG_BK, 128, SUB, 1};
+            st = make_tmap(&tw, p.w, 4, wdims, wstr, wbox);
+        }
+        const cuuint64_t xdims[3] = {GG_BK, (cuuint64_t)p.M, KBS};
+        const cuuint64_t xstr[2] = {K * 2, GG_BK * 2};
+        for (int i = 0; i < 5 && st == MOE_OK; ++i) {
+            const cuuint32_t xbox[3] = {GG_BK, (cuuint32_t)(128 >> i), SUB};
+            st = make_tmap(&tx.x[i], p.a, 3, xdims, xstr, xbox);
+        }
+    } else {
+        if (GATEUP) {  // [G][2][f][K]: one box = 64 gate rows and the matching 64 up rows
+            const cuuint64_t wdims[4] = {K, f, 2, G};
+            const cuuint64_t wstr[3] = {K * 2, f * K * 2, 2 * f * K * 2};
+            const cuuint32_t wbox[4] = {GG_BK, 64, 2, 1};
+            st = make_tmap(&tw, p.w, 4, wdims, wstr, wbox);
+        } else {  // [G][d][K]
+            const cuuint64_t wdims[3] = {K, n_out, G};
+            const cuuint64_t wstr[2] = {K * 2, n_out * K * 2};
+            const cuuint32_t wbox[3] = {GG_BK, 128, 1};
+            st = make_tmap(&tw, p.w, 3, wdims, wstr, wbox);
+        }
+        const cuuint64_t xdims[2] = {K, (cuuint64_t)p.M};
+        const cuuint64_t xstr[1] = {K * 2};
+        for (int i = 0; i < 5 && st == MOE_OK; ++i) {
+            const cuuint32_t xbox[2] = {GG_BK, (cuuint32_t)(128 >> i)};
+            st = make_tmap(&tx.x[i], p.a, 2, xdims, xstr, xbox);
+        }
     }
     if (st == MOE_OK) st = make_out_map(p, &to);
     if (st != MOE_OK) return st;
@@ -329,9 +358,15 @@ moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
     const long upper = ((long)p.M / GS_MAX_N + p.G) * (long)args.n_tiles;  // >= the real tile count
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GS_MAX_N ? 1 : 0;
-    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES>, dim3(2 * clusters),
+    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX>, dim3(2 * clusters),
                                      dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, args, streamed_once);
     return check_launch(GATEUP ? "grouped_gemm_gateup (swap pair)" : "grouped_gemm_down (swap pair)", e);
+}
+
+template <bool GATEUP>
+moe_status_t launch_swap_auto(const GemmProblem& p, int sms, cudaStream_t stream) {
+    if (p.K % GG_BK == 0) return launch_swap<GATEUP, 2, 3, true>(p, sms, stream);
+    return launch_swap<GATEUP, 2, 3, false>(p, sms, stream);
 }
 
 // A kernel family chosen with moe_set_gemm_kernel.
@@ -353,31 +388,20 @@ moe_status_t launch_forced(int kind, const GemmProblem& p, bool gateup, int sms,
             return wide240 ? launch_wide<240, 4, false>(p, sms, stream) : launch_wide<256, 4, false>(p, sms, stream);
         }
         default:
-            return gateup ? launch_swap<true, 2, 3>(p, sms, stream) : launch_swap<false, 2, 3>(p, sms, stream);
+            return gateup ? launch_swap_auto<true>(p, sms, stream) : launch_swap_auto<false>(p, sms, stream);
     }
 }
 
-// Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs. Otherwise a single CTA
-// per tile, 256 wide unless that leaves SMs idle (e.g. one small group), then 64 wide.
+// Kernel choice. Groups averaging at least 128 rows (prefill) run on CTA pairs with the weights as the MMA's M
+// dimension (gemm_swap.cuh): tiles of any multiple of 16 token rows, so ragged groups cost almost no padding;
+// measured faster than the 256-row pair tiles and the two-accumulator tiles on every prefill workload (gpt-oss
+// gate|up -9%, Mixtral gate|up -5%, zipf-128e -8%). Otherwise (a few rows per expert, decode) a single CTA per
+// 128-row tile streams the weights, 256 wide unless that leaves SMs idle (e.g. one small group), then 64 wide.
 moe_status_t launch_grouped_gemm(const GemmProblem& p, bool gateup, int sms, cudaStream_t stream) {
     const int forced = g_gemm_kernel.load(std::memory_order_relaxed);
     if (forced != MOE_GEMM_AUTO && sms >= 2) return launch_forced(forced, p, gateup, sms, stream);
-    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2 && p.K >= (gateup ? kWideMinK : kWideMinKDown)) {
-        // columns padded per tile: gate|up NH per tile, down 2*NH per tile; pick the width that pads less
-        const long span = gateup ? 1 : 2;
-        const long w256 = (long)(p.n_out + 256 * span - 1) / (256 * span) * (256 * span);
-        const long w240 = (long)(p.n_out + 240 * span - 1) / (240 * span) * (240 * span);
-        if (gateup)
-            return w240 < w256 ? launch_wide<240, 4, true>(p, sms, stream) : launch_wide<256, 4, true>(p, sms, stream);
-        return w240 < w256 ? launch_wide<240, 4, false>(p, sms, stream) : launch_wide<256, 4, false>(p, sms, stream);
-    }
-    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2) {
-        if (gateup)
-            return p.K >= kSub2MinK ? launch_pair<256, 3, true, 2>(p, sms, stream) : launch_pair<256, 6, true>(p, sms, stream);
-        const long w256 = (long)(p.n_out + 255) / 256 * 256, w240 = (long)(p.n_out + 239) / 240 * 240;
-        if (w240 < w256) return launch_pair<240, 6, false>(p, sms, stream);
-        return launch_pair<256, 6, false>(p, sms, stream);
-    }
+    if ((long)p.M >= (long)p.G * GG_BM && sms >= 2)
+        return gateup ? launch_swap_auto<true>(p, sms, stream) : launch_swap_auto<false>(p, sms, stream);
     const long row_tiles = std::max<long>((p.M + GG_BM - 1) / GG_BM, std::min<long>(p.G, p.M));
     const long wide_tiles = row_tiles * ((p.n_out + (gateup ? 127 : 255)) / (gateup ? 128 : 256));
     if (wide_tiles >= sms)
