@@ -40,23 +40,20 @@ L2_FLUSH_BYTES = 256 << 20
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an ncu capture, keyed by the
 # kernel, the workload and a hash of the GEMM sources (comments stripped) at capture time. A stale hash -> null.
-# Captured (one pass, full-size workload) with
-#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --clock-control none
-#       -k regex:grouped_gemm -s 4 -c 4 --csv python bench.py --steps 3 --warmup 3 --settle-seconds 0
-#       --no-cpu-baseline --no-e2e --workload W
-# averaging the two launches of each GEMM (decode: the routed-expert launches, not the shared expert's).
-# Re-keyed once without a new capture, when the MXFP4 kernels were added: in these files that change only added
-# lines (helpers, entry points, an include; `git diff 34c60ab -- <files>` removes none), so the bf16 GEMM kernels
-# compile from the same code as when these figures were taken.
+# Captured on one launch of the GEMM timed alone on the workload's routing, L2 flushed before it, as the bench
+# does before each step:
+#   python bench.py --kernel K --workload W --steps 2 --warmup 3 > plain.log 2>&1 &&
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:grouped_gemm -s 4 -c 1
+#       python bench.py --kernel K --workload W --steps 2 --warmup 3
 TRAFFIC = {
-    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "b23bf8a046918afc"): 1248037760,
-    ("grouped_gemm_down", "gpt-oss-20b-prefill", "b23bf8a046918afc"): 713720448,
-    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "b23bf8a046918afc"): 2475335040,
-    ("grouped_gemm_down", "mixtral-8x7b-prefill", "b23bf8a046918afc"): 3088177664,
-    ("grouped_gemm_gateup", "zipf-128e", "b23bf8a046918afc"): 1631391488,
-    ("grouped_gemm_down", "zipf-128e", "b23bf8a046918afc"): 1081674880,
-    ("grouped_gemm_gateup", "decode-256e-shared", "b23bf8a046918afc"): 12926854144,
-    ("grouped_gemm_down", "decode-256e-shared", "b23bf8a046918afc"): 6464814848,
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "5eb5b456683cd862"): 1247501824,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "5eb5b456683cd862"): 710778112,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "5eb5b456683cd862"): 2479206400,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "5eb5b456683cd862"): 2457910272,
+    ("grouped_gemm_gateup", "zipf-128e", "5eb5b456683cd862"): 1605244928,
+    ("grouped_gemm_down", "zipf-128e", "5eb5b456683cd862"): 1082768384,
+    ("grouped_gemm_gateup", "decode-256e-shared", "5eb5b456683cd862"): 12929945344,
+    ("grouped_gemm_down", "decode-256e-shared", "5eb5b456683cd862"): 6466502144,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "sm100.cuh", "common.cuh",
