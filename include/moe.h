@@ -276,6 +276,95 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
                                    const moe_bf16_t* shared, int T, int d, int k, moe_bf16_t* y,
                                    cudaStream_t stream);
 
+/* ---- Backward pass (training) ----
+ * The blog post trains MoE layers through the same grouped expert backend
+ * ("Training MoEs with Transformers"). With the top-k selection held fixed (it
+ * is piecewise constant in the router logits), the gradients of one layer
+ * call y = combine(down(swiglu(gateup(x_perm)))) for an upstream gradient dy:
+ *   moe_permute_backward            dy_perm[r] = w[t,j] dy[t], dw[t,j] = <dy[t], y_perm[r]>
+ *   moe_grouped_gemm_down           dh = dy_perm W_down[e]        (weights transposed: W_down^T [E][f][d])
+ *   moe_grouped_gemm_gateup_preact  g | u of the forward, recomputed [M][2f]
+ *   moe_swiglu_backward             dg = dh u silu'(g), du = dh silu(g)
+ *   moe_grouped_gemm_down           dx_perm = [dg|du] W_gateup[e] (weights transposed: W_gateup^T [E][d][2f])
+ *   moe_unpermute_combine           dx = sum over slots of dx_perm (unit weights) + the router's share
+ *   moe_grouped_weight_grad         dW_down[e] = dy_perm_e^T h_e, dW_gateup[e] = [dg|du]_e^T x_perm_e
+ *   moe_router_backward             dlogits, dW_r, dbias and the router's share of dx
+ * Every reduction runs in a fixed order (no atomics): the results are
+ * deterministic. moe_transpose_weights makes the transposed weight copies
+ * once per weight update. */
+
+/* Pre-activations of the gate|up projection: gu[r][n] = sum_i a[r][i] w[g][n][i]
+ * for n < 2f (columns [0, f) the gate, [f, 2f) the up projection), fp32
+ * accumulation rounded to bf16; the same sums as moe_grouped_gemm_gateup before
+ * its SwiGLU. Arguments and limits as moe_grouped_gemm_gateup; gu [M][2f]. */
+moe_status_t moe_grouped_gemm_gateup_preact(const moe_bf16_t* a, const moe_bf16_t* w_gateup,
+                                            const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* gu,
+                                            cudaStream_t stream);
+
+/* SwiGLU derivative: with s = 1 / (1 + exp(-g)), for every row and n < f
+ *   dgu[r][n] = dh[r][n] * u * s * (1 + g * (1 - s)),  dgu[r][f + n] = dh[r][n] * g * s,
+ * g = gu[r][n], u = gu[r][f + n]; fp32 arithmetic, bf16 in and out.
+ *   dh [M][f], gu [M][2f], dgu [M][2f]; f a positive multiple of 8. */
+moe_status_t moe_swiglu_backward(const moe_bf16_t* dh, const moe_bf16_t* gu, int M, int f, moe_bf16_t* dgu,
+                                 cudaStream_t stream);
+
+/* Gradient of moe_unpermute_combine: for assignment a = t*k+j and its row
+ * r = inv_perm[a], dy_perm[r] = bf16(topk_w[a] * dy[t]) and dw[a] = sum_c
+ * dy[t][c] * y_perm[r][c] (fp32, fixed order).
+ *   dy [T][d], y_perm [T*k][d] (the forward's), dy_perm [T*k][d] bf16; dw [T][k] fp32.
+ * Limits as moe_unpermute_combine. */
+moe_status_t moe_permute_backward(const moe_bf16_t* dy, const int32_t* inv_perm, const float* topk_w,
+                                  const moe_bf16_t* y_perm, int T, int d, int k, moe_bf16_t* dy_perm, float* dw,
+                                  cudaStream_t stream);
+
+/* wt[g][c][r] = w[g][r][c]: per-expert transposed copies of the weights, for the
+ * backward GEMMs (W_down [E][d][f] -> [E][f][d], W_gateup [E][2f][d] -> [E][d][2f]).
+ * Not in place. G <= 65535, rows <= 2,097,120. */
+moe_status_t moe_transpose_weights(const moe_bf16_t* w, int G, int rows, int cols, moe_bf16_t* wt,
+                                   cudaStream_t stream);
+
+/* Bytes of workspace moe_grouped_weight_grad needs (a multiple of 256). */
+size_t moe_grouped_weight_grad_workspace_size(int M, int G, int P, int Q);
+
+/* Weight gradient of a grouped projection, a GEMM grouped over its reduction
+ * axis: dw[g][p][q] = sum over rows r of group g of a[r][p] * b[r][q], fp32
+ * (bf16 products, fp32 accumulation in row order blocks of 64), one output tile
+ * per CTA pair over the group's whole range (deterministic). An empty group
+ * gets zeros.
+ *   a [M][P], b [M][Q] bf16 (rows grouped by group_offsets [G+1], device)
+ *   dw [G][P][Q] fp32
+ *   ws, ws_bytes   workspace of moe_grouped_weight_grad_workspace_size(M, G, P, Q)
+ *                  bytes, 256-byte aligned (the transposed, per-group
+ *                  zero-padded operands)
+ * Limits: 1 <= G <= 1024, P and Q positive multiples of 8. */
+moe_status_t moe_grouped_weight_grad(const moe_bf16_t* a, const moe_bf16_t* b, const int32_t* group_offsets, int G,
+                                     int M, int P, int Q, float* dw, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Bytes of workspace moe_router_backward needs. */
+size_t moe_router_backward_workspace_size(int T, int k);
+
+/* Router backward, the top-k selection held fixed. From dw (the routing
+ * weights' gradient, moe_permute_backward) the gradient of each selected
+ * logit: softmax over the selected logits (also SOFTMAX_TOPK_RENORM, the same
+ * function of them) dl_j = w_j (dw_j - sum_i w_i dw_i); sigmoid normalised,
+ * with s_i = sigmoid(l_i) and S = sum s_i, dl_i = (dw_i - sum_j w_j dw_j) / S *
+ * s_i (1 - s_i). Then
+ *   dw_router[e][c] = sum over tokens t selecting e of dl * x[t][c]   (fp32)
+ *   dbias[e]        = sum over tokens t selecting e of dl             (fp32; NULL: skipped)
+ *   dx[t][c]        = dx_addend[t][c] + sum_j dl_j * w_router[e_j][c] (bf16; dx_addend may be NULL)
+ * The sums over tokens run over the grouped rows (perm_src, expert_offsets of
+ * moe_permute) in order: deterministic.
+ *   logits [T][E] fp32 (the forward's), topk_idx / topk_w / dw [T][k],
+ *   perm_src / inv_perm [T*k], expert_offsets [E+1], ws of
+ *   moe_router_backward_workspace_size(T, k) bytes, 256-byte aligned.
+ * Limits as moe_route_topk. */
+moe_status_t moe_router_backward(const moe_bf16_t* x, const float* w_router, const float* logits,
+                                 const int32_t* topk_idx, const float* topk_w, const float* dw,
+                                 const int32_t* perm_src, const int32_t* inv_perm, const int32_t* expert_offsets,
+                                 int T, int d, int E, int k, moe_route_mode_t mode, const moe_bf16_t* dx_addend,
+                                 moe_bf16_t* dx, float* dw_router, float* dbias, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream);
+
 /* ---- Measurement and test hook ----
  * The bf16 grouped GEMMs (moe_grouped_gemm_gateup / _down) pick one of
  * several kernel families from the problem's shape. All of them compute the

@@ -25,7 +25,10 @@ ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm":
 EXPORTS = ("moe_route_topk", "moe_router_split_weights", "moe_route_topk_split", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
            "moe_permute_static_ws",
            "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_mxfp4_quantize", "moe_grouped_gemm_gateup_mxfp4",
-           "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_set_gemm_kernel", "moe_test_set_wait", "moe_get_device_error",
+           "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_grouped_gemm_gateup_preact",
+           "moe_swiglu_backward", "moe_permute_backward", "moe_transpose_weights",
+           "moe_grouped_weight_grad_workspace_size", "moe_grouped_weight_grad", "moe_router_backward_workspace_size",
+           "moe_router_backward", "moe_set_gemm_kernel", "moe_test_set_wait", "moe_get_device_error",
            "moe_last_error_string")
 GEMM_KERNELS = {"auto": 0, "single": 1, "pair": 2, "wide": 3, "swap": 4}
 
@@ -56,6 +59,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_gemm_gateup_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_down_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_unpermute_combine": [vp, vp, vp, vp, ci, ci, ci, vp, vp],
+        "moe_grouped_gemm_gateup_preact": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_swiglu_backward": [vp, vp, ci, ci, vp, vp],
+        "moe_permute_backward": [vp, vp, vp, vp, ci, ci, ci, vp, vp, vp],
+        "moe_transpose_weights": [vp, ci, ci, ci, vp, vp],
+        "moe_grouped_weight_grad_workspace_size": [ci, ci, ci, ci],
+        "moe_grouped_weight_grad": [vp, vp, vp, ci, ci, ci, ci, vp, vp, sz, vp],
+        "moe_router_backward_workspace_size": [ci, ci],
+        "moe_router_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, sz, vp],
         "moe_set_gemm_kernel": [ci],
         "moe_test_set_wait": [ctypes.c_ulonglong, ci],
         "moe_get_device_error": [ctypes.POINTER(ctypes.c_uint), vp],
@@ -66,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn.argtypes = args
         fn.restype = ci
     lib.moe_permute_workspace_size.restype = sz
+    lib.moe_grouped_weight_grad_workspace_size.restype = sz
+    lib.moe_router_backward_workspace_size.restype = sz
     lib.moe_last_error_string.restype = ctypes.c_char_p
     return lib
 
@@ -260,6 +273,99 @@ def unpermute_combine(y_perm, inv_perm, topk_w, shared, y, stream=None):
     _need(y, torch.bfloat16, (T, d), "y")
     _check(_lib.moe_unpermute_combine(_p(y_perm), _p(inv_perm), _p(topk_w), _p(shared), T, d, k, _p(y),
                                       _stream(stream)), "moe_unpermute_combine")
+
+
+# ---- backward ----
+
+def grouped_gemm_gateup_preact(a, w_gateup, group_offsets, gu, stream=None):
+    """gu [M, 2f] <- the gate (columns [0, f)) and up (columns [f, 2f)) pre-activations of the grouped projection."""
+    M, d = a.shape
+    G, two_f, _ = w_gateup.shape
+    f = two_f // 2
+    _need(a, torch.bfloat16, (M, d), "a")
+    _need(w_gateup, torch.bfloat16, (G, 2 * f, d), "w_gateup")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(gu, torch.bfloat16, (M, 2 * f), "gu")
+    _check(_lib.moe_grouped_gemm_gateup_preact(_p(a), _p(w_gateup), _p(group_offsets), G, M, d, f, _p(gu),
+                                               _stream(stream)), "moe_grouped_gemm_gateup_preact")
+
+
+def swiglu_backward(dh, gu, dgu, stream=None):
+    M, f = dh.shape
+    _need(dh, torch.bfloat16, (M, f), "dh")
+    _need(gu, torch.bfloat16, (M, 2 * f), "gu")
+    _need(dgu, torch.bfloat16, (M, 2 * f), "dgu")
+    _check(_lib.moe_swiglu_backward(_p(dh), _p(gu), M, f, _p(dgu), _stream(stream)), "moe_swiglu_backward")
+
+
+def permute_backward(dy, inv_perm, topk_w, y_perm, dy_perm, dw, stream=None):
+    T, d = dy.shape
+    k = topk_w.shape[1]
+    _need(dy, torch.bfloat16, (T, d), "dy")
+    _need(inv_perm, torch.int32, (T * k,), "inv_perm")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    _need(y_perm, torch.bfloat16, (T * k, d), "y_perm")
+    _need(dy_perm, torch.bfloat16, (T * k, d), "dy_perm")
+    _need(dw, torch.float32, (T, k), "dw")
+    _check(_lib.moe_permute_backward(_p(dy), _p(inv_perm), _p(topk_w), _p(y_perm), T, d, k, _p(dy_perm), _p(dw),
+                                     _stream(stream)), "moe_permute_backward")
+
+
+def transpose_weights(w, wt, stream=None):
+    """wt [G, C, R] <- per-group transpose of w [G, R, C] (bf16)."""
+    G, R, C = w.shape
+    _need(w, torch.bfloat16, (G, R, C), "w")
+    _need(wt, torch.bfloat16, (G, C, R), "wt")
+    _check(_lib.moe_transpose_weights(_p(w), G, R, C, _p(wt), _stream(stream)), "moe_transpose_weights")
+
+
+def grouped_weight_grad_workspace_size(M: int, G: int, P: int, Q: int) -> int:
+    return int(_lib.moe_grouped_weight_grad_workspace_size(M, G, P, Q))
+
+
+def grouped_weight_grad(a, b, group_offsets, dw, ws, stream=None):
+    """dw [G, P, Q] fp32 <- for each group g: sum over its rows of a[r]^T b[r] (a [M, P], b [M, Q] bf16)."""
+    M, P = a.shape
+    Q = b.shape[1]
+    G = group_offsets.shape[0] - 1
+    _need(a, torch.bfloat16, (M, P), "a")
+    _need(b, torch.bfloat16, (M, Q), "b")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(dw, torch.float32, (G, P, Q), "dw")
+    ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.moe_grouped_weight_grad(_p(a), _p(b), _p(group_offsets), G, M, P, Q, _p(dw), _p(ws), ws_bytes,
+                                        _stream(stream)), "moe_grouped_weight_grad")
+
+
+def router_backward_workspace_size(T: int, k: int) -> int:
+    return int(_lib.moe_router_backward_workspace_size(T, k))
+
+
+def router_backward(x, w_router, logits, topk_idx, topk_w, dw, perm_src, inv_perm, expert_offsets, mode, dx,
+                    dw_router, dbias=None, dx_addend=None, ws=None, stream=None):
+    T, d = x.shape
+    E = w_router.shape[0]
+    k = topk_idx.shape[1]
+    _need(x, torch.bfloat16, (T, d), "x")
+    _need(w_router, torch.float32, (E, d), "w_router")
+    _need(logits, torch.float32, (T, E), "logits")
+    _need(topk_idx, torch.int32, (T, k), "topk_idx")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    _need(dw, torch.float32, (T, k), "dw")
+    _need(perm_src, torch.int32, (T * k,), "perm_src")
+    _need(inv_perm, torch.int32, (T * k,), "inv_perm")
+    _need(expert_offsets, torch.int32, (E + 1,), "expert_offsets")
+    _need(dx, torch.bfloat16, (T, d), "dx")
+    _need(dw_router, torch.float32, (E, d), "dw_router")
+    if dbias is not None:
+        _need(dbias, torch.float32, (E,), "dbias")
+    if dx_addend is not None:
+        _need(dx_addend, torch.bfloat16, (T, d), "dx_addend")
+    ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.moe_router_backward(_p(x), _p(w_router), _p(logits), _p(topk_idx), _p(topk_w), _p(dw), _p(perm_src),
+                                    _p(inv_perm), _p(expert_offsets), T, d, E, k, ROUTE_MODES[mode], _p(dx_addend),
+                                    _p(dx), _p(dw_router), _p(dbias), _p(ws), ws_bytes, _stream(stream)),
+           "moe_router_backward")
 
 
 def set_gemm_kernel(name: str) -> None:

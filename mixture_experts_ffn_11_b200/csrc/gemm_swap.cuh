@@ -124,7 +124,9 @@ __device__ __forceinline__ int swap_box_index(int half) {
 // and the matching 64 up rows), down as [G][d][K] with box {64, 128, 1}; with BIGBOX the same views with a K-block
 // dimension {64, rows.., K/64} boxing SUB K blocks. tmX: the token rows, [M][K] (or [K/64][M][64] with BIGBOX).
 // tmO: the output [M][n_out], 32 x 32 boxes, 64-byte swizzle.
-template <bool GATEUP, int SUB, int STAGES, bool BIGBOX>
+// RAW (gate|up only): no SwiGLU; every warp stores its own lanes, gate rows to columns [0, f) and up rows to
+// columns [f, 2f) of an [M][2f] output (the pre-activations a backward pass needs).
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ SwapMaps tmX,
                              const __grid_constant__ CUtensorMap tmO, const GemmArgs args, int weights_streamed_once) {
@@ -355,10 +357,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
         const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
         // gate|up: the warps of lanes 0-63 (q = 0, 1: gate rows) hand their values to the warps of lanes 64-127
         // (q = 2, 3: up rows), which compute and store h
-        const bool ferry = GATEUP && q < 2;
+        const bool ferry = GATEUP && !RAW && q < 2;
         const int p = q & 1;  // hand-off pair (gate|up)
         uint8_t* xbuf = epi + 8192 + p * 4096;
-        uint8_t* stage_base = epi + (GATEUP ? p : (warp - 2)) * 4096;
+        uint8_t* stage_base = epi + ((GATEUP && !RAW) ? p : (warp - 2)) * 4096;
+        // output row stride and this warp's column limit: RAW gate|up stores gate rows below f, up rows from f on
+        const int ld_out = RAW ? 2 * args.f : args.n_out;
+        const int col_off = (RAW && q >= 2) ? args.f : 0;
+        const int col_end = RAW ? col_off + args.f : args.n_out;
         int acc = 0;
         uint32_t acc_phase = 0;
         uint32_t blocks = 0;  // blocks staged (alternating buffers) or handed off by this warp
@@ -373,13 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
             tc_fence_after_sync();
             const uint32_t t_acc = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * GS_MAX_N);
             // output columns of this warp's lanes
-            const int col0 = GATEUP ? wb * 128 + 64 * (int)rank + 32 * p : wb * 256 + 128 * (int)rank + 32 * q;
+            const int col0 = col_off + (GATEUP ? wb * 128 + 64 * (int)rank + 32 * p : wb * 256 + 128 * (int)rank + 32 * q);
 #pragma unroll 1
             for (int c0 = 0; c0 < rows && ok; c0 += 32) {
                 uint32_t raw[32];
                 tmem_load_32cols(t_acc + (uint32_t)c0, raw);
                 float v[32];
-                if constexpr (GATEUP) {
+                if constexpr (GATEUP && !RAW) {
                     const uint32_t par = blocks & 1u;
                     if (ferry) {
                         // hand off: thread = gate row, 32 token values as eight 16-byte units, XOR-swizzled by lane
@@ -420,7 +426,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                 if (lane == 0) bulk_wait_group_read<1>();  // the TMA store that last read this buffer is done
                 __syncwarp();
                 stage_transposed(my_stage, v, lane);
-                flush_staged_block(my_stage, lane, &tmO, args.out, args.n_out, r0 + c0, row_end, col0, args.n_out);
+                flush_staged_block(my_stage, lane, &tmO, args.out, ld_out, r0 + c0, row_end, col0, col_end);
             }
             if (!ok) break;
             tc_fence_before_sync();

@@ -21,6 +21,8 @@
 #include "gemm_wide.cuh"
 #include "gemm_swap.cuh"
 #include "gemm_fp4.cuh"
+#include "gemm_wgrad.cuh"
+#include "backward.cuh"
 #include "combine.cuh"
 
 using namespace moe;
@@ -113,6 +115,11 @@ cudaError_t set_gemm_attributes() {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, false>, a, SwapDN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true>, a, SwapGU::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, true>, a, SwapDN::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, false, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_wgrad_kernel, a, GemmWgradShape::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<16, true>, a, GemmFp4Shape<16, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<32, true>, a, GemmFp4Shape<32, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<64, true>, a, GemmFp4Shape<64, true>::SMEM_BYTES);
@@ -307,7 +314,7 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)", e);
 }
 
-template <bool GATEUP, int SUB, int STAGES, bool BIGBOX>
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false>
 moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
     using S = GemmSwapShape<GATEUP, SUB, STAGES>;
     CUtensorMap tw, to;
@@ -352,15 +359,24 @@ moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
             st = make_tmap(&tx.x[i], p.a, 2, xdims, xstr, xbox);
         }
     }
-    if (st == MOE_OK) st = make_out_map(p, &to);
+    if (st == MOE_OK) {
+        if (RAW) {  // [M][2f] pre-activations: gate in columns [0, f), up in [f, 2f)
+            GemmProblem q = p;
+            q.n_out = 2 * p.f;
+            st = make_out_map(q, &to);
+        } else {
+            st = make_out_map(p, &to);
+        }
+    }
     if (st != MOE_OK) return st;
     const GemmArgs args = gemm_args(p, S::TILE_W);
     const long upper = ((long)p.M / GS_MAX_N + p.G) * (long)args.n_tiles;  // >= the real tile count
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GS_MAX_N ? 1 : 0;
-    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX>, dim3(2 * clusters),
+    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX, RAW>, dim3(2 * clusters),
                                      dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, args, streamed_once);
-    return check_launch(GATEUP ? "grouped_gemm_gateup (swap pair)" : "grouped_gemm_down (swap pair)", e);
+    return check_launch(RAW ? "grouped_gemm_gateup_preact (swap pair)"
+                            : (GATEUP ? "grouped_gemm_gateup (swap pair)" : "grouped_gemm_down (swap pair)"), e);
 }
 
 template <bool GATEUP>
@@ -860,6 +876,195 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
                                      reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
                                      reinterpret_cast<__nv_bfloat16*>(y));
     return check_launch("unpermute_combine", e);
+}
+
+// ---- backward ----
+
+moe_status_t moe_grouped_gemm_gateup_preact(const moe_bf16_t* a, const moe_bf16_t* w_gateup,
+                                            const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* gu,
+                                            cudaStream_t stream) {
+    moe_status_t st = check_gemm_args(a, w_gateup, group_offsets, G, M, d, f, gu);
+    if (st != MOE_OK) return st;
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    if (di.sms < 2) return fail(MOE_ERR_UNSUPPORTED, "the pre-activation GEMM needs CTA pairs");
+    const GemmProblem p{a, w_gateup, group_offsets, G, M, d, f, f, gu};
+    if (d % GG_BK == 0) return launch_swap<true, 2, 3, true, true>(p, di.sms, stream);
+    return launch_swap<true, 2, 3, false, true>(p, di.sms, stream);
+}
+
+moe_status_t moe_swiglu_backward(const moe_bf16_t* dh, const moe_bf16_t* gu, int M, int f, moe_bf16_t* dgu,
+                                 cudaStream_t stream) {
+    if (M < 0 || f < 8 || f % 8) return fail(MOE_ERR_INVALID_ARG, "M=%d, f=%d (f a positive multiple of 8)", M, f);
+    if (M == 0) return MOE_OK;
+    if (!dh || !gu || !dgu) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(dh) || !aligned16(gu) || !aligned16(dgu)) return fail(MOE_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const long items = (long)M * (f / 8);
+    const cudaError_t e = launch_pdl(swiglu_backward_kernel, dim3(grid_cap((items + 255) / 256, di.sms, 8)), dim3(256),
+                                     0, stream, reinterpret_cast<const __nv_bfloat16*>(dh),
+                                     reinterpret_cast<const __nv_bfloat16*>(gu), (long)M, f,
+                                     reinterpret_cast<__nv_bfloat16*>(dgu));
+    return check_launch("swiglu_backward", e);
+}
+
+moe_status_t moe_permute_backward(const moe_bf16_t* dy, const int32_t* inv_perm, const float* topk_w,
+                                  const moe_bf16_t* y_perm, int T, int d, int k, moe_bf16_t* dy_perm, float* dw,
+                                  cudaStream_t stream) {
+    if (T < 0 || k < 1 || k > 32) return fail(MOE_ERR_INVALID_ARG, "T=%d, k=%d (need T >= 0, 1 <= k <= 32)", T, k);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if ((long)T * k > 0x7fffffffL) return fail(MOE_ERR_INVALID_ARG, "T*k exceeds int32");
+    if (T == 0) return MOE_OK;
+    if (!dy || !inv_perm || !topk_w || !y_perm || !dy_perm || !dw) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(dy) || !aligned16(y_perm) || !aligned16(dy_perm))
+        return fail(MOE_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const long R = (long)T * k;
+    const cudaError_t e = launch_pdl(permute_backward_kernel, dim3(grid_cap((R + PB_WARPS - 1) / PB_WARPS, di.sms, 16)),
+                                     dim3(PB_WARPS * 32), 0, stream, reinterpret_cast<const __nv_bfloat16*>(dy),
+                                     inv_perm, topk_w, reinterpret_cast<const __nv_bfloat16*>(y_perm), T, d, k,
+                                     reinterpret_cast<__nv_bfloat16*>(dy_perm), dw);
+    return check_launch("permute_backward", e);
+}
+
+moe_status_t moe_transpose_weights(const moe_bf16_t* w, int G, int rows, int cols, moe_bf16_t* wt,
+                                   cudaStream_t stream) {
+    if (G < 0 || rows < 0 || cols < 0 || G > 65535) return fail(MOE_ERR_INVALID_ARG, "G=%d, rows=%d, cols=%d", G, rows, cols);
+    if (G == 0 || rows == 0 || cols == 0) return MOE_OK;
+    if (!w || !wt) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (w == wt) return fail(MOE_ERR_INVALID_ARG, "the transpose cannot be done in place");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const dim3 grid((cols + 31) / 32, (rows + 31) / 32, G);
+    if (grid.y > 65535) return fail(MOE_ERR_INVALID_ARG, "rows=%d too large", rows);
+    const cudaError_t e = launch_pdl(transpose_kernel, grid, dim3(256), 0, stream,
+                                     reinterpret_cast<const __nv_bfloat16*>(w), rows, cols,
+                                     reinterpret_cast<__nv_bfloat16*>(wt));
+    return check_launch("transpose", e);
+}
+
+namespace {
+long wgrad_cap(int M, int G) { return ((long)M + (long)(WG_PAD - 1) * G + WG_PAD - 1) / WG_PAD * WG_PAD; }
+size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+}  // namespace
+
+size_t moe_grouped_weight_grad_workspace_size(int M, int G, int P, int Q) {
+    if (M <= 0 || G <= 0 || P <= 0 || Q <= 0) return 0;
+    const long cap = wgrad_cap(M, G);
+    return round256((size_t)(G + 1) * 4) + round256((size_t)P * cap * 2) + round256((size_t)Q * cap * 2);
+}
+
+moe_status_t moe_grouped_weight_grad(const moe_bf16_t* a, const moe_bf16_t* b, const int32_t* group_offsets, int G,
+                                     int M, int P, int Q, float* dw, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (G < 1 || G > GG_MAX_GROUPS) return fail(MOE_ERR_INVALID_ARG, "G=%d outside [1, %d]", G, GG_MAX_GROUPS);
+    if (M < 0) return fail(MOE_ERR_INVALID_ARG, "M=%d < 0", M);
+    if (P < 8 || Q < 8 || P % 8 || Q % 8) return fail(MOE_ERR_INVALID_ARG, "P=%d and Q=%d must be positive multiples of 8", P, Q);
+    if (!group_offsets || !dw || (M > 0 && (!a || !b))) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(a) || !aligned16(b) || !aligned16(dw)) return fail(MOE_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(group_offsets) & 3u) != 0) return fail(MOE_ERR_INVALID_ARG, "offsets misaligned");
+    const int Mw = M > 0 ? M : 1;
+    const size_t need = moe_grouped_weight_grad_workspace_size(Mw, G, P, Q);
+    if (!ws || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    if (di.sms < 2) return fail(MOE_ERR_UNSUPPORTED, "the weight-gradient GEMM needs CTA pairs");
+    const long cap = wgrad_cap(Mw, G);
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    int32_t* pad_off = reinterpret_cast<int32_t*>(base);
+    __nv_bfloat16* aT = reinterpret_cast<__nv_bfloat16*>(base + round256((size_t)(G + 1) * 4));
+    __nv_bfloat16* bT = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(aT) + round256((size_t)P * cap * 2));
+    cudaError_t e = launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, stream, group_offsets, G, M, pad_off);
+    if ((st = check_launch("pad_offsets", e)) != MOE_OK) return st;
+    if (M > 0) {
+        if (cap / 32 > 65535) return fail(MOE_ERR_INVALID_ARG, "M=%d too large for the weight-gradient transpose", M);
+        e = launch_pdl(transpose_pad_kernel, dim3((P + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
+                       reinterpret_cast<const __nv_bfloat16*>(a), group_offsets, (const int32_t*)pad_off, G, M, P, cap, aT);
+        if ((st = check_launch("transpose_pad", e)) != MOE_OK) return st;
+        e = launch_pdl(transpose_pad_kernel, dim3((Q + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
+                       reinterpret_cast<const __nv_bfloat16*>(b), group_offsets, (const int32_t*)pad_off, G, M, Q, cap, bT);
+        if ((st = check_launch("transpose_pad", e)) != MOE_OK) return st;
+    }
+    CUtensorMap ta, tb, to;
+    const cuuint64_t adims[2] = {(cuuint64_t)cap, (cuuint64_t)P};
+    const cuuint64_t astr[1] = {(cuuint64_t)cap * 2};
+    const cuuint32_t box[2] = {GG_BK, 128};
+    if ((st = make_tmap(&ta, aT, 2, adims, astr, box)) != MOE_OK) return st;
+    const cuuint64_t bdims[2] = {(cuuint64_t)cap, (cuuint64_t)Q};
+    if ((st = make_tmap(&tb, bT, 2, bdims, astr, box)) != MOE_OK) return st;
+    const cuuint64_t odims[3] = {(cuuint64_t)Q, (cuuint64_t)P, (cuuint64_t)G};
+    const cuuint64_t ostr[2] = {(cuuint64_t)Q * 4, (cuuint64_t)P * Q * 4};
+    const cuuint32_t obox[3] = {32, 32, 1};
+    if ((st = make_tmap(&to, dw, 3, odims, ostr, obox, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B)) !=
+        MOE_OK)
+        return st;
+    WgradArgs args;
+    args.pad_off = pad_off;
+    args.G = G;
+    args.P = P;
+    args.Q = Q;
+    const long tiles = (long)G * ((P + WG_TILE - 1) / WG_TILE) * ((Q + WG_TILE - 1) / WG_TILE);
+    const int clusters = (int)(tiles < di.sms / 2 ? tiles : di.sms / 2);
+    e = launch_pdl(grouped_wgrad_kernel, dim3(2 * clusters), dim3(WG_THREADS), GemmWgradShape::SMEM_BYTES, stream, ta,
+                   tb, to, args);
+    return check_launch("grouped_weight_grad", e);
+}
+
+size_t moe_router_backward_workspace_size(int T, int k) {
+    if (T <= 0 || k <= 0) return 0;
+    return round256((size_t)T * k * 4) * 2;
+}
+
+moe_status_t moe_router_backward(const moe_bf16_t* x, const float* w_router, const float* logits,
+                                 const int32_t* topk_idx, const float* topk_w, const float* dw,
+                                 const int32_t* perm_src, const int32_t* inv_perm, const int32_t* expert_offsets,
+                                 int T, int d, int E, int k, moe_route_mode_t mode, const moe_bf16_t* dx_addend,
+                                 moe_bf16_t* dx, float* dw_router, float* dbias, void* ws, size_t ws_bytes,
+                                 cudaStream_t stream) {
+    moe_status_t st = check_route_sizes(T, E, k);
+    if (st != MOE_OK) return st;
+    if (mode < MOE_ROUTE_TOPK_SOFTMAX || mode > MOE_ROUTE_SIGMOID_TOPK_NORM)
+        return fail(MOE_ERR_INVALID_ARG, "unknown routing mode %d", (int)mode);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (!dw_router || !expert_offsets) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (T == 0) {  // no tokens: the router's weight gradient (and the bias gradient) is zero
+        cudaError_t e = cudaMemsetAsync(dw_router, 0, sizeof(float) * (size_t)E * d, stream);
+        if (e == cudaSuccess && dbias) e = cudaMemsetAsync(dbias, 0, sizeof(float) * (size_t)E, stream);
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+        return MOE_OK;
+    }
+    if (!x || !w_router || !logits || !topk_idx || !topk_w || !dw || !perm_src || !inv_perm || !dx)
+        return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(dx) || (dx_addend && !aligned16(dx_addend)))
+        return fail(MOE_ERR_INVALID_ARG, "x, w_router, dx and dx_addend must be 16-byte aligned");
+    const size_t need = moe_router_backward_workspace_size(T, k);
+    if (!ws || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
+    float* dl_tk = reinterpret_cast<float*>(ws);
+    float* dl_perm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)T * k * 4));
+    const int R = T * k;
+    cudaError_t e = launch_pdl(router_dlogits_kernel, dim3(grid_cap((T + 255) / 256, di.sms, 4)), dim3(256), 0,
+                               stream, logits, topk_idx, topk_w, dw, inv_perm, T, E, k, (int)mode, dl_tk, dl_perm);
+    if ((st = check_launch("router_dlogits", e)) != MOE_OK) return st;
+    e = launch_pdl(router_weight_grad_kernel, dim3((d + RB_COLS - 1) / RB_COLS, E), dim3(RB_COLS), 0, stream,
+                   reinterpret_cast<const __nv_bfloat16*>(x), perm_src, expert_offsets, (const float*)dl_perm, T, d, E,
+                   R, dw_router, dbias);
+    if ((st = check_launch("router_weight_grad", e)) != MOE_OK) return st;
+    e = launch_pdl(router_input_grad_kernel, dim3(grid_cap((T + 7) / 8, di.sms, 16)), dim3(256), 0, stream, topk_idx,
+                   (const float*)dl_tk, w_router, reinterpret_cast<const __nv_bfloat16*>(dx_addend), T, d, E, k,
+                   reinterpret_cast<__nv_bfloat16*>(dx));
+    return check_launch("router_input_grad", e);
 }
 
 moe_status_t moe_set_gemm_kernel(moe_gemm_kernel_t kind) {

@@ -121,6 +121,7 @@ class MoEFFN:
         T = x.shape[0]
         b = self.buffers(T)
         s = stream if stream is not None else torch.cuda.current_stream(x.device)
+        self._x = x  # the backward pass reads the forward's input and intermediates
 
         def mark(name, first):
             if timing is None:
@@ -187,6 +188,105 @@ class MoEFFN:
         else:
             w = self.w_down if which == "routed" else self.w_down_shared.unsqueeze(0)
             N.grouped_gemm_down(h, w, offsets, y, stream)
+
+    # ---- training: gradients of the last forward() call ----------------------------------------------------
+
+    def _transposed(self):
+        """Per-expert transposed weight copies for the backward GEMMs, made once (call refresh_backward after
+        changing the weights in place)."""
+        if getattr(self, "_wt", None) is None:
+            if self.weights != "bf16":
+                raise NotImplementedError("the backward pass needs the bf16 expert weights")
+            E, d, f = self.E, self.d, self.f
+            wt = {"down": torch.empty(E, f, d, dtype=torch.bfloat16, device=self.device),
+                  "gateup": torch.empty(E, d, 2 * f, dtype=torch.bfloat16, device=self.device)}
+            N.transpose_weights(self.w_down, wt["down"])
+            N.transpose_weights(self.w_gateup, wt["gateup"])
+            if self.shared_f:
+                fs = self.shared_f
+                wt["down_shared"] = torch.empty(1, fs, d, dtype=torch.bfloat16, device=self.device)
+                wt["gateup_shared"] = torch.empty(1, d, 2 * fs, dtype=torch.bfloat16, device=self.device)
+                N.transpose_weights(self.w_down_shared.unsqueeze(0), wt["down_shared"])
+                N.transpose_weights(self.w_gateup_shared.unsqueeze(0), wt["gateup_shared"])
+            self._wt = wt
+        return self._wt
+
+    def refresh_backward(self):
+        """Drop the transposed weight copies (rebuilt by the next backward)."""
+        self._wt = None
+
+    def _grad_buffers(self, T: int) -> dict:
+        if getattr(self, "_gT", None) == T:
+            return self._gbuf
+        dev, E, d, f, k = self.device, self.E, self.d, self.f, self.k
+        R = T * k
+        bf, f32 = torch.bfloat16, torch.float32
+        g = {"dy_perm": torch.empty(R, d, dtype=bf, device=dev), "dtopk_w": torch.empty(T, k, dtype=f32, device=dev),
+             "dh": torch.empty(R, f, dtype=bf, device=dev), "gu": torch.empty(R, 2 * f, dtype=bf, device=dev),
+             "dgu": torch.empty(R, 2 * f, dtype=bf, device=dev), "dx_perm": torch.empty(R, d, dtype=bf, device=dev),
+             "dx_router": torch.empty(T, d, dtype=bf, device=dev), "dx": torch.empty(T, d, dtype=bf, device=dev),
+             "ones": torch.ones(T, k, dtype=f32, device=dev),
+             "router_ws": torch.empty(max(N.router_backward_workspace_size(T, k), 256), dtype=torch.uint8, device=dev),
+             "dw_router": torch.empty(E, d, dtype=f32, device=dev),
+             "dbias": torch.empty(E, dtype=f32, device=dev) if self.bias is not None else None,
+             "dw_down": torch.empty(E, d, f, dtype=f32, device=dev),
+             "dw_gateup": torch.empty(E, 2 * f, d, dtype=f32, device=dev)}
+        wsz = max(N.grouped_weight_grad_workspace_size(max(R, 1), E, d, f),
+                  N.grouped_weight_grad_workspace_size(max(R, 1), E, 2 * f, d))
+        if self.shared_f:
+            fs = self.shared_f
+            g.update({"dh_s": torch.empty(T, fs, dtype=bf, device=dev), "gu_s": torch.empty(T, 2 * fs, dtype=bf, device=dev),
+                      "dgu_s": torch.empty(T, 2 * fs, dtype=bf, device=dev), "dx_s": torch.empty(T, d, dtype=bf, device=dev),
+                      "dw_down_shared": torch.empty(1, d, fs, dtype=f32, device=dev),
+                      "dw_gateup_shared": torch.empty(1, 2 * fs, d, dtype=f32, device=dev)})
+            wsz = max(wsz, N.grouped_weight_grad_workspace_size(max(T, 1), 1, d, fs),
+                      N.grouped_weight_grad_workspace_size(max(T, 1), 1, 2 * fs, d))
+        g["wgrad_ws"] = torch.empty(max(wsz, 256), dtype=torch.uint8, device=dev)
+        self._gbuf, self._gT = g, T
+        return g
+
+    def backward(self, dy, stream=None, weight_grads: bool = True) -> dict:
+        """Gradients of the last forward() call for the upstream gradient dy [T, d] (bf16), the top-k selection
+        held fixed. Returns a dict of device tensors owned by the layer (overwritten by the next backward):
+        dx [T, d] bf16 (experts and router), dtopk_w [T, k] (routing weights), dw_router [E, d], dbias [E] (with
+        a router bias), and with weight_grads dw_gateup [E, 2f, d], dw_down [E, d, f] (fp32), plus the shared
+        expert's dw_gateup_shared [1, 2fs, d] and dw_down_shared [1, d, fs]."""
+        T = dy.shape[0]
+        if self._T != T or getattr(self, "_x", None) is None or self._x.shape[0] != T:
+            raise RuntimeError("backward() follows a forward() over the same tokens")
+        s = stream if stream is not None else torch.cuda.current_stream(dy.device)
+        b = self.buf
+        wt = self._transposed()
+        g = self._grad_buffers(T)
+        x = self._x
+        N.permute_backward(dy, b["inv_perm"], b["topk_w"], b["y_perm"], g["dy_perm"], g["dtopk_w"], s)
+        N.grouped_gemm_down(g["dy_perm"], wt["down"], b["offsets"], g["dh"], s)
+        N.grouped_gemm_gateup_preact(b["x_perm"], self.w_gateup, b["offsets"], g["gu"], s)
+        N.swiglu_backward(g["dh"], g["gu"], g["dgu"], s)
+        N.grouped_gemm_down(g["dgu"], wt["gateup"], b["offsets"], g["dx_perm"], s)
+        addend = None
+        if self.shared_f:
+            so = b["shared_offsets"]
+            N.grouped_gemm_down(dy, wt["down_shared"], so, g["dh_s"], s)
+            N.grouped_gemm_gateup_preact(x, self.w_gateup_shared.unsqueeze(0), so, g["gu_s"], s)
+            N.swiglu_backward(g["dh_s"], g["gu_s"], g["dgu_s"], s)
+            N.grouped_gemm_down(g["dgu_s"], wt["gateup_shared"], so, g["dx_s"], s)
+            addend = g["dx_s"]
+        N.router_backward(x, self.w_router, b["logits"], b["topk_idx"], b["topk_w"], g["dtopk_w"], b["perm_src"],
+                          b["inv_perm"], b["offsets"], self.route, g["dx_router"], g["dw_router"], g["dbias"], addend,
+                          g["router_ws"], s)
+        N.unpermute_combine(g["dx_perm"], b["inv_perm"], g["ones"], g["dx_router"], g["dx"], s)
+        out = {"dx": g["dx"], "dtopk_w": g["dtopk_w"], "dw_router": g["dw_router"], "dbias": g["dbias"]}
+        if weight_grads:
+            N.grouped_weight_grad(g["dy_perm"], b["h"], b["offsets"], g["dw_down"], g["wgrad_ws"], s)
+            N.grouped_weight_grad(g["dgu"], b["x_perm"], b["offsets"], g["dw_gateup"], g["wgrad_ws"], s)
+            out["dw_down"], out["dw_gateup"] = g["dw_down"], g["dw_gateup"]
+            if self.shared_f:
+                so = b["shared_offsets"]
+                N.grouped_weight_grad(dy, b["h_shared"], so, g["dw_down_shared"], g["wgrad_ws"], s)
+                N.grouped_weight_grad(g["dgu_s"], x, so, g["dw_gateup_shared"], g["wgrad_ws"], s)
+                out["dw_down_shared"], out["dw_gateup_shared"] = g["dw_down_shared"], g["dw_gateup_shared"]
+        return out
 
     def kernel_launches(self, T: int) -> int:
         """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the
