@@ -99,6 +99,8 @@ def parse_args(argv=None):
     ap.add_argument("--gemm", choices=["auto", "single", "pair", "wide", "swap"], default="auto",
                     help="force a grouped-GEMM kernel family")
     ap.add_argument("--shape", default="", help="comma-separated workload overrides, e.g. T=1024,E=64 (profiling)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the training step: forward + backward with weight gradients (not the headline)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -430,6 +432,7 @@ def run_kernel(args):
 def run_ours(args):
     import torch
 
+    import synth
     from mixture_experts_ffn_11_b200 import _native as N
     from mixture_experts_ffn_11_b200 import get_device_error
 
@@ -447,8 +450,17 @@ def run_ours(args):
     sampler = ClockSampler(torch.cuda.get_device_properties(dev).uuid.__str__() if rank >= 0 else None)
     sampler.start()
 
+    dy = None
+    if args.backward:
+        dy = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
+        synth.fill_device(dy, wl.seed, synth.TID_DY, 0, synth.X_SIGMA)
+        launches_per_step += layer.backward_kernel_launches(wl.T)
+
     def step(timing=None):
-        return layer.forward(x, timing=timing)
+        y = layer.forward(x, timing=timing)
+        if dy is not None:
+            layer.backward(dy, timing=timing)
+        return y
 
     # warm-up: W steps, then keep the same load going for ~2 s so clocks and power settle
     for _ in range(args.warmup):
@@ -502,7 +514,7 @@ def run_ours(args):
     # neighbouring steps. Two buffer sets (layer objects sharing the weights) alternate; events order every
     # reuse of a buffer after the last reader of its previous contents.
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not args.backward:
         layers = [layer, layer.sibling()]
         x_host = [x.cpu().pin_memory() for _ in range(2)]
         y_host = [torch.empty(wl.T, wl.d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -583,7 +595,24 @@ def run_ours(args):
             "parallelism": "replicas" if world > 1 else "single GPU"}
     if args.gemm != "auto":
         line["gemm_family"] = args.gemm
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if args.backward:
+        # the training step: forward + backward (top-k selection held fixed), weight gradients included
+        R, d, f, fs = wl.R, wl.d, wl.f, wl.shared_f
+        bwd_flop = {"bwd_dh": 2.0 * R * d * f, "bwd_preact": 4.0 * R * d * f, "bwd_dx_perm": 4.0 * R * d * f,
+                    "bwd_dw_down": 2.0 * R * d * f, "bwd_dw_gateup": 4.0 * R * d * f}
+        train_flop = lflop + 16.0 * R * d * f + 16.0 * wl.T * d * fs
+        top = max(bwd_flop, key=lambda n: stages[n])  # the backward stage that takes longest
+        tr_roof = roofline_entry(top, {"flop": bwd_flop[top], "bytes": 0.0}, stages[top], peaks, peak_kind, None)
+        line.update({"metric": "MoE-layer training step (forward + backward) tokens/s and TFLOP/s, 1xB200",
+                     "training_step": {"flop": train_flop,
+                                       "achieved_tflops": round(train_flop / (ms_per_step * 1e-3) / 1e12, 2),
+                                       "frac_of_peak": round(train_flop / (ms_per_step * 1e-3) / 1e12 /
+                                                             peaks[peak_kind], 4)},
+                     "roofline_backward": tr_roof,
+                     "roofline_backward_all": {n: roofline_entry(n, {"flop": fl, "bytes": 0.0}, stages[n], peaks,
+                                                                 peak_kind, None)["frac"]
+                                               for n, fl in bwd_flop.items()}})
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.backward:
         line["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)

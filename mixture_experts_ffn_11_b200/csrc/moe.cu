@@ -66,6 +66,22 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// The backward pass's elementwise, gather and transpose kernels are launched without programmatic stream
+// serialization: they start after the previous kernel ends. Measured on B200: the SwiGLU-derivative kernel launched
+// early as a programmatic dependent (of the pre-activation GEMM or of the combine) and followed by the CTA-pair
+// dx_perm GEMM stalled the stream within a few hundred layer steps; launched plainly it did not (thousands of steps).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_plain(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Grouped-GEMM configurations compiled into the library:
@@ -904,7 +920,7 @@ moe_status_t moe_swiglu_backward(const moe_bf16_t* dh, const moe_bf16_t* gu, int
     moe_status_t st = device_info(di);
     if (st != MOE_OK) return st;
     const long items = (long)M * (f / 8);
-    const cudaError_t e = launch_pdl(swiglu_backward_kernel, dim3(grid_cap((items + 255) / 256, di.sms, 8)), dim3(256),
+    const cudaError_t e = launch_plain(swiglu_backward_kernel, dim3(grid_cap((items + 255) / 256, di.sms, 8)), dim3(256),
                                      0, stream, reinterpret_cast<const __nv_bfloat16*>(dh),
                                      reinterpret_cast<const __nv_bfloat16*>(gu), (long)M, f,
                                      reinterpret_cast<__nv_bfloat16*>(dgu));
@@ -925,7 +941,7 @@ moe_status_t moe_permute_backward(const moe_bf16_t* dy, const int32_t* inv_perm,
     moe_status_t st = device_info(di);
     if (st != MOE_OK) return st;
     const long R = (long)T * k;
-    const cudaError_t e = launch_pdl(permute_backward_kernel, dim3(grid_cap((R + PB_WARPS - 1) / PB_WARPS, di.sms, 16)),
+    const cudaError_t e = launch_plain(permute_backward_kernel, dim3(grid_cap((R + PB_WARPS - 1) / PB_WARPS, di.sms, 16)),
                                      dim3(PB_WARPS * 32), 0, stream, reinterpret_cast<const __nv_bfloat16*>(dy),
                                      inv_perm, topk_w, reinterpret_cast<const __nv_bfloat16*>(y_perm), T, d, k,
                                      reinterpret_cast<__nv_bfloat16*>(dy_perm), dw);
@@ -943,7 +959,7 @@ moe_status_t moe_transpose_weights(const moe_bf16_t* w, int G, int rows, int col
     if (st != MOE_OK) return st;
     const dim3 grid((cols + 31) / 32, (rows + 31) / 32, G);
     if (grid.y > 65535) return fail(MOE_ERR_INVALID_ARG, "rows=%d too large", rows);
-    const cudaError_t e = launch_pdl(transpose_kernel, grid, dim3(256), 0, stream,
+    const cudaError_t e = launch_plain(transpose_kernel, grid, dim3(256), 0, stream,
                                      reinterpret_cast<const __nv_bfloat16*>(w), rows, cols,
                                      reinterpret_cast<__nv_bfloat16*>(wt));
     return check_launch("transpose", e);
@@ -982,14 +998,14 @@ moe_status_t moe_grouped_weight_grad(const moe_bf16_t* a, const moe_bf16_t* b, c
     int32_t* pad_off = reinterpret_cast<int32_t*>(base);
     __nv_bfloat16* aT = reinterpret_cast<__nv_bfloat16*>(base + round256((size_t)(G + 1) * 4));
     __nv_bfloat16* bT = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(aT) + round256((size_t)P * cap * 2));
-    cudaError_t e = launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, stream, group_offsets, G, M, pad_off);
+    cudaError_t e = launch_plain(pad_offsets_kernel, dim3(1), dim3(1024), 0, stream, group_offsets, G, M, pad_off);
     if ((st = check_launch("pad_offsets", e)) != MOE_OK) return st;
     if (M > 0) {
         if (cap / 32 > 65535) return fail(MOE_ERR_INVALID_ARG, "M=%d too large for the weight-gradient transpose", M);
-        e = launch_pdl(transpose_pad_kernel, dim3((P + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
+        e = launch_plain(transpose_pad_kernel, dim3((P + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
                        reinterpret_cast<const __nv_bfloat16*>(a), group_offsets, (const int32_t*)pad_off, G, M, P, cap, aT);
         if ((st = check_launch("transpose_pad", e)) != MOE_OK) return st;
-        e = launch_pdl(transpose_pad_kernel, dim3((Q + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
+        e = launch_plain(transpose_pad_kernel, dim3((Q + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
                        reinterpret_cast<const __nv_bfloat16*>(b), group_offsets, (const int32_t*)pad_off, G, M, Q, cap, bT);
         if ((st = check_launch("transpose_pad", e)) != MOE_OK) return st;
     }
@@ -1054,14 +1070,14 @@ moe_status_t moe_router_backward(const moe_bf16_t* x, const float* w_router, con
     float* dl_tk = reinterpret_cast<float*>(ws);
     float* dl_perm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)T * k * 4));
     const int R = T * k;
-    cudaError_t e = launch_pdl(router_dlogits_kernel, dim3(grid_cap((T + 255) / 256, di.sms, 4)), dim3(256), 0,
+    cudaError_t e = launch_plain(router_dlogits_kernel, dim3(grid_cap((T + 255) / 256, di.sms, 4)), dim3(256), 0,
                                stream, logits, topk_idx, topk_w, dw, inv_perm, T, E, k, (int)mode, dl_tk, dl_perm);
     if ((st = check_launch("router_dlogits", e)) != MOE_OK) return st;
-    e = launch_pdl(router_weight_grad_kernel, dim3((d + RB_COLS - 1) / RB_COLS, E), dim3(RB_COLS), 0, stream,
+    e = launch_plain(router_weight_grad_kernel, dim3((d + RB_COLS - 1) / RB_COLS, E), dim3(RB_COLS), 0, stream,
                    reinterpret_cast<const __nv_bfloat16*>(x), perm_src, expert_offsets, (const float*)dl_perm, T, d, E,
                    R, dw_router, dbias);
     if ((st = check_launch("router_weight_grad", e)) != MOE_OK) return st;
-    e = launch_pdl(router_input_grad_kernel, dim3(grid_cap((T + 7) / 8, di.sms, 16)), dim3(256), 0, stream, topk_idx,
+    e = launch_plain(router_input_grad_kernel, dim3(grid_cap((T + 7) / 8, di.sms, 16)), dim3(256), 0, stream, topk_idx,
                    (const float*)dl_tk, w_router, reinterpret_cast<const __nv_bfloat16*>(dx_addend), T, d, E, k,
                    reinterpret_cast<__nv_bfloat16*>(dx));
     return check_launch("router_input_grad", e);

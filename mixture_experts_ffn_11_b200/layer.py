@@ -245,12 +245,15 @@ class MoEFFN:
         self._gbuf, self._gT = g, T
         return g
 
-    def backward(self, dy, stream=None, weight_grads: bool = True) -> dict:
+    def backward(self, dy, stream=None, weight_grads: bool = True, timing=None) -> dict:
         """Gradients of the last forward() call for the upstream gradient dy [T, d] (bf16), the top-k selection
         held fixed. Returns a dict of device tensors owned by the layer (overwritten by the next backward):
         dx [T, d] bf16 (experts and router), dtopk_w [T, k] (routing weights), dw_router [E, d], dbias [E] (with
         a router bias), and with weight_grads dw_gateup [E, 2f, d], dw_down [E, d, f] (fp32), plus the shared
-        expert's dw_gateup_shared [1, 2fs, d] and dw_down_shared [1, d, fs]."""
+        expert's dw_gateup_shared [1, 2fs, d] and dw_down_shared [1, d, fs].
+        timing: optional dict; if given, (start, end) CUDA events are recorded around each stage ("bwd_permute",
+        "bwd_dh", "bwd_preact", "bwd_swiglu", "bwd_dx_perm", "bwd_shared", "bwd_router", "bwd_combine", "bwd_dw_down",
+        "bwd_dw_gateup", "bwd_dw_shared")."""
         T = dy.shape[0]
         if self._T != T or getattr(self, "_x", None) is None or self._x.shape[0] != T:
             raise RuntimeError("backward() follows a forward() over the same tokens")
@@ -259,34 +262,75 @@ class MoEFFN:
         wt = self._transposed()
         g = self._grad_buffers(T)
         x = self._x
+
+        def mark(name, first):
+            if timing is None:
+                return
+            if first:
+                timing[name] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            timing[name][0 if first else 1].record(s)
+
+        mark("bwd_permute", True)
         N.permute_backward(dy, b["inv_perm"], b["topk_w"], b["y_perm"], g["dy_perm"], g["dtopk_w"], s)
+        mark("bwd_permute", False)
+        mark("bwd_dh", True)
         N.grouped_gemm_down(g["dy_perm"], wt["down"], b["offsets"], g["dh"], s)
+        mark("bwd_dh", False)
+        mark("bwd_preact", True)
         N.grouped_gemm_gateup_preact(b["x_perm"], self.w_gateup, b["offsets"], g["gu"], s)
+        mark("bwd_preact", False)
+        mark("bwd_swiglu", True)
         N.swiglu_backward(g["dh"], g["gu"], g["dgu"], s)
+        mark("bwd_swiglu", False)
+        mark("bwd_dx_perm", True)
         N.grouped_gemm_down(g["dgu"], wt["gateup"], b["offsets"], g["dx_perm"], s)
+        mark("bwd_dx_perm", False)
         addend = None
         if self.shared_f:
+            mark("bwd_shared", True)
             so = b["shared_offsets"]
             N.grouped_gemm_down(dy, wt["down_shared"], so, g["dh_s"], s)
             N.grouped_gemm_gateup_preact(x, self.w_gateup_shared.unsqueeze(0), so, g["gu_s"], s)
             N.swiglu_backward(g["dh_s"], g["gu_s"], g["dgu_s"], s)
             N.grouped_gemm_down(g["dgu_s"], wt["gateup_shared"], so, g["dx_s"], s)
             addend = g["dx_s"]
+            mark("bwd_shared", False)
+        mark("bwd_router", True)
         N.router_backward(x, self.w_router, b["logits"], b["topk_idx"], b["topk_w"], g["dtopk_w"], b["perm_src"],
                           b["inv_perm"], b["offsets"], self.route, g["dx_router"], g["dw_router"], g["dbias"], addend,
                           g["router_ws"], s)
+        mark("bwd_router", False)
+        mark("bwd_combine", True)
         N.unpermute_combine(g["dx_perm"], b["inv_perm"], g["ones"], g["dx_router"], g["dx"], s)
+        mark("bwd_combine", False)
         out = {"dx": g["dx"], "dtopk_w": g["dtopk_w"], "dw_router": g["dw_router"], "dbias": g["dbias"]}
         if weight_grads:
+            mark("bwd_dw_down", True)
             N.grouped_weight_grad(g["dy_perm"], b["h"], b["offsets"], g["dw_down"], g["wgrad_ws"], s)
+            mark("bwd_dw_down", False)
+            mark("bwd_dw_gateup", True)
             N.grouped_weight_grad(g["dgu"], b["x_perm"], b["offsets"], g["dw_gateup"], g["wgrad_ws"], s)
+            mark("bwd_dw_gateup", False)
             out["dw_down"], out["dw_gateup"] = g["dw_down"], g["dw_gateup"]
             if self.shared_f:
+                mark("bwd_dw_shared", True)
                 so = b["shared_offsets"]
                 N.grouped_weight_grad(dy, b["h_shared"], so, g["dw_down_shared"], g["wgrad_ws"], s)
                 N.grouped_weight_grad(g["dgu_s"], x, so, g["dw_gateup_shared"], g["wgrad_ws"], s)
+                mark("bwd_dw_shared", False)
                 out["dw_down_shared"], out["dw_gateup_shared"] = g["dw_down_shared"], g["dw_gateup_shared"]
         return out
+
+    def backward_kernel_launches(self, T: int, weight_grads: bool = True) -> int:
+        """Kernels one backward() launches: permute-backward 1, dh 1, pre-activations 1, SwiGLU-backward 1,
+        dx_perm 1, router 3, combine 1, and per weight gradient 4 (padded offsets, two transposes, the GEMM);
+        the shared expert 4 more (+ 8 with weight gradients)."""
+        if T <= 0:
+            return 0
+        n = 9 + (8 if weight_grads else 0)
+        if self.shared_f:
+            n += 4 + (8 if weight_grads else 0)
+        return n
 
     def kernel_launches(self, T: int) -> int:
         """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the
