@@ -341,7 +341,7 @@ moe_status_t moe_grouped_weight_grad(const moe_bf16_t* a, const moe_bf16_t* b, c
                                      int M, int P, int Q, float* dw, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Bytes of workspace moe_router_backward needs. */
-size_t moe_router_backward_workspace_size(int T, int k);
+size_t moe_router_backward_workspace_size(int T, int d, int E, int k);
 
 /* Router backward, the top-k selection held fixed. From dw (the routing
  * weights' gradient, moe_permute_backward) the gradient of each selected
@@ -353,11 +353,12 @@ size_t moe_router_backward_workspace_size(int T, int k);
  *   dbias[e]        = sum over tokens t selecting e of dl             (fp32; NULL: skipped)
  *   dx[t][c]        = dx_addend[t][c] + sum_j dl_j * w_router[e_j][c] (bf16; dx_addend may be NULL)
  * The sums over tokens run over the grouped rows (perm_src, expert_offsets of
- * moe_permute) in order: deterministic.
+ * moe_permute): per expert in chunks of 256 rows, then the chunks in order
+ * (deterministic).
  *   logits [T][E] fp32 (the forward's), topk_idx / topk_w / dw [T][k],
  *   perm_src / inv_perm [T*k], expert_offsets [E+1], ws of
- *   moe_router_backward_workspace_size(T, k) bytes, 256-byte aligned.
- * Limits as moe_route_topk. */
+ *   moe_router_backward_workspace_size(T, d, E, k) bytes, 256-byte aligned.
+ * Limits as moe_route_topk, and T*k / 256 + E <= 65535. */
 moe_status_t moe_router_backward(const moe_bf16_t* x, const float* w_router, const float* logits,
                                  const int32_t* topk_idx, const float* topk_w, const float* dw,
                                  const int32_t* perm_src, const int32_t* inv_perm, const int32_t* expert_offsets,

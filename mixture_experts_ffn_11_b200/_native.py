@@ -65,7 +65,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_transpose_weights": [vp, ci, ci, ci, vp, vp],
         "moe_grouped_weight_grad_workspace_size": [ci, ci, ci, ci],
         "moe_grouped_weight_grad": [vp, vp, vp, ci, ci, ci, ci, vp, vp, sz, vp],
-        "moe_router_backward_workspace_size": [ci, ci],
+        "moe_router_backward_workspace_size": [ci, ci, ci, ci],
         "moe_router_backward": [vp, vp, vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp, sz, vp],
         "moe_set_gemm_kernel": [ci],
         "moe_test_set_wait": [ctypes.c_ulonglong, ci],
@@ -337,8 +337,8 @@ def grouped_weight_grad(a, b, group_offsets, dw, ws, stream=None):
                                         _stream(stream)), "moe_grouped_weight_grad")
 
 
-def router_backward_workspace_size(T: int, k: int) -> int:
-    return int(_lib.moe_router_backward_workspace_size(T, k))
+def router_backward_workspace_size(T: int, d: int, E: int, k: int) -> int:
+    return int(_lib.moe_router_backward_workspace_size(T, d, E, k))
 
 
 def router_backward(x, w_router, logits, topk_idx, topk_w, dw, perm_src, inv_perm, expert_offsets, mode, dx,

@@ -169,21 +169,23 @@ __global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t* __rest
 
 // dst[c][q] for padded positions q in [0, pad_cap): q in group g (pad_off[g] <= q < pad_off[g+1]) at row
 // q - pad_off[g] < rows_g holds src[offsets[g] + q - pad_off[g]][c]; the rest of the group's padding is zero.
-// Positions at or past pad_off[G] are not written (never read).
+// Positions at or past pad_off[G] are not written (never read). 64 x 64 tiles: each thread loads 16 bytes (8
+// columns) of a source row and stores 16 bytes (8 positions) of a destination row; the tile goes through shared
+// memory as 32-bit words with a padded pitch. cols a multiple of 8.
+constexpr int TP_TILE = 64;
 __global__ void __launch_bounds__(256) transpose_pad_kernel(const __nv_bfloat16* __restrict__ src,
                                                             const int32_t* __restrict__ offsets,
                                                             const int32_t* __restrict__ pad_off, int G, int M,
                                                             int cols, long pad_cap, __nv_bfloat16* __restrict__ dst) {
-    __shared__ __nv_bfloat16 tile[32][33];
-    __shared__ int src_row[32];
+    __shared__ uint16_t tile[TP_TILE][TP_TILE + 2];  // [q][c], pitch 66 halves
+    __shared__ int src_row[TP_TILE];
     grid_dep_wait();
     grid_dep_trigger();
-    const long q0 = (long)blockIdx.y * 32;
-    const int c0 = blockIdx.x * 32;
+    const long q0 = (long)blockIdx.y * TP_TILE;
+    const int c0 = blockIdx.x * TP_TILE;
     const int total = pad_off[G];
     if (q0 >= total) return;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-    if (threadIdx.x < 32) {
+    if (threadIdx.x < TP_TILE) {
         const long q = q0 + threadIdx.x;
         int sr = -1;
         if (q < total) {
@@ -202,17 +204,36 @@ __global__ void __launch_bounds__(256) transpose_pad_kernel(const __nv_bfloat16*
         src_row[threadIdx.x] = sr;
     }
     __syncthreads();
+    // load: 64 rows x 8 pieces of 8 columns, 256 threads -> 2 rounds
 #pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-        const int sr = src_row[ty + i], c = c0 + tx;
-        tile[ty + i][tx] = (sr >= 0 && c < cols) ? src[(long)sr * cols + c] : __float2bfloat16_rn(0.f);
+    for (int it = 0; it < 2; ++it) {
+        const int idx = threadIdx.x + it * 256;
+        const int r = idx >> 3, piece = idx & 7;
+        const int c = c0 + piece * 8;
+        const int sr = src_row[r];
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (sr >= 0 && c < cols) v = *reinterpret_cast<const uint4*>(src + (long)sr * cols + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            tile[r][piece * 8 + 2 * j] = (uint16_t)(w[j] & 0xffffu);
+            tile[r][piece * 8 + 2 * j + 1] = (uint16_t)(w[j] >> 16);
+        }
     }
     __syncthreads();
+    // store: 64 columns (destination rows) x 8 pieces of 8 positions
 #pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-        const int c = c0 + ty + i;
-        const long q = q0 + tx;
-        if (c < cols && q < total) dst[(long)c * pad_cap + q] = tile[tx][ty + i];
+    for (int it = 0; it < 2; ++it) {
+        const int idx = threadIdx.x + it * 256;
+        const int cc = idx >> 3, piece = idx & 7;
+        const int c = c0 + cc;
+        const long q = q0 + piece * 8;
+        if (c >= cols || q >= total) continue;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w[j] = (uint32_t)tile[piece * 8 + 2 * j][cc] | ((uint32_t)tile[piece * 8 + 2 * j + 1][cc] << 16);
+        *reinterpret_cast<uint4*>(dst + (long)c * pad_cap + q) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -265,30 +286,97 @@ __global__ void __launch_bounds__(256) router_dlogits_kernel(const float* __rest
 }
 
 // dW_r[e][c] = sum over the rows r of expert e (in grouped order) of dl_perm[r] * x[perm_src[r]][c], and
-// dbias[e] = sum of the same dl_perm[r]. One block per (expert, 256-column chunk); thread = column.
+// dbias[e] = sum of the same dl_perm[r], in two deterministic passes: each expert's rows are cut into chunks of
+// RB_ROWS (chunk_prefix[e] = chunks before expert e, router_chunk_prefix_kernel); router_chunk_partial_kernel sums
+// one chunk per block and 256-column slice into partial[chunk][c]; router_chunk_reduce_kernel adds an expert's
+// chunk partials in chunk order.
 constexpr int RB_COLS = 256;
-__global__ void __launch_bounds__(RB_COLS) router_weight_grad_kernel(const __nv_bfloat16* __restrict__ x,
-                                                                     const int32_t* __restrict__ perm_src,
-                                                                     const int32_t* __restrict__ offsets,
-                                                                     const float* __restrict__ dl_perm, int T, int d,
-                                                                     int E, int R, float* __restrict__ dw_router,
-                                                                     float* __restrict__ dbias) {
+constexpr int RB_ROWS = 256;
+__global__ void __launch_bounds__(1024) router_chunk_prefix_kernel(const int32_t* __restrict__ offsets, int E, int R,
+                                                                   int32_t* __restrict__ chunk_prefix) {
+    __shared__ int warp_sums[32];
     grid_dep_wait();
     grid_dep_trigger();
-    const int e = blockIdx.y;
+    const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+    int v = 0;
+    if (e < E) {
+        const int a = min(max(offsets[e], 0), R), b = min(max(offsets[e + 1], a), R);
+        v = (b - a + RB_ROWS - 1) / RB_ROWS;
+    }
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_sums[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        int sm = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int u = __shfl_up_sync(0xffffffffu, sm, o);
+            if (lane >= o) sm += u;
+        }
+        warp_sums[lane] = sm;
+    }
+    __syncthreads();
+    const int excl = incl - v + (w > 0 ? warp_sums[w - 1] : 0);
+    if (e < E) chunk_prefix[e] = excl;
+    if (e == E - 1) chunk_prefix[E] = excl + v;
+}
+
+__global__ void __launch_bounds__(RB_COLS) router_chunk_partial_kernel(
+    const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm_src, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ chunk_prefix, const float* __restrict__ dl_perm, int T, int d, int E, int R,
+    float* __restrict__ partial, float* __restrict__ pbias) {
+    grid_dep_wait();
+    grid_dep_trigger();
+    const int chunk = blockIdx.y;
+    if (chunk >= chunk_prefix[E]) return;
+    int lo = 0, hi = E - 1;  // the last expert whose first chunk is <= chunk
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_prefix[mid] <= chunk)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    const int e = lo;
+    const int a = min(max(offsets[e], 0), R), b = min(max(offsets[e + 1], a), R);
+    const int r0 = a + (chunk - chunk_prefix[e]) * RB_ROWS, r1 = min(r0 + RB_ROWS, b);
     const int c = blockIdx.x * RB_COLS + threadIdx.x;
-    int a = offsets[e], b = offsets[e + 1];
-    a = min(max(a, 0), R);
-    b = min(max(b, a), R);
     float acc = 0.f, bsum = 0.f;
-    for (int r = a; r < b; ++r) {
+    for (int r = r0; r < r1; ++r) {
         const float dl = dl_perm[r];
         const int t = perm_src[r];
         bsum += dl;
         if (c < d && t >= 0 && t < T) acc = fmaf(dl, __bfloat162float(x[(long)t * d + c]), acc);
     }
-    if (c < d) dw_router[(long)e * d + c] = acc;
-    if (dbias && blockIdx.x == 0 && threadIdx.x == 0) dbias[e] = bsum;
+    if (c < d) partial[(long)chunk * d + c] = acc;
+    if (blockIdx.x == 0 && threadIdx.x == 0) pbias[chunk] = bsum;
+}
+
+__global__ void __launch_bounds__(RB_COLS) router_chunk_reduce_kernel(const int32_t* __restrict__ chunk_prefix,
+                                                                      const float* __restrict__ partial,
+                                                                      const float* __restrict__ pbias, int d, int E,
+                                                                      float* __restrict__ dw_router,
+                                                                      float* __restrict__ dbias) {
+    grid_dep_wait();
+    grid_dep_trigger();
+    const int e = blockIdx.y;
+    const int c = blockIdx.x * RB_COLS + threadIdx.x;
+    const int k0 = chunk_prefix[e], k1 = chunk_prefix[e + 1];
+    float acc = 0.f;
+    if (c < d) {
+        for (int ch = k0; ch < k1; ++ch) acc += partial[(long)ch * d + c];
+        dw_router[(long)e * d + c] = acc;
+    }
+    if (dbias && blockIdx.x == 0 && threadIdx.x == 0) {
+        float bs = 0.f;
+        for (int ch = k0; ch < k1; ++ch) bs += pbias[ch];
+        dbias[e] = bs;
+    }
 }
 
 // dx_router[t][c] = sum_j dl_tk[t][j] * W_r[e_j][c] (+ addend[t][c]), fp32 sum in slot order, rounded to bf16.

@@ -1001,11 +1001,11 @@ moe_status_t moe_grouped_weight_grad(const moe_bf16_t* a, const moe_bf16_t* b, c
     cudaError_t e = launch_plain(pad_offsets_kernel, dim3(1), dim3(1024), 0, stream, group_offsets, G, M, pad_off);
     if ((st = check_launch("pad_offsets", e)) != MOE_OK) return st;
     if (M > 0) {
-        if (cap / 32 > 65535) return fail(MOE_ERR_INVALID_ARG, "M=%d too large for the weight-gradient transpose", M);
-        e = launch_plain(transpose_pad_kernel, dim3((P + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
+        if (cap / TP_TILE > 65535) return fail(MOE_ERR_INVALID_ARG, "M=%d too large for the weight-gradient transpose", M);
+        e = launch_plain(transpose_pad_kernel, dim3((P + TP_TILE - 1) / TP_TILE, (unsigned)(cap / TP_TILE)), dim3(256), 0, stream,
                        reinterpret_cast<const __nv_bfloat16*>(a), group_offsets, (const int32_t*)pad_off, G, M, P, cap, aT);
         if ((st = check_launch("transpose_pad", e)) != MOE_OK) return st;
-        e = launch_plain(transpose_pad_kernel, dim3((Q + 31) / 32, (unsigned)(cap / 32)), dim3(256), 0, stream,
+        e = launch_plain(transpose_pad_kernel, dim3((Q + TP_TILE - 1) / TP_TILE, (unsigned)(cap / TP_TILE)), dim3(256), 0, stream,
                        reinterpret_cast<const __nv_bfloat16*>(b), group_offsets, (const int32_t*)pad_off, G, M, Q, cap, bT);
         if ((st = check_launch("transpose_pad", e)) != MOE_OK) return st;
     }
@@ -1034,9 +1034,16 @@ moe_status_t moe_grouped_weight_grad(const moe_bf16_t* a, const moe_bf16_t* b, c
     return check_launch("grouped_weight_grad", e);
 }
 
-size_t moe_router_backward_workspace_size(int T, int k) {
-    if (T <= 0 || k <= 0) return 0;
-    return round256((size_t)T * k * 4) * 2;
+namespace {
+// router backward workspace: dl_tk [T*k] | dl_perm [T*k] | chunk_prefix [E+1] | pbias [chunks] | partial [chunks][d]
+long router_chunks_cap(int T, int E, int k) { return ((long)T * k + RB_ROWS - 1) / RB_ROWS + E; }
+}  // namespace
+
+size_t moe_router_backward_workspace_size(int T, int d, int E, int k) {
+    if (T <= 0 || k <= 0 || E <= 0 || d <= 0) return 0;
+    const long chunks = router_chunks_cap(T, E, k);
+    return round256((size_t)T * k * 4) * 2 + round256((size_t)(E + 1) * 4) + round256((size_t)chunks * 4) +
+           round256((size_t)chunks * d * 4);
 }
 
 moe_status_t moe_router_backward(const moe_bf16_t* x, const float* w_router, const float* logits,
@@ -1063,20 +1070,35 @@ moe_status_t moe_router_backward(const moe_bf16_t* x, const float* w_router, con
         return fail(MOE_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(x) || !aligned16(w_router) || !aligned16(dx) || (dx_addend && !aligned16(dx_addend)))
         return fail(MOE_ERR_INVALID_ARG, "x, w_router, dx and dx_addend must be 16-byte aligned");
-    const size_t need = moe_router_backward_workspace_size(T, k);
+    const size_t need = moe_router_backward_workspace_size(T, d, E, k);
     if (!ws || ws_bytes < need)
         return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : (size_t)0);
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return fail(MOE_ERR_WORKSPACE, "workspace not 256-byte aligned");
-    float* dl_tk = reinterpret_cast<float*>(ws);
-    float* dl_perm = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + round256((size_t)T * k * 4));
+    const long chunks = router_chunks_cap(T, E, k);
+    if (chunks > 65535) return fail(MOE_ERR_INVALID_ARG, "T*k=%ld too large for the router backward", (long)T * k);
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    float* dl_tk = reinterpret_cast<float*>(base);
+    base += round256((size_t)T * k * 4);
+    float* dl_perm = reinterpret_cast<float*>(base);
+    base += round256((size_t)T * k * 4);
+    int32_t* chunk_prefix = reinterpret_cast<int32_t*>(base);
+    base += round256((size_t)(E + 1) * 4);
+    float* pbias = reinterpret_cast<float*>(base);
+    base += round256((size_t)chunks * 4);
+    float* partial = reinterpret_cast<float*>(base);
     const int R = T * k;
     cudaError_t e = launch_plain(router_dlogits_kernel, dim3(grid_cap((T + 255) / 256, di.sms, 4)), dim3(256), 0,
                                stream, logits, topk_idx, topk_w, dw, inv_perm, T, E, k, (int)mode, dl_tk, dl_perm);
     if ((st = check_launch("router_dlogits", e)) != MOE_OK) return st;
-    e = launch_plain(router_weight_grad_kernel, dim3((d + RB_COLS - 1) / RB_COLS, E), dim3(RB_COLS), 0, stream,
-                   reinterpret_cast<const __nv_bfloat16*>(x), perm_src, expert_offsets, (const float*)dl_perm, T, d, E,
-                   R, dw_router, dbias);
-    if ((st = check_launch("router_weight_grad", e)) != MOE_OK) return st;
+    e = launch_plain(router_chunk_prefix_kernel, dim3(1), dim3(1024), 0, stream, expert_offsets, E, R, chunk_prefix);
+    if ((st = check_launch("router_chunk_prefix", e)) != MOE_OK) return st;
+    e = launch_plain(router_chunk_partial_kernel, dim3((d + RB_COLS - 1) / RB_COLS, (unsigned)chunks), dim3(RB_COLS), 0,
+                     stream, reinterpret_cast<const __nv_bfloat16*>(x), perm_src, expert_offsets,
+                     (const int32_t*)chunk_prefix, (const float*)dl_perm, T, d, E, R, partial, pbias);
+    if ((st = check_launch("router_chunk_partial", e)) != MOE_OK) return st;
+    e = launch_plain(router_chunk_reduce_kernel, dim3((d + RB_COLS - 1) / RB_COLS, E), dim3(RB_COLS), 0, stream,
+                     (const int32_t*)chunk_prefix, (const float*)partial, (const float*)pbias, d, E, dw_router, dbias);
+    if ((st = check_launch("router_chunk_reduce", e)) != MOE_OK) return st;
     e = launch_plain(router_input_grad_kernel, dim3(grid_cap((T + 7) / 8, di.sms, 16)), dim3(256), 0, stream, topk_idx,
                    (const float*)dl_tk, w_router, reinterpret_cast<const __nv_bfloat16*>(dx_addend), T, d, E, k,
                    reinterpret_cast<__nv_bfloat16*>(dx));

@@ -226,7 +226,8 @@ class MoEFFN:
              "dgu": torch.empty(R, 2 * f, dtype=bf, device=dev), "dx_perm": torch.empty(R, d, dtype=bf, device=dev),
              "dx_router": torch.empty(T, d, dtype=bf, device=dev), "dx": torch.empty(T, d, dtype=bf, device=dev),
              "ones": torch.ones(T, k, dtype=f32, device=dev),
-             "router_ws": torch.empty(max(N.router_backward_workspace_size(T, k), 256), dtype=torch.uint8, device=dev),
+             "router_ws": torch.empty(max(N.router_backward_workspace_size(T, d, E, k), 256), dtype=torch.uint8,
+                                      device=dev),
              "dw_router": torch.empty(E, d, dtype=f32, device=dev),
              "dbias": torch.empty(E, dtype=f32, device=dev) if self.bias is not None else None,
              "dw_down": torch.empty(E, d, f, dtype=f32, device=dev),
@@ -323,11 +324,11 @@ class MoEFFN:
 
     def backward_kernel_launches(self, T: int, weight_grads: bool = True) -> int:
         """Kernels one backward() launches: permute-backward 1, dh 1, pre-activations 1, SwiGLU-backward 1,
-        dx_perm 1, router 3, combine 1, and per weight gradient 4 (padded offsets, two transposes, the GEMM);
+        dx_perm 1, router 5, combine 1, and per weight gradient 4 (padded offsets, two transposes, the GEMM);
         the shared expert 4 more (+ 8 with weight gradients)."""
         if T <= 0:
             return 0
-        n = 9 + (8 if weight_grads else 0)
+        n = 11 + (8 if weight_grads else 0)
         if self.shared_f:
             n += 4 + (8 if weight_grads else 0)
         return n
