@@ -98,6 +98,8 @@ def parse_args(argv=None):
                     help="time one grouped GEMM alone (kernel-only mode, for profilers)")
     ap.add_argument("--gemm", choices=["auto", "single", "pair", "wide", "swap"], default="auto",
                     help="force a grouped-GEMM kernel family")
+    ap.add_argument("--dispatch", choices=["fused", "separate"], default="separate",
+                    help="prefill: row gather and combine as their own kernels (default), or inside the grouped GEMMs")
     ap.add_argument("--shape", default="", help="comma-separated workload overrides, e.g. T=1024,E=64 (profiling)")
     ap.add_argument("--backward", action="store_true",
                     help="time the training step: forward + backward with weight gradients (not the headline)")
@@ -376,8 +378,10 @@ def setup_layer(args, dev):
     wl = bench_workload(args)
     synth.build_cuda()
     inp = synth.device_inputs(wl, dev)
+    # a forced kernel family applies to the grouped-copy path only
+    fuse = args.dispatch == "fused" and args.gemm in ("auto", "swap")
     layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
-                   inp["w_gateup_shared"], inp["w_down_shared"], weights=wl.weights)
+                   inp["w_gateup_shared"], inp["w_down_shared"], weights=wl.weights, fused=fuse)
     if wl.weights != "bf16":  # the layer keeps only its encoded weights
         for key in ("w_gateup", "w_down", "w_gateup_shared", "w_down_shared"):
             inp[key] = None
@@ -400,7 +404,10 @@ def run_kernel(args):
     layer.forward(inp["x"])
     b = layer.buf
     s = torch.cuda.current_stream(dev)
-    if args.kernel == "gateup":
+    if args.kernel == "gateup" and layer._fused(wl.T):
+        launch = lambda: N.grouped_gemm_gateup_gather(inp["x"], b["perm_src"], layer.w_gateup, b["offsets"],  # noqa
+                                                      b["h"], None, s)
+    elif args.kernel == "gateup":
         launch = lambda: layer._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)  # noqa: E731
     else:
         launch = lambda: layer._down(b["h"], "routed", b["offsets"], b["y_perm"], s)  # noqa: E731
@@ -595,6 +602,8 @@ def run_ours(args):
             "parallelism": "replicas" if world > 1 else "single GPU"}
     if args.gemm != "auto":
         line["gemm_family"] = args.gemm
+    line["config"]["dispatch"] = ("gather in gate|up GEMM, combine in down GEMM" if layer._fused(wl.T)
+                                  else "moe_permute gather, moe_unpermute_combine")
     if args.backward:
         # the training step: forward + backward (top-k selection held fixed), weight gradients included
         R, d, f, fs = wl.R, wl.d, wl.f, wl.shared_f

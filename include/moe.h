@@ -14,8 +14,12 @@
  *   moe_permute             expert histogram, exclusive scan, stable scatter,
  *                           gather of x rows into expert-contiguous order
  *   moe_grouped_gemm_gateup h = silu(x_perm Wg^T) * (x_perm Wu^T), per expert
+ *                           (moe_grouped_gemm_gateup_gather: the same with
+ *                           the gather folded into the GEMM's operand load)
  *   moe_grouped_gemm_down   y_perm = h Wd^T, per expert
  *   moe_unpermute_combine   y[t] = sum_j w[t,j] * y_perm[row of (t,j)] (+ shared[t])
+ *                           (moe_grouped_gemm_down_combine: down and combine
+ *                           in one call, the combine in the GEMM's epilogue)
  *
  * With MXFP4 expert weights (encoded once by moe_mxfp4_quantize) the two
  * grouped GEMMs are moe_grouped_gemm_gateup_mxfp4 / moe_grouped_gemm_down_mxfp4.
@@ -205,12 +209,76 @@ moe_status_t moe_permute_static_ws(const moe_bf16_t* x, const int32_t* topk_idx,
 moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_gateup, const int32_t* group_offsets,
                                      int G, int M, int d, int f, moe_bf16_t* h, cudaStream_t stream);
 
+/* Bytes of workspace moe_grouped_gemm_gateup_gather needs: 0 when the groups
+ * average 128 rows or more (M >= 128*G), else M*d*2 rounded up to 256. */
+size_t moe_grouped_gemm_gateup_gather_workspace_size(int G, int M, int d);
+
+/* moe_grouped_gemm_gateup with the dispatch folded in (section "Expert
+ * Backend": tokens are dispatched to their experts' weights, here without a
+ * grouped copy of x): row r of the GEMM's A operand is x[row_src[r]], e.g.
+ * row_src = perm_src of moe_permute called with x = x_perm = NULL. Same sums
+ * and the same h bits as moe_permute's gather followed by
+ * moe_grouped_gemm_gateup.
+ *   x        [T][d] bf16, 16-byte aligned
+ *   row_src  [M] int32, DEVICE memory, entries in [0, T); an entry outside it
+ *            is flagged (MOE_DEVERR_ROW_RANGE) and the h row it feeds is
+ *            unspecified (no out-of-range read is made)
+ *   ws       workspace of moe_grouped_gemm_gateup_gather_workspace_size(G,
+ *            M, d) bytes, 16-byte aligned (may be NULL when that is 0):
+ *            with fewer than 128 rows per group on average the rows are
+ *            gathered there first and the GEMM runs on the copy.
+ * Other arguments and limits as moe_grouped_gemm_gateup. The kernel family
+ * hook (moe_set_gemm_kernel) applies only to the workspace path. */
+moe_status_t moe_grouped_gemm_gateup_gather(const moe_bf16_t* x, const int32_t* row_src, int T,
+                                            const moe_bf16_t* w_gateup, const int32_t* group_offsets, int G, int M,
+                                            int d, int f, moe_bf16_t* h, void* ws, size_t ws_bytes,
+                                            cudaStream_t stream);
+
+/* out[r] = x[row_src[r]] for r < R: the gather of moe_permute on its own.
+ *   x [T][d], out [R][d] bf16, 16-byte aligned; row_src [R] int32 in [0, T)
+ *   (an entry outside it is flagged, MOE_DEVERR_ROW_RANGE, and its row
+ *   zeroed). d a positive multiple of 8. */
+moe_status_t moe_gather_rows(const moe_bf16_t* x, const int32_t* row_src, int T, int d, int R, moe_bf16_t* out,
+                             cudaStream_t stream);
+
 /* Grouped down projection: y[r][c] = sum_n h[r][n] * w[g][c][n] (fp32
  * accumulation, rounded to bf16) for r in group g. w is the packed down_proj
  * tensor [G][d][f] (experts' w2 stacked on dim 0, same section).
  *   h [M][f] bf16, y [M][d] bf16, group_offsets as above. */
 moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down, const int32_t* group_offsets,
                                    int G, int M, int d, int f, moe_bf16_t* y, cudaStream_t stream);
+
+/* Bytes of workspace moe_grouped_gemm_down_combine needs: T * ceil(d/32) * 4
+ * rounded up to 256 (arrival counters). */
+size_t moe_grouped_gemm_down_combine_workspace_size(int T, int d);
+
+/* moe_grouped_gemm_down followed by moe_unpermute_combine in one call, with
+ * the collect step (section "Expert Backend": apply the routing weights, then
+ * collect and reorder) folded into the GEMM when the groups average 128 rows
+ * or more (M >= 128*G): as each tile's y_perm rows are stored, one arrival
+ * per row is counted on a counter of (token, 32-column block), and the tile
+ * that brings a token's k-th arrival for a block sums the token's k rows of
+ * that block in slot order. Writes y_perm (as moe_grouped_gemm_down) and y (as
+ * moe_unpermute_combine), with the same bits as those two calls.
+ *   h, w_down, group_offsets, G, M, d, f   as moe_grouped_gemm_down; M = T*k
+ *   perm_src, inv_perm  [T*k] int32 of moe_permute (one the inverse of the
+ *                       other: a row of group g holds assignment a of token
+ *                       perm_src[row] with inv_perm[a] = row)
+ *   topk_w [T][k] fp32, shared [T][d] bf16 or NULL, y_perm [M][d], y [T][d]
+ *   ws, ws_bytes        workspace of
+ *                       moe_grouped_gemm_down_combine_workspace_size(T, d)
+ *                       bytes, 16-byte aligned; need not be initialised
+ *                       (the call clears what it uses).
+ * Entries of perm_src or inv_perm out of range are flagged
+ * (MOE_DEVERR_ROW_RANGE); a pair that is not mutually inverse leaves rows of
+ * y unspecified. The kernel family hook (moe_set_gemm_kernel) applies only
+ * when the groups are smaller (then the two calls run one after the other).
+ * Limits: those of both calls. */
+moe_status_t moe_grouped_gemm_down_combine(const moe_bf16_t* h, const moe_bf16_t* w_down,
+                                           const int32_t* group_offsets, int G, int M, int d, int f,
+                                           const int32_t* perm_src, const int32_t* inv_perm, const float* topk_w,
+                                           const moe_bf16_t* shared, int T, int k, moe_bf16_t* y_perm, moe_bf16_t* y,
+                                           void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* ---- MXFP4 expert weights ----
  * The blog post's section "From Dense to Sparse: What Are MoEs?" estimates

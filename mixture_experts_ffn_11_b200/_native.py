@@ -24,7 +24,9 @@ ROUTE_MODES = {"topk_softmax": 0, "softmax_topk_renorm": 1, "sigmoid_topk_norm":
 # every entry point of include/moe.h
 EXPORTS = ("moe_route_topk", "moe_router_split_weights", "moe_route_topk_split", "moe_topk_from_logits", "moe_permute_workspace_size", "moe_permute",
            "moe_permute_static_ws",
-           "moe_grouped_gemm_gateup", "moe_grouped_gemm_down", "moe_mxfp4_quantize", "moe_grouped_gemm_gateup_mxfp4",
+           "moe_grouped_gemm_gateup", "moe_grouped_gemm_gateup_gather_workspace_size",
+           "moe_grouped_gemm_gateup_gather", "moe_gather_rows", "moe_grouped_gemm_down",
+           "moe_grouped_gemm_down_combine_workspace_size", "moe_grouped_gemm_down_combine", "moe_mxfp4_quantize", "moe_grouped_gemm_gateup_mxfp4",
            "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_grouped_gemm_gateup_preact",
            "moe_swiglu_backward", "moe_permute_backward", "moe_transpose_weights",
            "moe_grouped_weight_grad_workspace_size", "moe_grouped_weight_grad", "moe_router_backward_workspace_size",
@@ -54,7 +56,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_permute": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp, sz, vp],
         "moe_permute_static_ws": [vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, vp, vp],
         "moe_grouped_gemm_gateup": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_grouped_gemm_gateup_gather_workspace_size": [ci, ci, ci],
+        "moe_grouped_gemm_gateup_gather": [vp, vp, ci, vp, vp, ci, ci, ci, ci, vp, vp, sz, vp],
+        "moe_gather_rows": [vp, vp, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_down": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_grouped_gemm_down_combine_workspace_size": [ci, ci],
+        "moe_grouped_gemm_down_combine": [vp, vp, vp, ci, ci, ci, ci, vp, vp, vp, vp, ci, ci, vp, vp, vp, sz, vp],
         "moe_mxfp4_quantize": [vp, ci, ci, ci, vp, vp, vp],
         "moe_grouped_gemm_gateup_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_down_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
@@ -78,6 +85,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn.restype = ci
     lib.moe_permute_workspace_size.restype = sz
     lib.moe_grouped_weight_grad_workspace_size.restype = sz
+    lib.moe_grouped_gemm_gateup_gather_workspace_size.restype = sz
+    lib.moe_grouped_gemm_down_combine_workspace_size.restype = sz
     lib.moe_router_backward_workspace_size.restype = sz
     lib.moe_last_error_string.restype = ctypes.c_char_p
     return lib
@@ -217,6 +226,38 @@ def grouped_gemm_gateup(a, w_gateup, group_offsets, h, stream=None):
                                         _stream(stream)), "moe_grouped_gemm_gateup")
 
 
+def grouped_gemm_gateup_gather_workspace_size(G: int, M: int, d: int) -> int:
+    return int(_lib.moe_grouped_gemm_gateup_gather_workspace_size(G, M, d))
+
+
+def grouped_gemm_gateup_gather(x, row_src, w_gateup, group_offsets, h, ws=None, stream=None):
+    """h for A rows x[row_src[r]] (moe_grouped_gemm_gateup_gather); ws: a uint8 tensor of at least
+    grouped_gemm_gateup_gather_workspace_size(G, M, d) bytes, or None when that is 0."""
+    T, d = x.shape
+    M = row_src.shape[0]
+    G, two_f, d2 = w_gateup.shape
+    f = two_f // 2
+    _need(x, torch.bfloat16, (T, d), "x")
+    _need(row_src, torch.int32, (M,), "row_src")
+    _need(w_gateup, torch.bfloat16, (G, 2 * f, d), "w_gateup")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(h, torch.bfloat16, (M, f), "h")
+    ws_bytes = ws.numel() * ws.element_size() if ws is not None else 0
+    _check(_lib.moe_grouped_gemm_gateup_gather(_p(x), _p(row_src), T, _p(w_gateup), _p(group_offsets), G, M, d, f,
+                                               _p(h), _p(ws), ws_bytes, _stream(stream)),
+           "moe_grouped_gemm_gateup_gather")
+
+
+def gather_rows(x, row_src, out, stream=None):
+    """out[r] = x[row_src[r]] (moe_gather_rows)."""
+    T, d = x.shape
+    R = row_src.shape[0]
+    _need(x, torch.bfloat16, (T, d), "x")
+    _need(row_src, torch.int32, (R,), "row_src")
+    _need(out, torch.bfloat16, (R, d), "out")
+    _check(_lib.moe_gather_rows(_p(x), _p(row_src), T, d, R, _p(out), _stream(stream)), "moe_gather_rows")
+
+
 def grouped_gemm_down(h, w_down, group_offsets, y, stream=None):
     M, f = h.shape
     G, d, f2 = w_down.shape
@@ -226,6 +267,33 @@ def grouped_gemm_down(h, w_down, group_offsets, y, stream=None):
     _need(y, torch.bfloat16, (M, d), "y")
     _check(_lib.moe_grouped_gemm_down(_p(h), _p(w_down), _p(group_offsets), G, M, d, f, _p(y), _stream(stream)),
            "moe_grouped_gemm_down")
+
+
+def grouped_gemm_down_combine_workspace_size(T: int, d: int) -> int:
+    return int(_lib.moe_grouped_gemm_down_combine_workspace_size(T, d))
+
+
+def grouped_gemm_down_combine(h, w_down, group_offsets, perm_src, inv_perm, topk_w, shared, y_perm, y, ws,
+                              stream=None):
+    """y_perm = down(h) and y = combine(y_perm) in one call (moe_grouped_gemm_down_combine); ws: a uint8 tensor of
+    at least grouped_gemm_down_combine_workspace_size(T, d) bytes."""
+    M, f = h.shape
+    G, d, f2 = w_down.shape
+    T, k = topk_w.shape
+    _need(h, torch.bfloat16, (M, f), "h")
+    _need(w_down, torch.bfloat16, (G, d, f), "w_down")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(perm_src, torch.int32, (M,), "perm_src")
+    _need(inv_perm, torch.int32, (M,), "inv_perm")
+    _need(topk_w, torch.float32, (T, k), "topk_w")
+    if shared is not None:
+        _need(shared, torch.bfloat16, (T, d), "shared")
+    _need(y_perm, torch.bfloat16, (M, d), "y_perm")
+    _need(y, torch.bfloat16, (T, d), "y")
+    _need(ws, torch.uint8, None, "ws")
+    _check(_lib.moe_grouped_gemm_down_combine(_p(h), _p(w_down), _p(group_offsets), G, M, d, f, _p(perm_src),
+                                              _p(inv_perm), _p(topk_w), _p(shared), T, k, _p(y_perm), _p(y), _p(ws),
+                                              ws.numel(), _stream(stream)), "moe_grouped_gemm_down_combine")
 
 
 def mxfp4_quantize(w, q, s, stream=None):

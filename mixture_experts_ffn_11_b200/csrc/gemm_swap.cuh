@@ -110,6 +110,112 @@ __device__ __forceinline__ void flush_staged_block(uint8_t* stage, int lane, con
     __syncwarp();
 }
 
+// The weighted combine fused into the down GEMM (COMBINE): "apply the routing weights and then collect and
+// reorder the results" (blog post "Mixture of Experts (MoEs) in Transformers", section "Expert Backend"),
+//   y[t][c] = sum_{j<k} w[t][j] * y_perm[inv_perm[t*k+j]][c] (+ shared[t][c]),  fp32 in slot order, bf16 out,
+// the arithmetic of the stand-alone combine kernel. The k rows of a token come from k groups, computed by
+// different tiles in any order, so no tile can sum them as it goes without fixing an order by waiting. Instead
+// each epilogue warp, once its y_perm rows of a tile are stored, counts one arrival per row on a counter of
+// (token, 32-column block); the warp whose arrival is the k-th reads the k rows back (from L2, just written)
+// and sums them in slot order. The sum is the same whoever finishes last: deterministic, no waiting.
+struct CombineArgs {
+    const int32_t* perm_src = nullptr;      // [M] grouped row -> token
+    const int32_t* inv_perm = nullptr;      // [T*k] assignment -> grouped row
+    const float* topk_w = nullptr;          // [T*k]
+    const __nv_bfloat16* shared = nullptr;  // [T][n_out] or null
+    __nv_bfloat16* y = nullptr;             // [T][n_out]
+    int* counters = nullptr;                // [T][ceil(n_out / 32)], zero when the kernel starts
+    int T = 0, k = 0;
+};
+
+// Sum one token's k slot rows over the 32 columns [c0, c0 + 32) (those below n_out) into y[t].
+__device__ __noinline__ void combine_token_columns(const CombineArgs& ca, const __nv_bfloat16* y_perm, int M,
+                                                   int n_out, int t, int c0) {
+    const int nunit = min(4, (n_out - c0) >> 3);  // 16-byte units (8 columns) inside the output
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll 4
+    for (int j = 0; j < ca.k; ++j) {
+        const int row = __ldg(ca.inv_perm + (size_t)t * ca.k + j);
+        const float w = __ldg(ca.topk_w + (size_t)t * ca.k + j);
+        if (row < 0 || row >= M) {
+            flag_error(MOE_DEVERR_ROW_RANGE);
+            continue;
+        }
+        // written by other CTAs in this kernel: read through L2 (ld.global.cg), after the acquire fence
+        const uint4* src = reinterpret_cast<const uint4*>(y_perm + (size_t)row * n_out + c0);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (u < nunit) {
+                const uint4 q = __ldcg(src + u);
+                const uint32_t uq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = unpack_bf16x2(uq[i]);
+                    acc[8 * u + 2 * i] = fmaf(w, f.x, acc[8 * u + 2 * i]);
+                    acc[8 * u + 2 * i + 1] = fmaf(w, f.y, acc[8 * u + 2 * i + 1]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (u >= nunit) continue;
+        if (ca.shared) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(ca.shared + (size_t)t * n_out + c0) + u);
+            const uint32_t uq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float2 f = unpack_bf16x2(uq[i]);
+                acc[8 * u + 2 * i] += f.x;
+                acc[8 * u + 2 * i + 1] += f.y;
+            }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[8 * u + 0], acc[8 * u + 1]);
+        o.y = pack_bf16x2(acc[8 * u + 2], acc[8 * u + 3]);
+        o.z = pack_bf16x2(acc[8 * u + 4], acc[8 * u + 5]);
+        o.w = pack_bf16x2(acc[8 * u + 6], acc[8 * u + 7]);
+        reinterpret_cast<uint4*>(ca.y + (size_t)t * n_out + c0)[u] = o;
+    }
+}
+
+// After a warp has stored its 32 columns [c0, c0 + 32) of the tile's rows r0 .. r0 + rows - 1 of y_perm: publish
+// them, count one arrival per row, and finish the tokens whose last slot this was.
+__device__ __forceinline__ void combine_after_tile(const CombineArgs& ca, const __nv_bfloat16* y_perm, int M,
+                                                   int n_out, int r0, int rows, int c0, int lane) {
+    if (lane == 0) {
+        bulk_wait_all();             // this warp's TMA stores of the tile have landed
+        fence_proxy_async_global();  // ... and are ordered before the generic release below
+    }
+    __syncwarp();
+    __threadfence();  // release: the rows (and the masked edge stores) before the arrivals
+    const int ncb = (n_out + 31) >> 5;
+    const int cb = c0 >> 5;
+    int tok[GS_MAX_N / 32], old[GS_MAX_N / 32];
+#pragma unroll
+    for (int i = 0; i < GS_MAX_N / 32; ++i) {
+        const int rr = lane + 32 * i;
+        int t = -1;
+        if (rr < rows) {
+            t = __ldg(ca.perm_src + r0 + rr);
+            if (t < 0 || t >= ca.T) {
+                flag_error(MOE_DEVERR_ROW_RANGE);
+                t = -1;
+            }
+        }
+        tok[i] = t;
+    }
+#pragma unroll
+    for (int i = 0; i < GS_MAX_N / 32; ++i)
+        old[i] = tok[i] >= 0 ? atomicAdd(ca.counters + (size_t)tok[i] * ncb + cb, 1) : -1;
+    __threadfence();  // acquire: the other slots' rows, published before their arrivals
+#pragma unroll 1
+    for (int i = 0; i < GS_MAX_N / 32; ++i)
+        if (tok[i] >= 0 && old[i] == ca.k - 1) combine_token_columns(ca, y_perm, M, n_out, tok[i], c0);
+}
+
 // tmX[i]: the token rows [M][K] with boxes of 128 >> i rows (i = 0..4).
 struct SwapMaps {
     CUtensorMap x[5];
@@ -126,10 +232,17 @@ __device__ __forceinline__ int swap_box_index(int half) {
 // tmO: the output [M][n_out], 32 x 32 boxes, 64-byte swizzle.
 // RAW (gate|up only): no SwiGLU; every warp stores its own lanes, gate rows to columns [0, f) and up rows to
 // columns [f, 2f) of an [M][2f] output (the pre-activations a backward pass needs).
-template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false>
+// GATHER: token row r of the tile is row args.row_src[r] of x [src_rows][K] (the dispatch of the blog post's
+// expert backend folded into the operand load): tmX.x[0] views x with a one-row box, and each producer lane brings
+// four of the CTA's rows per K block with one TMA gather4 into the places a tile box would fill, so the MMA and
+// the epilogue are unchanged and no permuted copy of x is written.
+// COMBINE (down only): after each tile, the weighted combine of the tokens completed by it (CombineArgs).
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false, bool GATHER = false, bool COMBINE = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ SwapMaps tmX,
-                             const __grid_constant__ CUtensorMap tmO, const GemmArgs args, int weights_streamed_once) {
+                             const __grid_constant__ CUtensorMap tmO, const GemmArgs args, int weights_streamed_once,
+                             const __grid_constant__ CombineArgs cargs) {
+    static_assert(!COMBINE || !GATEUP, "the combine follows the down projection");
     using S = GemmSwapShape<GATEUP, SUB, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -257,11 +370,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
             const int xrow0 = r0 + (int)rank * half;
             const int wrow = GATEUP ? wb * 128 + 64 * (int)rank : wb * 256 + 128 * (int)rank;
             const uint32_t sub_tx = (uint32_t)(S::W_BYTES + (128 >> bi) * GG_BK * 2);
+            // GATHER: this lane's four token rows (4 * lane .. 4 * lane + 3 of the CTA's share) as rows of x
+            int src0 = 0, src1 = 0, src2 = 0, src3 = 0;
+            if constexpr (GATHER) {
+                int v[4] = {0, 0, 0, 0};
+                if (4 * lane < half) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = xrow0 + 4 * lane + i;  // rows past the tile (padding) are never stored
+                        int src = r < args.M ? __ldg(args.row_src + r) : 0;
+                        if (src < 0 || src >= args.src_rows) {
+                            flag_error(MOE_DEVERR_ROW_RANGE);
+                            src = 0;
+                        }
+                        v[i] = src;
+                    }
+                }
+                src0 = v[0];
+                src1 = v[1];
+                src2 = v[2];
+                src3 = v[3];
+            }
             for (int kb = 0; kb < KB; ++kb) {
                 if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
-                if (lane == 0) {
+                if constexpr (GATHER) {
+                    const int nsub = min(SUB, KBS - kb * SUB);
+                    uint8_t* sa = stages + stage * S::STAGE_BYTES;
+                    const uint32_t bar = mapa_shared(smem_u32(&full_bar[stage]), 0);
+                    if (lane == 0) {
+                        const uint32_t w_tx = (uint32_t)((BIGBOX ? SUB : nsub) * S::W_BYTES);
+                        if (leader)
+                            mbar_arrive_expect_tx(&full_bar[stage], 2u * (w_tx + (uint32_t)(nsub * half * GG_BK * 2)));
+                        if constexpr (BIGBOX) {
+                            if constexpr (GATEUP)
+                                tma_load_5d_pair(sa, &tmW, bar, 0, wrow, 0, kb * SUB, g, pol_w);
+                            else
+                                tma_load_4d_pair(sa, &tmW, bar, 0, wrow, kb * SUB, g, pol_w);
+                        } else {
+                            for (int sb = 0; sb < nsub; ++sb) {
+                                const int kc = (kb * SUB + sb) * GG_BK;
+                                if constexpr (GATEUP)
+                                    tma_load_4d_pair(sa + sb * S::W_BYTES, &tmW, bar, kc, wrow, 0, g, pol_w);
+                                else
+                                    tma_load_3d_pair(sa + sb * S::W_BYTES, &tmW, bar, kc, wrow, g, pol_w);
+                            }
+                        }
+                    }
+                    if (4 * lane < half) {
+                        for (int sb = 0; sb < nsub; ++sb)
+                            tma_gather4_pair(sa + S::X_OFF + sb * (128 >> bi) * GG_BK * 2 + lane * 4 * GG_BK * 2,
+                                             &tmX.x[0], bar, (kb * SUB + sb) * GG_BK, src0, src1, src2, src3, pol_x);
+                    }
+                    __syncwarp();
+                } else if (lane == 0) {
                     uint8_t* sa = stages + stage * S::STAGE_BYTES;
                     const uint32_t bar = mapa_shared(smem_u32(&full_bar[stage]), 0);
                     if constexpr (BIGBOX) {  // one box per operand: SUB K blocks (past the end: zeros)
@@ -434,6 +597,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
             if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
+            if constexpr (COMBINE) {
+                if (col0 < args.n_out) combine_after_tile(cargs, args.out, args.M, args.n_out, r0, rows, col0, lane);
+            }
         }
         if (ferry && ok && blocks > 0) {  // the last hand-off has been read before the buffer goes away
             mbar_wait_bounded(&xempty_bar[p], (blocks & 1u) ^ 1u, abort_flag);

@@ -21,6 +21,7 @@
 #include "gemm_wide.cuh"
 #include "gemm_swap.cuh"
 #include "gemm_fp4.cuh"
+#include "gemm_fp4_mma.cuh"
 #include "gemm_wgrad.cuh"
 #include "backward.cuh"
 #include "combine.cuh"
@@ -135,7 +136,21 @@ cudaError_t set_gemm_attributes() {
         e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, false, true>, a, SwapGU::SMEM_BYTES);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess)  // row gather in the operand load
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, false, false, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true, false, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess)  // combine in the epilogue
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, false, false, false, true>, a,
+                                 SwapDN::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, true, false, false, true>, a,
+                                 SwapDN::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_wgrad_kernel, a, GemmWgradShape::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_fp4_warp_kernel<true>, a, GemmFp4WarpShape<true>::MAX_SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_fp4_warp_kernel<false>, a, GemmFp4WarpShape<false>::MAX_SMEM);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<16, true>, a, GemmFp4Shape<16, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<32, true>, a, GemmFp4Shape<32, true>::SMEM_BYTES);
     if (e == cudaSuccess) e = cudaFuncSetAttribute(grouped_gemm_fp4_kernel<64, true>, a, GemmFp4Shape<64, true>::SMEM_BYTES);
@@ -246,6 +261,8 @@ struct GemmProblem {
     const int32_t* offsets;
     int G, M, K, n_out, f;
     void* out;
+    const int32_t* row_src = nullptr;  // gathering gate|up: A row r is row row_src[r] of a [src_rows][K] tensor
+    int src_rows = 0;
 };
 
 // Tensor maps: A [M][K] in 128-row x 64 boxes; B slabs [G][rows][K] (rows = 2f for gate|up, n_out for
@@ -281,6 +298,8 @@ GemmArgs gemm_args(const GemmProblem& p, int out_cols) {
     args.f = p.f;
     args.n_tiles = (p.n_out + out_cols - 1) / out_cols;
     args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    args.row_src = p.row_src;
+    args.src_rows = p.src_rows;
     return args;
 }
 
@@ -330,8 +349,8 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)", e);
 }
 
-template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false>
-moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false, bool GATHER = false, bool COMBINE = false>
+moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream, const CombineArgs& ca = CombineArgs()) {
     using S = GemmSwapShape<GATEUP, SUB, STAGES>;
     CUtensorMap tw, to;
     SwapMaps tx;
@@ -375,6 +394,13 @@ moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
             st = make_tmap(&tx.x[i], p.a, 2, xdims, xstr, xbox);
         }
     }
+    if (GATHER && st == MOE_OK) {  // the source rows [src_rows][K], one row per box (TMA gather4)
+        const cuuint64_t gdims[2] = {K, (cuuint64_t)p.src_rows};
+        const cuuint64_t gstr[1] = {K * 2};
+        const cuuint32_t gbox[2] = {GG_BK, 1};
+        st = make_tmap(&tx.x[0], p.a, 2, gdims, gstr, gbox);
+        for (int i = 1; i < 5; ++i) tx.x[i] = tx.x[0];
+    }
     if (st == MOE_OK) {
         if (RAW) {  // [M][2f] pre-activations: gate in columns [0, f), up in [f, 2f)
             GemmProblem q = p;
@@ -389,10 +415,13 @@ moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream) {
     const long upper = ((long)p.M / GS_MAX_N + p.G) * (long)args.n_tiles;  // >= the real tile count
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GS_MAX_N ? 1 : 0;
-    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX, RAW>, dim3(2 * clusters),
-                                     dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, args, streamed_once);
+    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX, RAW, GATHER, COMBINE>,
+                                     dim3(2 * clusters), dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, args,
+                                     streamed_once, ca);
     return check_launch(RAW ? "grouped_gemm_gateup_preact (swap pair)"
-                            : (GATEUP ? "grouped_gemm_gateup (swap pair)" : "grouped_gemm_down (swap pair)"), e);
+                            : (GATEUP ? "grouped_gemm_gateup (swap pair)"
+                                      : (COMBINE ? "grouped_gemm_down_combine (swap pair)"
+                                                 : "grouped_gemm_down (swap pair)")), e);
 }
 
 template <bool GATEUP>
@@ -487,10 +516,60 @@ moe_status_t launch_fp4(const Fp4Problem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup_mxfp4" : "grouped_gemm_down_mxfp4", e);
 }
 
-// Token tile: the smallest of 16, 32, 64 that holds an average group (decode: 2 rows of 512 over 256 experts;
-// a shared expert: all T rows in one group). Larger groups take several token tiles.
+// Warp-MMA kernel (gemm_fp4_mma.cuh): 8-row token tiles, one weight block per tile.
+template <bool GATEUP>
+moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) {
+    using S = GemmFp4WarpShape<GATEUP>;
+    const int stages = S::stages_for(p.K);
+    CUtensorMap tx, tq, ts;
+    // token rows as [M][K/32][32]: one box = one whole row
+    const cuuint64_t xdims[3] = {32, (cuuint64_t)p.K / 32, (cuuint64_t)p.M};
+    const cuuint64_t xstr[2] = {64, (cuuint64_t)p.K * 2};
+    const cuuint32_t xbox[3] = {32, (cuuint32_t)(p.K / 32), 1};
+    moe_status_t st = make_tmap(&tx, p.a, 3, xdims, xstr, xbox, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                                CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != MOE_OK) return st;
+    const cuuint64_t qdims[3] = {(cuuint64_t)p.K / 2, (cuuint64_t)p.rows, (cuuint64_t)p.G};
+    const cuuint64_t qstr[2] = {(cuuint64_t)p.K / 2, (cuuint64_t)p.rows * (p.K / 2)};
+    const cuuint32_t qbox[3] = {FW_KS / 2, FW_BM, 1};
+    if ((st = make_tmap(&tq, p.q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_DATA_TYPE_UINT8)) != MOE_OK) return st;
+    const cuuint64_t sdims[3] = {(cuuint64_t)p.rows, (cuuint64_t)p.K / 32, (cuuint64_t)p.G};
+    const cuuint64_t sstr[2] = {(cuuint64_t)p.rows, (cuuint64_t)p.rows * (p.K / 32)};
+    const cuuint32_t sbox[3] = {FW_BM, FW_KS / 32, 1};
+    if ((st = make_tmap(&ts, p.s, 3, sdims, sstr, sbox, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
+        MOE_OK)
+        return st;
+    GemmArgs args;
+    args.group_offsets = p.offsets;
+    args.G = p.G;
+    args.M = p.M;
+    args.K = p.K;
+    args.n_out = p.n_out;
+    args.f = p.f;
+    args.n_tiles = (p.n_out + FW_BM - 1) / FW_BM;
+    args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
+    // weight blocks per tile: the token rows are loaded and converted once per tile, so a tile should stream
+    // several times their bytes (down: 139 KB of codes per block at d = 7168, f = 2048; gate|up twice that per
+    // block and 3.5x the K); fewer blocks per tile when that would leave fewer than 8 tiles per SM
+    int wpt = GATEUP ? 2 : 4;
+    const long token_blocks = std::min<long>(p.G, p.M);  // at least one per non-empty group
+    while (wpt > 1 && token_blocks * ((args.n_tiles + wpt - 1) / wpt) < 8L * sms) wpt >>= 1;
+    const long upper = ((long)p.M / FW_NT + p.G) * (long)((args.n_tiles + wpt - 1) / wpt);  // >= the tile count
+    const int grid = (int)(upper < sms ? upper : sms);
+    const int streamed_once = (long)p.M <= (long)p.G * FW_NT ? 1 : 0;
+    const cudaError_t e = launch_pdl(grouped_gemm_fp4_warp_kernel<GATEUP>, dim3(grid), dim3(FW_THREADS),
+                                     (size_t)S::smem_bytes(p.K, stages), stream, tx, tq, ts, args, streamed_once,
+                                     stages, wpt);
+    return check_launch(GATEUP ? "grouped_gemm_gateup_mxfp4 (warp MMA)" : "grouped_gemm_down_mxfp4 (warp MMA)", e);
+}
+
+// A few rows per expert (at most 8 on average: decode) and K <= 8192: the warp-MMA kernel. Otherwise the
+// tensor-memory kernel with the smallest token tile of 16, 32, 64 that holds an average group (a shared expert:
+// all T rows in one group). Larger groups take several token tiles.
 template <bool GATEUP>
 moe_status_t launch_fp4_nt(const Fp4Problem& p, int sms, cudaStream_t stream) {
+    if ((long)p.M <= 8L * p.G && p.K <= FW_MAX_K && GemmFp4WarpShape<GATEUP>::stages_for(p.K) >= 2)
+        return launch_fp4_warp<GATEUP>(p, sms, stream);
     if ((long)p.M <= 8L * p.G) return launch_fp4<16, GATEUP>(p, sms, stream);
     if ((long)p.M <= 24L * p.G) return launch_fp4<32, GATEUP>(p, sms, stream);
     return launch_fp4<64, GATEUP>(p, sms, stream);
@@ -819,6 +898,63 @@ moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_ga
     return launch_grouped_gemm(p, true, di.sms, stream);
 }
 
+size_t moe_grouped_gemm_gateup_gather_workspace_size(int G, int M, int d) {
+    if (G < 1 || M <= 0 || d <= 0 || (long)M >= (long)G * GG_BM) return 0;
+    return ((size_t)M * (size_t)d * 2 + 255) / 256 * 256;
+}
+
+moe_status_t moe_grouped_gemm_gateup_gather(const moe_bf16_t* x, const int32_t* row_src, int T,
+                                            const moe_bf16_t* w_gateup, const int32_t* group_offsets, int G, int M,
+                                            int d, int f, moe_bf16_t* h, void* ws, size_t ws_bytes,
+                                            cudaStream_t stream) {
+    moe_status_t st = check_gemm_args(x, w_gateup, group_offsets, G, M, d, f, h);
+    if (st != MOE_OK) return st;
+    if (T < 0 || (M > 0 && (T == 0 || !row_src))) return fail(MOE_ERR_INVALID_ARG, "x rows T=%d / row_src", T);
+    if ((reinterpret_cast<uintptr_t>(row_src) & 3u) != 0) return fail(MOE_ERR_INVALID_ARG, "row_src misaligned");
+    if ((long)T * (long)d > 0x7fffffffffffL) return fail(MOE_ERR_INVALID_ARG, "x too large");
+    const size_t need = moe_grouped_gemm_gateup_gather_workspace_size(G, M, d);
+    if (need && (!ws || ws_bytes < need))
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : (size_t)0);
+    if (need && !aligned16(ws)) return fail(MOE_ERR_WORKSPACE, "workspace not 16-byte aligned");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    if (need == 0) {  // groups of 128 rows or more on average: the gather rides in the operand load
+        if (di.sms < 2) return fail(MOE_ERR_UNSUPPORTED, "the gathering GEMM needs CTA pairs");
+        GemmProblem p{x, w_gateup, group_offsets, G, M, d, f, f, h};
+        p.row_src = row_src;
+        p.src_rows = T;
+        if (d % GG_BK == 0) return launch_swap<true, 2, 3, true, false, true>(p, di.sms, stream);
+        return launch_swap<true, 2, 3, false, false, true>(p, di.sms, stream);
+    }
+    // a few rows per expert: gather the rows into the workspace, then the GEMM the shape calls for
+    const int grid = grid_cap((M + 7) / 8, di.sms, 16);
+    const cudaError_t e = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, stream,
+                                     reinterpret_cast<const __nv_bfloat16*>(x), row_src, M, T, d,
+                                     reinterpret_cast<__nv_bfloat16*>(ws));
+    if ((st = check_launch("gather_rows", e)) != MOE_OK) return st;
+    const GemmProblem p{ws, w_gateup, group_offsets, G, M, d, f, f, h};
+    return launch_grouped_gemm(p, true, di.sms, stream);
+}
+
+moe_status_t moe_gather_rows(const moe_bf16_t* x, const int32_t* row_src, int T, int d, int R, moe_bf16_t* out,
+                             cudaStream_t stream) {
+    if (T < 0 || R < 0) return fail(MOE_ERR_INVALID_ARG, "T=%d, R=%d must be >= 0", T, R);
+    if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+    if (R == 0) return MOE_OK;
+    if (!x || !row_src || !out || T == 0) return fail(MOE_ERR_INVALID_ARG, "null pointer or T = 0");
+    if (!aligned16(x) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "x / out not 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(row_src) & 3u) != 0) return fail(MOE_ERR_INVALID_ARG, "row_src misaligned");
+    DeviceInfo di;
+    moe_status_t st = device_info(di);
+    if (st != MOE_OK) return st;
+    const int grid = grid_cap((R + 7) / 8, di.sms, 16);
+    const cudaError_t e = launch_pdl(gather_rows_kernel, dim3(grid), dim3(256), 0, stream,
+                                     reinterpret_cast<const __nv_bfloat16*>(x), row_src, R, T, d,
+                                     reinterpret_cast<__nv_bfloat16*>(out));
+    return check_launch("gather_rows", e);
+}
+
 moe_status_t moe_grouped_gemm_down(const moe_bf16_t* h, const moe_bf16_t* w_down, const int32_t* group_offsets,
                                    int G, int M, int d, int f, moe_bf16_t* y, cudaStream_t stream) {
     moe_status_t st = check_gemm_args(h, w_down, group_offsets, G, M, d, f, y);
@@ -892,6 +1028,51 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
                                      reinterpret_cast<const __nv_bfloat16*>(shared), T, d, k, T * k,
                                      reinterpret_cast<__nv_bfloat16*>(y));
     return check_launch("unpermute_combine", e);
+}
+
+size_t moe_grouped_gemm_down_combine_workspace_size(int T, int d) {
+    if (T <= 0 || d <= 0) return 0;
+    return ((size_t)T * (size_t)((d + 31) / 32) * sizeof(int32_t) + 255) / 256 * 256;
+}
+
+moe_status_t moe_grouped_gemm_down_combine(const moe_bf16_t* h, const moe_bf16_t* w_down,
+                                           const int32_t* group_offsets, int G, int M, int d, int f,
+                                           const int32_t* perm_src, const int32_t* inv_perm, const float* topk_w,
+                                           const moe_bf16_t* shared, int T, int k, moe_bf16_t* y_perm, moe_bf16_t* y,
+                                           void* ws, size_t ws_bytes, cudaStream_t stream) {
+    moe_status_t st = check_gemm_args(h, w_down, group_offsets, G, M, d, f, y_perm);
+    if (st != MOE_OK) return st;
+    if (T < 0 || k < 1 || k > 32) return fail(MOE_ERR_INVALID_ARG, "T=%d, k=%d (need T >= 0, 1 <= k <= 32)", T, k);
+    if ((long)T * k != (long)M) return fail(MOE_ERR_INVALID_ARG, "M=%d must be T*k=%ld", M, (long)T * k);
+    if (T == 0) return MOE_OK;
+    if (!perm_src || !inv_perm || !topk_w || !y) return fail(MOE_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(y) || (shared && !aligned16(shared)))
+        return fail(MOE_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+    const size_t need = moe_grouped_gemm_down_combine_workspace_size(T, d);
+    if (!ws || ws_bytes < need)
+        return fail(MOE_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, ws ? ws_bytes : (size_t)0);
+    if ((reinterpret_cast<uintptr_t>(ws) & 15u) != 0) return fail(MOE_ERR_WORKSPACE, "workspace not 16-byte aligned");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    const GemmProblem p{h, w_down, group_offsets, G, M, f, d, f, y_perm};
+    if ((long)M >= (long)G * GG_BM && di.sms >= 2) {  // prefill: the combine runs in the GEMM's epilogue
+        cudaError_t e = cudaMemsetAsync(ws, 0, need, stream);  // arrival counters
+        if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+        CombineArgs ca;
+        ca.perm_src = perm_src;
+        ca.inv_perm = inv_perm;
+        ca.topk_w = topk_w;
+        ca.shared = reinterpret_cast<const __nv_bfloat16*>(shared);
+        ca.y = reinterpret_cast<__nv_bfloat16*>(y);
+        ca.counters = reinterpret_cast<int*>(ws);
+        ca.T = T;
+        ca.k = k;
+        if (f % GG_BK == 0) return launch_swap<false, 2, 3, true, false, false, true>(p, di.sms, stream, ca);
+        return launch_swap<false, 2, 3, false, false, false, true>(p, di.sms, stream, ca);
+    }
+    // a few rows per expert: the GEMM the shape calls for, then the stand-alone combine
+    if ((st = launch_grouped_gemm(p, false, di.sms, stream)) != MOE_OK) return st;
+    return moe_unpermute_combine(y_perm, inv_perm, topk_w, shared, T, d, k, y, stream);
 }
 
 // ---- backward ----

@@ -172,6 +172,19 @@ __device__ __forceinline__ void tma_load_5d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// Four rows r0..r3 (any order, any rows of the 2D tensor) of one box width from column c0, written one after the
+// other at dst (4 x the box's row bytes, swizzled like a 4-row box). The map's box is one row high. Completion is
+// counted on the pair leader's barrier, as the other *_pair loads. No multicast.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster_addr, int c0,
+                                                 int r0, int r1, int r2, int r3, uint64_t cache_policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.cta_group::2"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster_addr), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+        "l"(cache_policy)
+        : "memory");
+}
+
 // Generic-proxy writes to shared memory made visible to the async proxy (TMA engine, tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -198,6 +211,8 @@ __device__ __forceinline__ void bulk_wait_group_read() {
 }
 // every committed group complete (its global writes done)
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// completed TMA stores (async proxy) ordered before this thread's later generic accesses and fences
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 // ---- tcgen05 / TMEM -------------------------------------------------------------------------------
 

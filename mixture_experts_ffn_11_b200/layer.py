@@ -35,10 +35,17 @@ class MoEFFN:
     weights: "bf16" keeps the expert weights as given; "mxfp4" encodes them once (moe_mxfp4_quantize, 4.25 bits
     per weight) and the layer then computes with the weights the encoding represents, through the MXFP4 grouped
     GEMMs; the bf16 tensors are not kept.
+    fused: with bf16 weights and groups of 128 rows or more on average (prefill), let the dispatch and the
+    collect steps ride in the grouped GEMMs: the gate|up GEMM reads its rows straight from x through perm_src
+    (moe_grouped_gemm_gateup_gather) instead of a grouped copy x_perm made by moe_permute, and the down GEMM's
+    epilogue does the weighted combine (moe_grouped_gemm_down_combine). Same results, bit for bit; the backward
+    pass then gathers x_perm itself. Off by default: on B200 the separate gather and combine kernels are faster
+    (the per-row gather loads and the combine's arrival counting slow the GEMMs by more than the two kernels
+    take).
     """
 
     def __init__(self, w_router, w_gateup, w_down, k: int, route: str = "topk_softmax", bias=None,
-                 w_gateup_shared=None, w_down_shared=None, weights: str = "bf16"):
+                 w_gateup_shared=None, w_down_shared=None, weights: str = "bf16", fused: bool = False):
         self.E, self.d = w_router.shape
         self.f = w_gateup.shape[1] // 2
         self.k = k
@@ -48,6 +55,8 @@ class MoEFFN:
         if weights not in ("bf16", "mxfp4"):
             raise ValueError(f"unknown weight format {weights!r}")
         self.weights = weights
+        self.fused = fused
+        self._x_perm_valid = False
         self.w_router, self.w_gateup, self.w_down, self.bias = w_router, w_gateup, w_down, bias
         self.w_gateup_shared, self.w_down_shared = w_gateup_shared, w_down_shared
         self.shared_f = w_gateup_shared.shape[0] // 2 if w_gateup_shared is not None else 0
@@ -102,6 +111,8 @@ class MoEFFN:
             "h": torch.empty(R, f, dtype=bf, device=dev),
             "y_perm": torch.empty(R, d, dtype=bf, device=dev),
             "ws": torch.empty(max(N.permute_workspace_size(T, E, k), 256), dtype=torch.uint8, device=dev),
+            "combine_ws": torch.empty(max(N.grouped_gemm_down_combine_workspace_size(T, d), 256), dtype=torch.uint8,
+                                      device=dev),
             "y": torch.empty(T, d, dtype=bf, device=dev),
         }
         if self.shared_f:
@@ -153,17 +164,31 @@ class MoEFFN:
         else:
             N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"], s)
         mark("route", False)
+        fused = self._fused(T)
         mark("permute", True)
-        N.permute(x, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], b["x_perm"],
-                  b["ws"], s)
+        if fused:  # grouping only; the gate|up GEMM gathers its rows from x
+            N.permute(None, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], None,
+                      b["ws"], s)
+        else:
+            N.permute(x, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], b["x_perm"],
+                      b["ws"], s)
+        self._x_perm_valid = not fused
         mark("permute", False)
         if shared is not None:
             # the routed GEMMs are persistent kernels sized to every SM: they start once the shared expert is done
             s.wait_event(shared_done)
         mark("gateup", True)
-        self._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)
+        if fused:
+            N.grouped_gemm_gateup_gather(x, b["perm_src"], self.w_gateup, b["offsets"], b["h"], None, s)
+        else:
+            self._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)
         mark("gateup", False)
         mark("down", True)
+        if fused:  # y_perm and, in the same kernel, y
+            N.grouped_gemm_down_combine(b["h"], self.w_down, b["offsets"], b["perm_src"], b["inv_perm"],
+                                        b["topk_w"], shared, b["y_perm"], b["y"], b["combine_ws"], s)
+            mark("down", False)
+            return b["y"]
         self._down(b["h"], "routed", b["offsets"], b["y_perm"], s)
         mark("down", False)
         mark("combine", True)
@@ -172,6 +197,12 @@ class MoEFFN:
         return b["y"]
 
     __call__ = forward
+
+    def _fused(self, T: int) -> bool:
+        """Whether forward() folds the row gather into the gate|up GEMM and the combine into the down GEMM for
+        T tokens."""
+        return (self.fused and self.weights == "bf16" and T > 0
+                and N.grouped_gemm_gateup_gather_workspace_size(self.E, T * self.k, self.d) == 0)
 
     def _gateup(self, a, which, offsets, h, stream):
         if self.weights == "mxfp4":
@@ -278,6 +309,9 @@ class MoEFFN:
         N.grouped_gemm_down(g["dy_perm"], wt["down"], b["offsets"], g["dh"], s)
         mark("bwd_dh", False)
         mark("bwd_preact", True)
+        if not self._x_perm_valid:  # the forward gathered its rows inside the GEMM: x_perm is made here
+            N.gather_rows(x, b["perm_src"], b["x_perm"], s)
+            self._x_perm_valid = True
         N.grouped_gemm_gateup_preact(b["x_perm"], self.w_gateup, b["offsets"], g["gu"], s)
         mark("bwd_preact", False)
         mark("bwd_swiglu", True)
@@ -323,12 +357,13 @@ class MoEFFN:
         return out
 
     def backward_kernel_launches(self, T: int, weight_grads: bool = True) -> int:
-        """Kernels one backward() launches: permute-backward 1, dh 1, pre-activations 1, SwiGLU-backward 1,
-        dx_perm 1, router 5, combine 1, and per weight gradient 4 (padded offsets, two transposes, the GEMM);
-        the shared expert 4 more (+ 8 with weight gradients)."""
+        """Kernels one backward() launches: permute-backward 1, dh 1, pre-activations 1 (+ 1 gather of x_perm
+        after a forward that folded it into the gate|up GEMM), SwiGLU-backward 1, dx_perm 1, router 5, combine 1,
+        and per weight gradient 4 (padded offsets, two transposes, the GEMM); the shared expert 4 more (+ 8 with
+        weight gradients)."""
         if T <= 0:
             return 0
-        n = 11 + (8 if weight_grads else 0)
+        n = 11 + (8 if weight_grads else 0) + (1 if self._fused(T) else 0)
         if self.shared_f:
             n += 4 + (8 if weight_grads else 0)
         return n
@@ -336,8 +371,10 @@ class MoEFFN:
     def kernel_launches(self, T: int) -> int:
         """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the
         tensor-core path with fused top-k is taken (E <= 128, T >= 2048), else logits + top-k;
-        permute 4; gate|up, down, combine 1 each; the shared expert 2 more."""
+        permute 4, gate|up, down, combine 1 each (fused: permute 3, gate|up 1, down with combine 1); the shared
+        expert 2 more."""
         if T <= 0:
             return 0
         route = 1 if (self.E <= 128 and T >= 2048) else 2
-        return route + 4 + 3 + (2 if self.shared_f else 0)
+        body = 3 + 2 if self._fused(T) else 4 + 3
+        return route + body + (2 if self.shared_f else 0)

@@ -53,6 +53,11 @@ def test_workspace_size(native):
     assert ws(64, 8, 2) == 256  # one 1024-assignment segment x 8 experts x 4 B, rounded to 256
     assert ws(16384, 128, 8) == 128 * 128 * 4
     assert ws(4096, 32, 4) % 256 == 0
+    gws = native.grouped_gemm_gateup_gather_workspace_size
+    assert gws(32, 16384, 2880) == 0  # >= 128 rows per group: the gather rides in the GEMM's operand load
+    assert gws(32, 32 * 128 - 1, 64) == ((32 * 128 - 1) * 64 * 2 + 255) // 256 * 256  # a grouped copy
+    assert gws(256, 512, 7168) == 512 * 7168 * 2
+    assert gws(4, 3, 8) == 256
 
 
 def test_invalid_arguments_rejected_before_any_launch(native):
@@ -78,6 +83,16 @@ def test_invalid_arguments_rejected_before_any_launch(native):
     assert lib.moe_grouped_gemm_gateup_mxfp4(16, 16, 16, 16, 1, 8, 64, 40, 16, null) == native.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_gemm_down_mxfp4(16, 16, null, 16, 1, 8, 64, 64, 16, null) == native.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_gemm_down_mxfp4(16, 24, 16, 16, 1, 8, 64, 64, 16, null) == native.MOE_ERR_INVALID_ARG
+    # gathering gate|up: no row_src; T = 0 with rows to compute; workspace missing on the small-group path
+    assert lib.moe_grouped_gemm_gateup_gather(16, null, 8, 16, 16, 1, 8, 8, 8, 16, null, 0, null) == \
+        native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_gateup_gather(16, 16, 0, 16, 16, 1, 8, 8, 8, 16, null, 0, null) == \
+        native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_gateup_gather(16, 16, 8, 16, 16, 1, 8, 8, 8, 16, null, 0, null) == \
+        native.MOE_ERR_WORKSPACE
+    # row gather: d not a multiple of 8; misaligned output
+    assert lib.moe_gather_rows(16, 16, 4, 12, 4, 16, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_gather_rows(16, 16, 4, 8, 4, 24, null) == native.MOE_ERR_INVALID_ARG
     # missing workspace
     st = lib.moe_permute(null, 16, 64, 0, 8, 2, 16, 16, 16, 16, null, null, 0, null)
     assert st == native.MOE_ERR_WORKSPACE
