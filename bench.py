@@ -365,7 +365,8 @@ def bench_workload(args):
                 raise SystemExit(f"--shape: {key} cannot be overridden")
             over[key] = int(val)
         tag = ",".join(f"{k}={v}" for k, v in over.items())
-        wl = synth.workload(args.workload, **over, name=f"{wl.name}[{tag}]")
+        wl = synth.workload(args.workload, **over)
+        wl = synth.Workload(**{**wl.__dict__, "name": f"{wl.name}[{tag}]"})
     return wl
 
 

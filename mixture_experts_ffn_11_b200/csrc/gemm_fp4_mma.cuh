@@ -26,12 +26,15 @@
 // token, block and t, 16 bytes of f16 in the order x0 x2 x4 x6 x1 x3 x5 x7 (x_i = element 32b + 8t + i), one
 // 16-byte load giving the B fragments of both MMAs. (A byte's low code goes to the low half of the f16 pair.)
 //
-// CTA (288 threads, one per SM, persistent over tiles): warps 0-7 compute, warp 8 is the TMA producer.
+// CTA (544 threads, one per SM, persistent over tiles): warps 0-15 compute, warp 16 is the TMA producer.
 // Tile = (group g, block of 8 token rows, run of `wpt` weight blocks of 128 rows; gate|up: 128 gate rows and the
 // matching 128 up rows). Per tile the producer loads the 8 token rows whole (one box per row) and then streams, per
 // weight block, stages of K = 256: codes [128 rows x 128 bytes] (128-byte swizzle) and scales [8 x 128] per
-// projection. The compute warps scale and convert the token rows in place once per tile (warp w takes row w),
-// then work through the stages; warp w computes weight rows 16w .. 16w+15 of each block. Every wait is bounded.
+// projection. Warps 0-7 scale and convert the token rows in place once per tile (warp w takes row w). Warps w and
+// w + 8 compute weight rows 16w .. 16w+15 of each block, w the even and w + 8 the odd 32-element blocks of every
+// stage (four warps per SM sub-partition hide the MMA and load latencies); at the end of a weight block warp w + 8
+// hands its partial sums to warp w through shared memory, which adds them to its own (always in that order) and
+// stores the outputs. Every wait is bounded.
 #pragma once
 #include "common.cuh"
 #include "gemm.cuh"
@@ -41,35 +44,40 @@
 namespace moe {
 
 constexpr int FW_NT = 8;                      // token rows per tile (the MMA's N)
-constexpr int FW_WARPS = 8;                   // compute warps
+constexpr int FW_WARPS = 16;                  // compute warps
 constexpr int FW_THREADS = (FW_WARPS + 1) * 32;
-constexpr int FW_BM = 16 * FW_WARPS;          // weight rows per block: 128, as the tensor-memory kernel's maps
 constexpr int FW_KS = GF_KS;                  // K per stage: 256 (128 bytes of codes per row)
 constexpr int FW_MAX_K = 8192;                // one TMA box per token row: K / 32 <= 256
 constexpr int FW_BAR_BYTES = 512;
 
+// gate|up: blocks of 128 weight rows (and the matching 128 up rows), two warps per 16 rows (even / odd K blocks);
+// down: blocks of 256 rows, one warp per 16 rows over all of K (no hand-off; K is short: d x f = 7168 x 2048)
 template <bool GATEUP>
 struct GemmFp4WarpShape {
+    static constexpr int RW = GATEUP ? 8 : 16;         // row warps, 16 weight rows each
+    static constexpr int KSPL = FW_WARPS / RW;         // warps per 16 rows
+    static constexpr int BM = 16 * RW;                 // weight rows per block
     static constexpr int BLOCKS = GATEUP ? 2 : 1;
-    static constexpr int Q_BYTES = FW_BM * (FW_KS / 2);  // 16 KB of codes per projection block
-    static constexpr int S_BYTES = (FW_KS / 32) * FW_BM; // 1 KB of scales
+    static constexpr int Q_BYTES = BM * (FW_KS / 2);   // codes of one projection block (16 or 32 KB)
+    static constexpr int S_BYTES = (FW_KS / 32) * BM;  // its scales
+    static constexpr int RED_BYTES = KSPL > 1 ? RW * 32 * 8 * 4 : 0;  // partial sums handed from warp w + RW to w
     static constexpr int STAGE_BYTES = BLOCKS * (Q_BYTES + S_BYTES);
-    static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;
+    __host__ __device__ static int table_bytes(int G) { return (2 * (G + 1) * 4 + 127) / 128 * 128; }
     static_assert(STAGE_BYTES % 1024 == 0, "stages start on 1024-byte atoms");
     // token row stride in shared memory: K rounded up to 64 elements (the odd rows' 32-element blocks are stored
     // swapped in pairs), in bytes
     __host__ __device__ static int row_bytes(int K) { return (K + 63) / 64 * 64 * 2; }
     __host__ __device__ static int b_bytes(int K) { return FW_NT * row_bytes(K); }
-    // smem: [token rows][ring][barriers][token scales][group tables], the first two 1024-aligned
+    // smem: [token rows][ring][barriers, token scales][partial sums][group tables], the first two 1024-aligned
     __host__ __device__ static int ring_offset(int K) { return (b_bytes(K) + 1023) / 1024 * 1024; }
-    __host__ __device__ static int smem_bytes(int K, int stages) {
-        return 1024 + ring_offset(K) + stages * STAGE_BYTES + FW_BAR_BYTES + TABLE_BYTES;
+    __host__ __device__ static int smem_bytes(int K, int stages, int G) {
+        return 1024 + ring_offset(K) + stages * STAGE_BYTES + FW_BAR_BYTES + RED_BYTES + table_bytes(G);
     }
     static constexpr int MAX_SMEM = 232448;
     // deepest ring (at most 8 stages) that fits beside the token rows
-    __host__ __device__ static int stages_for(int K) {
+    __host__ __device__ static int stages_for(int K, int G) {
         int s = 8;
-        while (s > 0 && smem_bytes(K, s) > MAX_SMEM) --s;
+        while (s > 0 && smem_bytes(K, s, G) > MAX_SMEM) --s;
         return s;
     }
 };
@@ -93,9 +101,9 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// E8M0 scale code -> 2^(s - 127) as fp32 (s = 0: 2^-127, a subnormal)
+// E8M0 scale code -> 2^(s - 127) as fp32 (s = 0: 2^-127, the subnormal 0x00400000; every s >= 1 gives bits above it)
 __device__ __forceinline__ float e8m0_to_f32(uint32_t s) {
-    return __uint_as_float(s ? (s << 23) : 0x00400000u);
+    return __uint_as_float(max(s << 23, 0x00400000u));
 }
 
 // 8 bf16 (one 16-byte chunk, elements 0..7 in order) times 2^-e as f16, in the order 0 2 4 6 1 3 5 7
@@ -132,16 +140,19 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
     uint64_t* bfull_bar = empty_bar + 8;
     uint64_t* bempty_bar = bfull_bar + 1;
     uint64_t* bconv_bar = bempty_bar + 1;  // every token row of the tile converted
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bconv_bar + 1);
-    float* tok_scale = reinterpret_cast<float*>(ring + stages_n * S::STAGE_BYTES + 256);  // [8]
-    int32_t* s_off = reinterpret_cast<int32_t*>(ring + stages_n * S::STAGE_BYTES + FW_BAR_BYTES);
-    int32_t* s_tp = s_off + (GG_MAX_GROUPS + 1);
+    uint64_t* red_full = bconv_bar + 1;  // [8] (two warps per rows) partial sums of warp w + RW are in red[w]
+    uint64_t* red_empty = red_full + 8;  // [8] red[w] has been read
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(red_empty + 8);
+    float* tok_scale = reinterpret_cast<float*>(ring + stages_n * S::STAGE_BYTES + 384);  // [8]
+    float* red = reinterpret_cast<float*>(ring + stages_n * S::STAGE_BYTES + FW_BAR_BYTES);  // [RW][32][8]
+    int32_t* s_off = reinterpret_cast<int32_t*>(ring + stages_n * S::STAGE_BYTES + FW_BAR_BYTES + S::RED_BYTES);
+    int32_t* s_tp = s_off + (args.G + 1);  // tables sized by G (table_bytes)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = args.G;
     const int KB32 = K / 32;                    // scale blocks per row
     const int KS = (K + FW_KS - 1) / FW_KS;     // stages per weight block
-    const int wblocks = args.n_tiles;           // weight blocks of 128 output columns
+    const int wblocks = args.n_tiles;           // weight blocks of S::BM output columns
     const int wchunks = (wblocks + wpt - 1) / wpt;
 
     if (threadIdx.x == 0) {
@@ -152,6 +163,10 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         mbar_init(bfull_bar, 1);
         mbar_init(bempty_bar, FW_WARPS);
         mbar_init(bconv_bar, FW_WARPS);
+        for (int w = 0; w < 8; ++w) {
+            mbar_init(&red_full[w], 32);
+            mbar_init(&red_empty[w], 32);
+        }
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmX);
@@ -237,7 +252,7 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
             if (!ok) break;
             const int wb_end = min(wblocks, (wc + 1) * wpt);
             for (int wb = wc * wpt; wb < wb_end && ok; ++wb) {
-                const int wrow = wb * FW_BM;
+                const int wrow = wb * S::BM;
                 for (int ks = 0; ks < KS; ++ks) {
                     if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -270,13 +285,18 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---------------- compute warps 0-7 ----------------
+        // ---------------- compute warps 0-15 ----------------
         const int gq = lane >> 2, t = lane & 3;
-        const int ra = warp * 16 + gq, rb = ra + 8;  // this thread's weight rows within the block
+        const int rw = warp % S::RW, kw = warp / S::RW;  // row group; K part (two per rows: even, odd blocks)
+        const int ra = rw * 16 + gq, rb = ra + 8;        // this thread's weight rows within the block
+        // byte offsets in a stage's code block of word t of 16-byte unit `kw` of rows ra, rb (128-byte swizzle: unit
+        // u of row r sits at u ^ (r % 8)); unit kw + KSPL * i is then offset ^ ((KSPL * i) << 4)
+        const uint32_t qa = (uint32_t)(ra * 128 + ((kw ^ (ra & 7)) << 4) + 4 * t);
+        const uint32_t qb = (uint32_t)(rb * 128 + ((kw ^ (rb & 7)) << 4) + 4 * t);
         const int nchunk = K / 8;                     // 16-byte chunks of a token row
         const int npairs = 4 * ((nchunk + 7) / 8);    // (chunk, chunk + 4) pairs, per 64 elements
         int stage = 0;
-        uint32_t phase = 0, bphase = 0;
+        uint32_t phase = 0, bphase = 0, rphase = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
             int g, tb, wc;
@@ -287,7 +307,7 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             bphase ^= 1u;
             if (!ok) break;
-            {  // token row `warp`: largest magnitude, scale exponent, in-place conversion to permuted f16
+            if (warp < FW_NT) {  // token row `warp`: largest magnitude, scale exponent, conversion to permuted f16
                 uint8_t* row = brows + warp * row_bytes;
                 uint32_t mx = 0;
                 for (int c = lane; c < nchunk; c += 32) {
@@ -328,8 +348,12 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             const float tsc0 = tok_scale[2 * t], tsc1 = tok_scale[2 * t + 1];
-            const uint8_t* brow = brows + gq * row_bytes;
-            const int bx = (gq & 1) * 4;  // this token row's unit swap
+            // token row gq, unit 4 kb + t of block kb = 8 ks + KSPL i + kw, stored at block kb ^ (gq % 2): with two
+            // warps per rows that is 8 ks + 2 i + (kw ^ (gq % 2)); with one, 8 ks + (i ^ (gq % 2)), i.e. +i for even
+            // i and i - 2 (gq % 2) for odd i
+            const int par = gq & 1;
+            const uint8_t* bx0 = brows + gq * row_bytes + (((S::KSPL > 1 ? (kw ^ par) : par) * 4 + t) << 4);
+            const uint8_t* bx1 = bx0 - (S::KSPL > 1 ? 0 : 2 * par * 64);  // odd i, one warp per rows
             const int wb_end = min(wblocks, (wc + 1) * wpt);
             for (int wb = wc * wpt; wb < wb_end && ok; ++wb) {
                 float acc_g[4] = {0.f, 0.f, 0.f, 0.f}, acc_u[4] = {0.f, 0.f, 0.f, 0.f};
@@ -338,19 +362,21 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     const uint8_t* st = ring + stage * S::STAGE_BYTES;
-                    const uint8_t* sc = st + S::BLOCKS * S::Q_BYTES;
-                    const int nb = min(FW_KS / 32, KB32 - ks * (FW_KS / 32));
-#pragma unroll 2
-                    for (int b = 0; b < nb; ++b) {
-                        const int kb = ks * (FW_KS / 32) + b;
-                        const uint4 xv = *reinterpret_cast<const uint4*>(brow + (((kb * 4 + t) ^ bx) << 4));
+                    const uint8_t* sc = st + S::BLOCKS * S::Q_BYTES + kw * S::BM;
+                    const int nb = KB32 - ks * (FW_KS / 32);  // blocks of this stage inside K (>= 8: all)
+#pragma unroll
+                    for (int i = 0; i < FW_KS / 32 / S::KSPL; ++i) {
+                        if (S::KSPL * i + kw >= nb) break;
+                        const uint8_t* bx = (S::KSPL > 1 || (i & 1) == 0) ? bx0 : bx1;
+                        const uint4 xv = *reinterpret_cast<const uint4*>(bx + ks * (FW_KS * 2) + i * (S::KSPL * 64));
 #pragma unroll
                         for (int blk = 0; blk < S::BLOCKS; ++blk) {
                             const uint8_t* q = st + blk * S::Q_BYTES;
-                            const uint32_t wa = *reinterpret_cast<const uint32_t*>(q + ra * 128 + ((b ^ (ra & 7)) << 4) + 4 * t);
-                            const uint32_t wbv = *reinterpret_cast<const uint32_t*>(q + rb * 128 + ((b ^ (rb & 7)) << 4) + 4 * t);
-                            const float sa = e8m0_to_f32(sc[blk * S::S_BYTES + b * FW_BM + ra]);
-                            const float sb = e8m0_to_f32(sc[blk * S::S_BYTES + b * FW_BM + rb]);
+                            const uint32_t sw = (uint32_t)((S::KSPL * i) << 4);
+                            const uint32_t wa = *reinterpret_cast<const uint32_t*>(q + (qa ^ sw));
+                            const uint32_t wbv = *reinterpret_cast<const uint32_t*>(q + (qb ^ sw));
+                            const float sa = e8m0_to_f32(sc[blk * S::S_BYTES + S::KSPL * i * S::BM + ra]);
+                            const float sb = e8m0_to_f32(sc[blk * S::S_BYTES + S::KSPL * i * S::BM + rb]);
                             const uint32_t a0[4] = {e2m1x2_to_f16x2(wa), e2m1x2_to_f16x2(wbv), e2m1x2_to_f16x2(wa >> 8),
                                                     e2m1x2_to_f16x2(wbv >> 8)};
                             const uint32_t a1[4] = {e2m1x2_to_f16x2(wa >> 16), e2m1x2_to_f16x2(wbv >> 16),
@@ -373,15 +399,42 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
                     }
                 }
                 if (!ok) break;
+                if constexpr (S::KSPL > 1) {
+                    float4* slot = reinterpret_cast<float4*>(red + (rw * 32 + lane) * 8);
+                    if (kw == 1) {  // partial sums of the odd blocks to warp rw
+                        ok = mbar_wait_bounded(&red_empty[rw], rphase ^ 1u, abort_flag);
+                        ok = __all_sync(0xffffffffu, ok);
+                        if (!ok) break;
+                        slot[0] = make_float4(acc_g[0], acc_g[1], acc_g[2], acc_g[3]);
+                        slot[1] = make_float4(acc_u[0], acc_u[1], acc_u[2], acc_u[3]);
+                        mbar_arrive(&red_full[rw]);
+                        rphase ^= 1u;
+                        continue;
+                    }
+                    ok = mbar_wait_bounded(&red_full[rw], rphase, abort_flag);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    const float4 og = slot[0], ou = slot[1];
+                    mbar_arrive(&red_empty[rw]);
+                    rphase ^= 1u;
+                    acc_g[0] += og.x;
+                    acc_g[1] += og.y;
+                    acc_g[2] += og.z;
+                    acc_g[3] += og.w;
+                    acc_u[0] += ou.x;
+                    acc_u[1] += ou.y;
+                    acc_u[2] += ou.z;
+                    acc_u[3] += ou.w;
+                }
                 // outputs: weight rows ra, rb (output columns) x tokens 2t, 2t+1
-                const int ca = wb * FW_BM + ra, cb = wb * FW_BM + rb;
+                const int ca = wb * S::BM + ra, cb = wb * S::BM + rb;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int tok = 2 * t + (i & 1);
-                    const int col = (i < 2) ? ca : cb;
+                for (int j = 0; j < 4; ++j) {
+                    const int tok = 2 * t + (j & 1);
+                    const int col = (j < 2) ? ca : cb;
                     if (tok >= rows || col >= args.n_out) continue;
-                    const float ts = (i & 1) ? tsc1 : tsc0;
-                    const float v = GATEUP ? swiglu(acc_g[i] * ts, acc_u[i] * ts) : acc_g[i] * ts;
+                    const float ts = (j & 1) ? tsc1 : tsc0;
+                    const float v = GATEUP ? swiglu(acc_g[j] * ts, acc_u[j] * ts) : acc_g[j] * ts;
                     args.out[(size_t)(row0 + tok) * args.n_out + col] = __float2bfloat16_rn(v);
                 }
             }

@@ -520,7 +520,7 @@ moe_status_t launch_fp4(const Fp4Problem& p, int sms, cudaStream_t stream) {
 template <bool GATEUP>
 moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) {
     using S = GemmFp4WarpShape<GATEUP>;
-    const int stages = S::stages_for(p.K);
+    const int stages = S::stages_for(p.K, p.G);
     CUtensorMap tx, tq, ts;
     // token rows as [M][K/32][32]: one box = one whole row
     const cuuint64_t xdims[3] = {32, (cuuint64_t)p.K / 32, (cuuint64_t)p.M};
@@ -531,11 +531,11 @@ moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) 
     if (st != MOE_OK) return st;
     const cuuint64_t qdims[3] = {(cuuint64_t)p.K / 2, (cuuint64_t)p.rows, (cuuint64_t)p.G};
     const cuuint64_t qstr[2] = {(cuuint64_t)p.K / 2, (cuuint64_t)p.rows * (p.K / 2)};
-    const cuuint32_t qbox[3] = {FW_KS / 2, FW_BM, 1};
+    const cuuint32_t qbox[3] = {FW_KS / 2, S::BM, 1};
     if ((st = make_tmap(&tq, p.q, 3, qdims, qstr, qbox, CU_TENSOR_MAP_DATA_TYPE_UINT8)) != MOE_OK) return st;
     const cuuint64_t sdims[3] = {(cuuint64_t)p.rows, (cuuint64_t)p.K / 32, (cuuint64_t)p.G};
     const cuuint64_t sstr[2] = {(cuuint64_t)p.rows, (cuuint64_t)p.rows * (p.K / 32)};
-    const cuuint32_t sbox[3] = {FW_BM, FW_KS / 32, 1};
+    const cuuint32_t sbox[3] = {S::BM, FW_KS / 32, 1};
     if ((st = make_tmap(&ts, p.s, 3, sdims, sstr, sbox, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
         MOE_OK)
         return st;
@@ -546,19 +546,20 @@ moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) 
     args.K = p.K;
     args.n_out = p.n_out;
     args.f = p.f;
-    args.n_tiles = (p.n_out + FW_BM - 1) / FW_BM;
+    args.n_tiles = (p.n_out + S::BM - 1) / S::BM;
     args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
     // weight blocks per tile: the token rows are loaded and converted once per tile, so a tile should stream
-    // several times their bytes (down: 139 KB of codes per block at d = 7168, f = 2048; gate|up twice that per
-    // block and 3.5x the K); fewer blocks per tile when that would leave fewer than 8 tiles per SM
-    int wpt = GATEUP ? 2 : 4;
+    // several times their bytes (down: 278 KB of codes per 256-row block at d = 7168, f = 2048; gate|up about as
+    // much per 128 + 128-row block and 3.5x the K); fewer blocks per tile when that would leave fewer than 8
+    // tiles per SM
+    int wpt = 4;
     const long token_blocks = std::min<long>(p.G, p.M);  // at least one per non-empty group
     while (wpt > 1 && token_blocks * ((args.n_tiles + wpt - 1) / wpt) < 8L * sms) wpt >>= 1;
     const long upper = ((long)p.M / FW_NT + p.G) * (long)((args.n_tiles + wpt - 1) / wpt);  // >= the tile count
     const int grid = (int)(upper < sms ? upper : sms);
     const int streamed_once = (long)p.M <= (long)p.G * FW_NT ? 1 : 0;
     const cudaError_t e = launch_pdl(grouped_gemm_fp4_warp_kernel<GATEUP>, dim3(grid), dim3(FW_THREADS),
-                                     (size_t)S::smem_bytes(p.K, stages), stream, tx, tq, ts, args, streamed_once,
+                                     (size_t)S::smem_bytes(p.K, stages, p.G), stream, tx, tq, ts, args, streamed_once,
                                      stages, wpt);
     return check_launch(GATEUP ? "grouped_gemm_gateup_mxfp4 (warp MMA)" : "grouped_gemm_down_mxfp4 (warp MMA)", e);
 }
@@ -568,7 +569,7 @@ moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) 
 // all T rows in one group). Larger groups take several token tiles.
 template <bool GATEUP>
 moe_status_t launch_fp4_nt(const Fp4Problem& p, int sms, cudaStream_t stream) {
-    if ((long)p.M <= 8L * p.G && p.K <= FW_MAX_K && GemmFp4WarpShape<GATEUP>::stages_for(p.K) >= 2)
+    if ((long)p.M <= 8L * p.G && p.K <= FW_MAX_K && GemmFp4WarpShape<GATEUP>::stages_for(p.K, p.G) >= 2)
         return launch_fp4_warp<GATEUP>(p, sms, stream);
     if ((long)p.M <= 8L * p.G) return launch_fp4<16, GATEUP>(p, sms, stream);
     if ((long)p.M <= 24L * p.G) return launch_fp4<32, GATEUP>(p, sms, stream);
