@@ -553,7 +553,8 @@ moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) 
     // much per 128 + 128-row block and 3.5x the K); fewer blocks per tile when that would leave fewer than 8
     // tiles per SM
     int wpt = 4;
-    const long token_blocks = std::min<long>(p.G, p.M);  // at least one per non-empty group
+    // token blocks: at least one per non-empty group, and M / 8 in all
+    const long token_blocks = std::max<long>(std::min<long>(p.G, p.M), (p.M + FW_NT - 1) / FW_NT);
     while (wpt > 1 && token_blocks * ((args.n_tiles + wpt - 1) / wpt) < 8L * sms) wpt >>= 1;
     const long upper = ((long)p.M / FW_NT + p.G) * (long)((args.n_tiles + wpt - 1) / wpt);  // >= the tile count
     const int grid = (int)(upper < sms ? upper : sms);
@@ -566,7 +567,9 @@ moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) 
 
 // A few rows per expert (at most 8 on average: decode) and K <= 8192: the warp-MMA kernel. Otherwise the
 // tensor-memory kernel with the smallest token tile of 16, 32, 64 that holds an average group (a shared expert:
-// all T rows in one group). Larger groups take several token tiles.
+// all T rows in one group; measured: on the decode layer's side stream the warp kernel took its 64 rows in 108
+// instead of 128 µs but, on every SM, slowed the routing and grouping beside it by as much). Larger groups take
+// several token tiles.
 template <bool GATEUP>
 moe_status_t launch_fp4_nt(const Fp4Problem& p, int sms, cudaStream_t stream) {
     if ((long)p.M <= 8L * p.G && p.K <= FW_MAX_K && GemmFp4WarpShape<GATEUP>::stages_for(p.K, p.G) >= 2)
