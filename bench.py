@@ -454,7 +454,7 @@ def run_ours(args):
     x = inp["x"]
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    launches_per_step = layer.kernel_launches(wl.T)
+    launches_per_step = layer.kernel_launches(wl.T, train=args.backward)
     sampler = ClockSampler(torch.cuda.get_device_properties(dev).uuid.__str__() if rank >= 0 else None)
     sampler.start()
 
@@ -462,10 +462,10 @@ def run_ours(args):
     if args.backward:
         dy = torch.empty(wl.T, wl.d, dtype=torch.bfloat16, device=dev)
         synth.fill_device(dy, wl.seed, synth.TID_DY, 0, synth.X_SIGMA)
-        launches_per_step += layer.backward_kernel_launches(wl.T)
+        launches_per_step += layer.backward_kernel_launches(wl.T, train_forward=True)
 
     def step(timing=None):
-        y = layer.forward(x, timing=timing)
+        y = layer.forward(x, timing=timing, train=dy is not None)
         if dy is not None:
             layer.backward(dy, timing=timing)
         return y
@@ -606,11 +606,12 @@ def run_ours(args):
     line["config"]["dispatch"] = ("gather in gate|up GEMM, combine in down GEMM" if layer._fused(wl.T)
                                   else "moe_permute gather, moe_unpermute_combine")
     if args.backward:
-        # the training step: forward + backward (top-k selection held fixed), weight gradients included
+        # the training step: forward (keeping the gate|up pre-activations) + backward (top-k selection held
+        # fixed), weight gradients included: 6 + 12 R d f, and the same for the shared expert over T rows
         R, d, f, fs = wl.R, wl.d, wl.f, wl.shared_f
-        bwd_flop = {"bwd_dh": 2.0 * R * d * f, "bwd_preact": 4.0 * R * d * f, "bwd_dx_perm": 4.0 * R * d * f,
+        bwd_flop = {"bwd_dh": 2.0 * R * d * f, "bwd_dx_perm": 4.0 * R * d * f,
                     "bwd_dw_down": 2.0 * R * d * f, "bwd_dw_gateup": 4.0 * R * d * f}
-        train_flop = lflop + 16.0 * R * d * f + 16.0 * wl.T * d * fs
+        train_flop = lflop + 12.0 * R * d * f + 12.0 * wl.T * d * fs
         top = max(bwd_flop, key=lambda n: stages[n])  # the backward stage that takes longest
         tr_roof = roofline_entry(top, {"flop": bwd_flop[top], "bytes": 0.0}, stages[top], peaks, peak_kind, None)
         line.update({"metric": "MoE-layer training step (forward + backward) tokens/s and TFLOP/s, 1xB200",

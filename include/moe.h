@@ -351,7 +351,8 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
  * call y = combine(down(swiglu(gateup(x_perm)))) for an upstream gradient dy:
  *   moe_permute_backward            dy_perm[r] = w[t,j] dy[t], dw[t,j] = <dy[t], y_perm[r]>
  *   moe_grouped_gemm_down           dh = dy_perm W_down[e]        (weights transposed: W_down^T [E][f][d])
- *   moe_grouped_gemm_gateup_preact  g | u of the forward, recomputed [M][2f]
+ *   moe_grouped_gemm_gateup_preact  g | u of the forward, recomputed [M][2f] (or kept by a
+ *                                   forward that ran moe_grouped_gemm_gateup_save)
  *   moe_swiglu_backward             dg = dh u silu'(g), du = dh silu(g)
  *   moe_grouped_gemm_down           dx_perm = [dg|du] W_gateup[e] (weights transposed: W_gateup^T [E][d][2f])
  *   moe_unpermute_combine           dx = sum over slots of dx_perm (unit weights) + the router's share
@@ -368,6 +369,18 @@ moe_status_t moe_unpermute_combine(const moe_bf16_t* y_perm, const int32_t* inv_
 moe_status_t moe_grouped_gemm_gateup_preact(const moe_bf16_t* a, const moe_bf16_t* w_gateup,
                                             const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* gu,
                                             cudaStream_t stream);
+
+/* A training forward's gate|up projection: h exactly as moe_grouped_gemm_gateup
+ * and, from the same sums, gu exactly as moe_grouped_gemm_gateup_preact (gate
+ * in columns [0, f), up in [f, 2f)), so that the backward pass need not
+ * recompute them. With 128 rows or more per group on average one kernel
+ * writes both (the epilogue stores g and u beside h: 2f more bf16 values per
+ * row, no second pass over the weights); otherwise the two calls run one after
+ * the other. Arguments and limits as moe_grouped_gemm_gateup; gu [M][2f],
+ * 16-byte aligned. */
+moe_status_t moe_grouped_gemm_gateup_save(const moe_bf16_t* a, const moe_bf16_t* w_gateup,
+                                          const int32_t* group_offsets, int G, int M, int d, int f, moe_bf16_t* h,
+                                          moe_bf16_t* gu, cudaStream_t stream);
 
 /* SwiGLU derivative: with s = 1 / (1 + exp(-g)), for every row and n < f
  *   dgu[r][n] = dh[r][n] * u * s * (1 + g * (1 - s)),  dgu[r][f + n] = dh[r][n] * g * s,

@@ -28,6 +28,7 @@ EXPORTS = ("moe_route_topk", "moe_router_split_weights", "moe_route_topk_split",
            "moe_grouped_gemm_gateup_gather", "moe_gather_rows", "moe_grouped_gemm_down",
            "moe_grouped_gemm_down_combine_workspace_size", "moe_grouped_gemm_down_combine", "moe_mxfp4_quantize", "moe_grouped_gemm_gateup_mxfp4",
            "moe_grouped_gemm_down_mxfp4", "moe_unpermute_combine", "moe_grouped_gemm_gateup_preact",
+           "moe_grouped_gemm_gateup_save",
            "moe_swiglu_backward", "moe_permute_backward", "moe_transpose_weights",
            "moe_grouped_weight_grad_workspace_size", "moe_grouped_weight_grad", "moe_router_backward_workspace_size",
            "moe_router_backward", "moe_set_gemm_kernel", "moe_test_set_wait", "moe_get_device_error",
@@ -67,6 +68,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "moe_grouped_gemm_down_mxfp4": [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp],
         "moe_unpermute_combine": [vp, vp, vp, vp, ci, ci, ci, vp, vp],
         "moe_grouped_gemm_gateup_preact": [vp, vp, vp, ci, ci, ci, ci, vp, vp],
+        "moe_grouped_gemm_gateup_save": [vp, vp, vp, ci, ci, ci, ci, vp, vp, vp],
         "moe_swiglu_backward": [vp, vp, ci, ci, vp, vp],
         "moe_permute_backward": [vp, vp, vp, vp, ci, ci, ci, vp, vp, vp],
         "moe_transpose_weights": [vp, ci, ci, ci, vp, vp],
@@ -356,6 +358,20 @@ def grouped_gemm_gateup_preact(a, w_gateup, group_offsets, gu, stream=None):
     _need(gu, torch.bfloat16, (M, 2 * f), "gu")
     _check(_lib.moe_grouped_gemm_gateup_preact(_p(a), _p(w_gateup), _p(group_offsets), G, M, d, f, _p(gu),
                                                _stream(stream)), "moe_grouped_gemm_gateup_preact")
+
+
+def grouped_gemm_gateup_save(a, w_gateup, group_offsets, h, gu, stream=None):
+    """h [M, f] as grouped_gemm_gateup and gu [M, 2f] as grouped_gemm_gateup_preact, from one pass where possible."""
+    M, d = a.shape
+    G, two_f, _ = w_gateup.shape
+    f = two_f // 2
+    _need(a, torch.bfloat16, (M, d), "a")
+    _need(w_gateup, torch.bfloat16, (G, 2 * f, d), "w_gateup")
+    _need(group_offsets, torch.int32, (G + 1,), "group_offsets")
+    _need(h, torch.bfloat16, (M, f), "h")
+    _need(gu, torch.bfloat16, (M, 2 * f), "gu")
+    _check(_lib.moe_grouped_gemm_gateup_save(_p(a), _p(w_gateup), _p(group_offsets), G, M, d, f, _p(h), _p(gu),
+                                             _stream(stream)), "moe_grouped_gemm_gateup_save")
 
 
 def swiglu_backward(dh, gu, dgu, stream=None):

@@ -46,6 +46,7 @@ struct GemmArgs {
     int f;        // gate|up: first up row inside an expert's [2f][d] slab
     int n_tiles;  // N-blocks per group
     __nv_bfloat16* out;  // [M][n_out]
+    __nv_bfloat16* out2 = nullptr;     // gate|up saving its pre-activations: [M][2f]
     const int32_t* row_src = nullptr;  // gathering kernels: A row r is row row_src[r] of a [src_rows][K] tensor
     int src_rows = 0;
 };

@@ -48,7 +48,7 @@ constexpr int GS_MAX_N = 256;  // token rows per tile (UMMA N for M = 256, a mul
 //   [W k0 | W k1 | ... | X k0 | X k1 | ...], W blocks 16 KB apart, X blocks (rows per CTA) * 128 bytes apart.
 // BIGBOX: the operands are read through tensor maps that view [rows][K] as [K/64][rows][64] (K a multiple of 64),
 // so one TMA box brings the SUB K blocks of a stage at once (a 32 KB box moves faster than two 16 KB ones).
-template <bool GATEUP, int SUB, int STAGES>
+template <bool GATEUP, int SUB, int STAGES, bool SAVE = false>
 struct GemmSwapShape {
     static constexpr int W_BYTES = 128 * GG_BK * 2;  // this CTA's 128 weight rows of one K block
     static constexpr int X_BYTES = 128 * GG_BK * 2;  // room for this CTA's share of the token rows (<= 128)
@@ -59,8 +59,9 @@ struct GemmSwapShape {
     static constexpr int TMEM_COLS = 512;
     static constexpr int BAR_BYTES = 256;
     static constexpr int TABLE_BYTES = (2 * (GG_MAX_GROUPS + 1) * 4 + 127) / 128 * 128;
-    // 4 x two 2 KB staging blocks (down); gate|up: two storing warps' staging blocks + two 4 KB hand-off buffers
-    static constexpr int EPI_BYTES = 4 * 2 * 2048;
+    // 4 x two 2 KB staging blocks (down); gate|up: two storing warps' staging blocks + two 4 KB hand-off buffers;
+    // SAVE: one more 2 KB block per epilogue warp for the pre-activations
+    static constexpr int EPI_BYTES = 4 * 2 * 2048 + (SAVE ? 4 * 2048 : 0);
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + TABLE_BYTES;
     static_assert(SUB_BYTES % 1024 == 0, "sub-block bases stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -237,13 +238,18 @@ __device__ __forceinline__ int swap_box_index(int half) {
 // four of the CTA's rows per K block with one TMA gather4 into the places a tile box would fill, so the MMA and
 // the epilogue are unchanged and no permuted copy of x is written.
 // COMBINE (down only): after each tile, the weighted combine of the tokens completed by it (CombineArgs).
-template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false, bool GATHER = false, bool COMBINE = false>
+// SAVE (gate|up with SwiGLU): h as usual, and the pre-activations g | u into args.out2 [M][2f] (gate in columns
+// [0, f), up in [f, 2f); tmG its map), the values the RAW mode stores: the gate warps store theirs after handing
+// them off, the up warps theirs before computing h. A training forward keeps them for the backward pass.
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false, bool GATHER = false, bool COMBINE = false,
+          bool SAVE = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ SwapMaps tmX,
-                             const __grid_constant__ CUtensorMap tmO, const GemmArgs args, int weights_streamed_once,
-                             const __grid_constant__ CombineArgs cargs) {
+                             const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmG,
+                             const GemmArgs args, int weights_streamed_once, const __grid_constant__ CombineArgs cargs) {
     static_assert(!COMBINE || !GATEUP, "the combine follows the down projection");
-    using S = GemmSwapShape<GATEUP, SUB, STAGES>;
+    static_assert(!SAVE || (GATEUP && !RAW), "saved pre-activations come with the SwiGLU epilogue");
+    using S = GemmSwapShape<GATEUP, SUB, STAGES, SAVE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* stages = smem;
@@ -524,6 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
         const int p = q & 1;  // hand-off pair (gate|up)
         uint8_t* xbuf = epi + 8192 + p * 4096;
         uint8_t* stage_base = epi + ((GATEUP && !RAW) ? p : (warp - 2)) * 4096;
+        uint8_t* save_buf = epi + 16384 + p * 4096 + (ferry ? 0 : 2048);  // SAVE: g (gate warps) or u
         // output row stride and this warp's column limit: RAW gate|up stores gate rows below f, up rows from f on
         const int ld_out = RAW ? 2 * args.f : args.n_out;
         const int col_off = (RAW && q >= 2) ? args.f : 0;
@@ -562,6 +569,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                             *reinterpret_cast<uint4*>(xbuf + lane * 128 + ((u ^ (lane & 7)) << 4)) =
                                 make_uint4(raw[4 * u], raw[4 * u + 1], raw[4 * u + 2], raw[4 * u + 3]);
                         mbar_arrive(&xfull_bar[p]);
+                        if constexpr (SAVE) {  // g of this warp's 32 columns (single buffer: one group per block)
+#pragma unroll
+                            for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(raw[t]);
+                            if (lane == 0) bulk_wait_group_read<0>();
+                            __syncwarp();
+                            stage_transposed(save_buf, v, lane);
+                            flush_staged_block(save_buf, lane, &tmG, args.out2, 2 * args.f, r0 + c0, row_end, col0,
+                                               args.f);
+                        }
                         ++blocks;
                         continue;
                     }
@@ -578,6 +594,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                         gt[4 * u + 3] = w4.w;
                     }
                     mbar_arrive(&xempty_bar[p]);
+                    if constexpr (SAVE) {  // u of these columns; groups per block: u, then h
+#pragma unroll
+                        for (int t = 0; t < 32; ++t) v[t] = __uint_as_float(raw[t]);
+                        if (lane == 0) bulk_wait_group_read<1>();  // the previous block's u store (h after it)
+                        __syncwarp();
+                        stage_transposed(save_buf, v, lane);
+                        flush_staged_block(save_buf, lane, &tmG, args.out2, 2 * args.f, r0 + c0, row_end,
+                                           args.f + col0, 2 * args.f);
+                    }
 #pragma unroll
                     for (int t = 0; t < 32; ++t) v[t] = swiglu(__uint_as_float(gt[t]), __uint_as_float(raw[t]));
                 } else {
@@ -586,7 +611,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GS_THREADS, 1)
                 }
                 uint8_t* my_stage = stage_base + (int)(blocks & 1u) * 2048;
                 ++blocks;
-                if (lane == 0) bulk_wait_group_read<1>();  // the TMA store that last read this buffer is done
+                // the TMA store that last read this buffer is done (SAVE: two blocks back, three groups since)
+                if (lane == 0) bulk_wait_group_read<SAVE ? 3 : 1>();
                 __syncwarp();
                 stage_transposed(my_stage, v, lane);
                 flush_staged_block(my_stage, lane, &tmO, args.out, ld_out, r0 + c0, row_end, col0, col_end);

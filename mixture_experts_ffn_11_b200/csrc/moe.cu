@@ -140,6 +140,12 @@ cudaError_t set_gemm_attributes() {
         e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, false, false, true>, a, SwapGU::SMEM_BYTES);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true, false, true>, a, SwapGU::SMEM_BYTES);
+    if (e == cudaSuccess)  // pre-activations saved beside h
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, false, false, false, false, true>, a,
+                                 GemmSwapShape<true, 2, 3, true>::SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<true, 2, 3, true, false, false, false, true>, a,
+                                 GemmSwapShape<true, 2, 3, true>::SMEM_BYTES);
     if (e == cudaSuccess)  // combine in the epilogue
         e = cudaFuncSetAttribute(grouped_gemm_swap_kernel<false, 2, 3, false, false, false, true>, a,
                                  SwapDN::SMEM_BYTES);
@@ -263,6 +269,7 @@ struct GemmProblem {
     void* out;
     const int32_t* row_src = nullptr;  // gathering gate|up: A row r is row row_src[r] of a [src_rows][K] tensor
     int src_rows = 0;
+    void* out2 = nullptr;  // gate|up saving its pre-activations [M][2f]
 };
 
 // Tensor maps: A [M][K] in 128-row x 64 boxes; B slabs [G][rows][K] (rows = 2f for gate|up, n_out for
@@ -300,6 +307,7 @@ GemmArgs gemm_args(const GemmProblem& p, int out_cols) {
     args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
     args.row_src = p.row_src;
     args.src_rows = p.src_rows;
+    args.out2 = reinterpret_cast<__nv_bfloat16*>(p.out2);
     return args;
 }
 
@@ -349,10 +357,11 @@ moe_status_t launch_wide(const GemmProblem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup (wide pair)" : "grouped_gemm_down (wide pair)", e);
 }
 
-template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false, bool GATHER = false, bool COMBINE = false>
+template <bool GATEUP, int SUB, int STAGES, bool BIGBOX, bool RAW = false, bool GATHER = false, bool COMBINE = false,
+          bool SAVE = false>
 moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream, const CombineArgs& ca = CombineArgs()) {
-    using S = GemmSwapShape<GATEUP, SUB, STAGES>;
-    CUtensorMap tw, to;
+    using S = GemmSwapShape<GATEUP, SUB, STAGES, SAVE>;
+    CUtensorMap tw, to, tg;
     SwapMaps tx;
     moe_status_t st;
     const cuuint64_t K = (cuuint64_t)p.K, f = (cuuint64_t)p.f, G = (cuuint64_t)p.G, n_out = (cuuint64_t)p.n_out;
@@ -411,12 +420,19 @@ moe_status_t launch_swap(const GemmProblem& p, int sms, cudaStream_t stream, con
         }
     }
     if (st != MOE_OK) return st;
+    tg = to;
+    if (SAVE) {  // [M][2f] pre-activations
+        GemmProblem q = p;
+        q.n_out = 2 * p.f;
+        q.out = p.out2;
+        if ((st = make_out_map(q, &tg)) != MOE_OK) return st;
+    }
     const GemmArgs args = gemm_args(p, S::TILE_W);
     const long upper = ((long)p.M / GS_MAX_N + p.G) * (long)args.n_tiles;  // >= the real tile count
     const int clusters = (int)(upper < sms / 2 ? upper : sms / 2);
     const int streamed_once = (long)p.M <= (long)p.G * GS_MAX_N ? 1 : 0;
-    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX, RAW, GATHER, COMBINE>,
-                                     dim3(2 * clusters), dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, args,
+    const cudaError_t e = launch_pdl(grouped_gemm_swap_kernel<GATEUP, SUB, STAGES, BIGBOX, RAW, GATHER, COMBINE, SAVE>,
+                                     dim3(2 * clusters), dim3(GS_THREADS), S::SMEM_BYTES, stream, tw, tx, to, tg, args,
                                      streamed_once, ca);
     return check_launch(RAW ? "grouped_gemm_gateup_preact (swap pair)"
                             : (GATEUP ? "grouped_gemm_gateup (swap pair)"
@@ -1093,6 +1109,28 @@ moe_status_t moe_grouped_gemm_gateup_preact(const moe_bf16_t* a, const moe_bf16_
     const GemmProblem p{a, w_gateup, group_offsets, G, M, d, f, f, gu};
     if (d % GG_BK == 0) return launch_swap<true, 2, 3, true, true>(p, di.sms, stream);
     return launch_swap<true, 2, 3, false, true>(p, di.sms, stream);
+}
+
+moe_status_t moe_grouped_gemm_gateup_save(const moe_bf16_t* a, const moe_bf16_t* w_gateup, const int32_t* group_offsets,
+                                          int G, int M, int d, int f, moe_bf16_t* h, moe_bf16_t* gu,
+                                          cudaStream_t stream) {
+    moe_status_t st = check_gemm_args(a, w_gateup, group_offsets, G, M, d, f, h);
+    if (st != MOE_OK) return st;
+    if (M > 0 && !gu) return fail(MOE_ERR_INVALID_ARG, "null pointer argument");
+    if (!aligned16(gu)) return fail(MOE_ERR_INVALID_ARG, "gu must be 16-byte aligned");
+    DeviceInfo di;
+    if ((st = device_info(di)) != MOE_OK) return st;
+    if (M == 0) return MOE_OK;
+    if (di.sms < 2) return fail(MOE_ERR_UNSUPPORTED, "the gate|up GEMM with saved pre-activations needs CTA pairs");
+    GemmProblem p{a, w_gateup, group_offsets, G, M, d, f, f, h};
+    if ((long)M >= (long)G * GG_BM) {  // prefill: one kernel writes h and g | u
+        p.out2 = gu;
+        if (d % GG_BK == 0) return launch_swap<true, 2, 3, true, false, false, false, true>(p, di.sms, stream);
+        return launch_swap<true, 2, 3, false, false, false, false, true>(p, di.sms, stream);
+    }
+    // a few rows per expert: h as moe_grouped_gemm_gateup, then the pre-activation GEMM
+    if ((st = launch_grouped_gemm(p, true, di.sms, stream)) != MOE_OK) return st;
+    return moe_grouped_gemm_gateup_preact(a, w_gateup, group_offsets, G, M, d, f, gu, stream);
 }
 
 moe_status_t moe_swiglu_backward(const moe_bf16_t* dh, const moe_bf16_t* gu, int M, int f, moe_bf16_t* dgu,

@@ -122,8 +122,11 @@ class MoEFFN:
         self.buf, self._T = b, T
         return b
 
-    def forward(self, x, stream=None, timing=None):
+    def forward(self, x, stream=None, timing=None, train: bool = False):
         """y = MoE(x) for x [T, d] bf16 on the GPU. Returns the layer's output buffer [T, d] (bf16).
+
+        train: keep the routed experts' gate|up pre-activations (moe_grouped_gemm_gateup_save, bf16 weights) so
+        that the following backward() does not recompute them; the output is the same.
 
         timing: optional dict; if given, a (start, end) pair of CUDA events is recorded around each stage
         ("route", "permute", "gateup", "down", "combine" on the layer's stream; "shared", the always-on
@@ -164,7 +167,9 @@ class MoEFFN:
         else:
             N.route_topk(x, self.w_router, self.bias, self.k, self.route, b["logits"], b["topk_idx"], b["topk_w"], s)
         mark("route", False)
-        fused = self._fused(T)
+        fused = self._fused(T) and not train  # the saving gate|up GEMM reads x_perm
+        save = train and self.weights == "bf16"
+        self._gu_saved = False
         mark("permute", True)
         if fused:  # grouping only; the gate|up GEMM gathers its rows from x
             N.permute(None, b["topk_idx"], self.E, b["counts"], b["offsets"], b["perm_src"], b["inv_perm"], None,
@@ -180,6 +185,9 @@ class MoEFFN:
         mark("gateup", True)
         if fused:
             N.grouped_gemm_gateup_gather(x, b["perm_src"], self.w_gateup, b["offsets"], b["h"], None, s)
+        elif save:
+            N.grouped_gemm_gateup_save(b["x_perm"], self.w_gateup, b["offsets"], b["h"], self._grad_buffers(T)["gu"], s)
+            self._gu_saved = True
         else:
             self._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)
         mark("gateup", False)
@@ -312,7 +320,8 @@ class MoEFFN:
         if not self._x_perm_valid:  # the forward gathered its rows inside the GEMM: x_perm is made here
             N.gather_rows(x, b["perm_src"], b["x_perm"], s)
             self._x_perm_valid = True
-        N.grouped_gemm_gateup_preact(b["x_perm"], self.w_gateup, b["offsets"], g["gu"], s)
+        if not getattr(self, "_gu_saved", False):  # a training forward kept them
+            N.grouped_gemm_gateup_preact(b["x_perm"], self.w_gateup, b["offsets"], g["gu"], s)
         mark("bwd_preact", False)
         mark("bwd_swiglu", True)
         N.swiglu_backward(g["dh"], g["gu"], g["dgu"], s)
@@ -356,25 +365,33 @@ class MoEFFN:
                 out["dw_down_shared"], out["dw_gateup_shared"] = g["dw_down_shared"], g["dw_gateup_shared"]
         return out
 
-    def backward_kernel_launches(self, T: int, weight_grads: bool = True) -> int:
-        """Kernels one backward() launches: permute-backward 1, dh 1, pre-activations 1 (+ 1 gather of x_perm
-        after a forward that folded it into the gate|up GEMM), SwiGLU-backward 1, dx_perm 1, router 5, combine 1,
-        and per weight gradient 4 (padded offsets, two transposes, the GEMM); the shared expert 4 more (+ 8 with
-        weight gradients)."""
+    def backward_kernel_launches(self, T: int, weight_grads: bool = True, train_forward: bool = False) -> int:
+        """Kernels one backward() launches: permute-backward 1, dh 1, pre-activations 1 (none after a training
+        forward, which kept them; + 1 gather of x_perm after a forward that folded it into the gate|up GEMM),
+        SwiGLU-backward 1, dx_perm 1, router 5, combine 1, and per weight gradient 4 (padded offsets, two
+        transposes, the GEMM); the shared expert 4 more (+ 8 with weight gradients)."""
         if T <= 0:
             return 0
-        n = 11 + (8 if weight_grads else 0) + (1 if self._fused(T) else 0)
+        n = 11 + (8 if weight_grads else 0)
+        if train_forward:
+            n -= 1
+        elif self._fused(T):
+            n += 1
         if self.shared_f:
             n += 4 + (8 if weight_grads else 0)
         return n
 
-    def kernel_launches(self, T: int) -> int:
+    def kernel_launches(self, T: int, train: bool = False) -> int:
         """Kernels one forward() launches (mirrors the library's dispatch): the router is one kernel when the
         tensor-core path with fused top-k is taken (E <= 128, T >= 2048), else logits + top-k;
-        permute 4, gate|up, down, combine 1 each (fused: permute 3, gate|up 1, down with combine 1); the shared
+        permute 4, gate|up, down, combine 1 each (fused: permute 3, gate|up 1, down with combine 1; train: the
+        gate|up that keeps its pre-activations is 1 kernel with 128 rows or more per expert, else 2); the shared
         expert 2 more."""
         if T <= 0:
             return 0
         route = 1 if (self.E <= 128 and T >= 2048) else 2
-        body = 3 + 2 if self._fused(T) else 4 + 3
+        if train and self.weights == "bf16":
+            body = 4 + 3 + (0 if T * self.k >= 128 * self.E else 1)
+        else:
+            body = 3 + 2 if self._fused(T) else 4 + 3
         return route + body + (2 if self.shared_f else 0)

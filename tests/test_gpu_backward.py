@@ -128,6 +128,31 @@ def test_grouped_weight_grad_matches_fp64(counts, P, Q):
 
 # ---- the layer ---------------------------------------------------------------------------------------------
 
+@pytest.mark.parametrize("counts,d,f", [([0, 1, 127, 300, 45, 0], 200, 136), ([447, 569, 0, 512], 2880, 2880),
+                                         ([3, 0, 5, 2], 256, 128)],
+                         ids=["ragged_small", "gpt_oss_width", "few_rows_two_calls"])
+def test_gateup_save_equals_gateup_and_preact(counts, d, f):
+    """The training forward's gate|up GEMM: h bit-identical to moe_grouped_gemm_gateup and the kept
+    pre-activations bit-identical to moe_grouped_gemm_gateup_preact (one kernel on the prefill path, the two
+    calls below 128 rows per group)."""
+    offs, _ = _ragged(counts, 0)
+    M, G = int(offs[-1]), len(counts)
+    a = to_dev_bf16(synth.normal_bf16(23, 0, 0, M * d, 1.0).reshape(M, d))
+    w = to_dev_bf16(synth.normal_bf16(23, 2, 0, G * 2 * f * d, 0.05).reshape(G, 2 * f, d))
+    o = torch.from_numpy(offs).cuda()
+    h_ref = torch.empty(M, f, dtype=torch.bfloat16, device="cuda")
+    gu_ref = torch.empty(M, 2 * f, dtype=torch.bfloat16, device="cuda")
+    N.grouped_gemm_gateup(a, w, o, h_ref)
+    N.grouped_gemm_gateup_preact(a, w, o, gu_ref)
+    h = torch.full((M, f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gu = torch.full((M, 2 * f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    N.grouped_gemm_gateup_save(a, w, o, h, gu)
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
+    assert torch.equal(h.view(torch.int16), h_ref.view(torch.int16))
+    assert torch.equal(gu.view(torch.int16), gu_ref.view(torch.int16))
+
+
 def _layer_and_grads(wl):
     inp = synth.device_inputs(wl)
     layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
@@ -202,3 +227,28 @@ def test_layer_backward_gpt_oss_sampled():
         r_gu, c_gu = rng.integers(0, 2 * wl.f, 48), rng.integers(0, wl.d, 48)
         want = oracle.weight_grad_entries(ref.x, gu_e, dn_e, e, ref.idx, ref.w, dy, "gateup", r_gu, c_gu)
         check_close(out["dw_gateup"][e].cpu().numpy()[r_gu, c_gu], want, f"dW_gateup entries, expert {e}")
+
+
+@pytest.mark.parametrize("name,over", [("gpt-oss-20b-prefill", {"T": 1024}), TINY[2]],
+                         ids=["gpt_oss_T1024", "tiny_sigmoid_bias_shared"])
+def test_training_forward_keeps_preactivations(name, over):
+    """forward(train=True) gives the same output, and the backward after it (no pre-activation recompute) the
+    same gradients, bit for bit, as forward() + backward()."""
+    wl = synth.workload(name, **over)
+    inp = synth.device_inputs(wl)
+    args = (inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"], inp["w_gateup_shared"],
+            inp["w_down_shared"])
+    a, b = MoEFFN(*args), MoEFFN(*args)
+    dy = to_dev_bf16(synth.dy_host(wl))
+    ya = a(inp["x"]).clone()
+    ga = {k: v.clone() for k, v in a.backward(dy).items() if v is not None}
+    yb = b.forward(inp["x"], train=True).clone()
+    gb = b.backward(dy)
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
+    assert torch.equal(ya.view(torch.int16), yb.view(torch.int16))
+    for key, v in ga.items():
+        w = gb[key]
+        if v.dtype == torch.bfloat16:
+            v, w = v.view(torch.int16), w.view(torch.int16)
+        assert torch.equal(v, w), key
