@@ -56,8 +56,8 @@ TRAFFIC = {
     ("grouped_gemm_down", "decode-256e-shared", "5eb5b456683cd862"): 6466502144,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
-                  ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "sm100.cuh", "common.cuh",
-                   "moe.cu")]
+                  ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "gemm_fp4.cuh", "gemm_fp4_mma.cuh",
+                   "sm100.cuh", "common.cuh", "moe.cu")]
 
 
 def kernel_source_hash() -> str:
