@@ -46,14 +46,16 @@ L2_FLUSH_BYTES = 256 << 20
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:grouped_gemm -s 4 -c 1
 #       python bench.py --kernel K --workload W --steps 2 --warmup 3
 TRAFFIC = {
-    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "5eb5b456683cd862"): 1247501824,
-    ("grouped_gemm_down", "gpt-oss-20b-prefill", "5eb5b456683cd862"): 710778112,
-    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "5eb5b456683cd862"): 2479206400,
-    ("grouped_gemm_down", "mixtral-8x7b-prefill", "5eb5b456683cd862"): 2457910272,
-    ("grouped_gemm_gateup", "zipf-128e", "5eb5b456683cd862"): 1605244928,
-    ("grouped_gemm_down", "zipf-128e", "5eb5b456683cd862"): 1082768384,
-    ("grouped_gemm_gateup", "decode-256e-shared", "5eb5b456683cd862"): 12929945344,
-    ("grouped_gemm_down", "decode-256e-shared", "5eb5b456683cd862"): 6466502144,
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "2fb30f955d264793"): 1249031168,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "2fb30f955d264793"): 713447168,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "2fb30f955d264793"): 3102232064,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "2fb30f955d264793"): 2468814336,
+    ("grouped_gemm_gateup", "zipf-128e", "2fb30f955d264793"): 1642825472,
+    ("grouped_gemm_down", "zipf-128e", "2fb30f955d264793"): 1083206144,
+    ("grouped_gemm_gateup", "decode-256e-shared", "2fb30f955d264793"): 12930168064,
+    ("grouped_gemm_down", "decode-256e-shared", "2fb30f955d264793"): 6467443200,
+    ("grouped_gemm_gateup", "decode-256e-shared-mxfp4", "2fb30f955d264793"): 3543669248,
+    ("grouped_gemm_down", "decode-256e-shared-mxfp4", "2fb30f955d264793"): 1724605184,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "gemm_fp4.cuh", "gemm_fp4_mma.cuh",
