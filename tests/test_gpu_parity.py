@@ -491,6 +491,12 @@ MXFP4_RAGGED = [
     ("nt32_ragged", [20, 0, 31, 33, 1, 40], 160, 224),
     ("nt64_one_group", [200], 352, 160),
     ("nt64_many", [0, 65, 64, 130, 7], 512, 544),
+    # the warp-MMA decode kernel at its limits: 1024 groups (group tables sized by G), K = 8192 (the whole token
+    # rows of a tile in shared memory, a 2-stage ring), and K = 8224 just past it (gate|up on the tensor-memory
+    # kernel, down on the warp kernel)
+    ("warp_1024_groups", [2] * 1024, 64, 64),
+    ("warp_k_8192", [3, 5, 0, 2], 8192, 64),
+    ("past_warp_k_limit", [3, 5, 0, 2], 8224, 64),
 ]
 
 
