@@ -46,16 +46,16 @@ L2_FLUSH_BYTES = 256 << 20
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:grouped_gemm -s 4 -c 1
 #       python bench.py --kernel K --workload W --steps 2 --warmup 3
 TRAFFIC = {
-    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "c98e5aef4dbe2c18"): 1249221376,
-    ("grouped_gemm_down", "gpt-oss-20b-prefill", "c98e5aef4dbe2c18"): 712037888,
-    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "c98e5aef4dbe2c18"): 2894431488,
-    ("grouped_gemm_down", "mixtral-8x7b-prefill", "c98e5aef4dbe2c18"): 2459405312,
-    ("grouped_gemm_gateup", "zipf-128e", "c98e5aef4dbe2c18"): 1602299904,
-    ("grouped_gemm_down", "zipf-128e", "c98e5aef4dbe2c18"): 1085322496,
-    ("grouped_gemm_gateup", "decode-256e-shared", "c98e5aef4dbe2c18"): 12929968896,
-    ("grouped_gemm_down", "decode-256e-shared", "c98e5aef4dbe2c18"): 6468377344,
-    ("grouped_gemm_gateup", "decode-256e-shared-mxfp4", "c98e5aef4dbe2c18"): 3543465472,
-    ("grouped_gemm_down", "decode-256e-shared-mxfp4", "c98e5aef4dbe2c18"): 1724120320,
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "478dde139e27b6a8"): 1248200960,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "478dde139e27b6a8"): 713675520,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "478dde139e27b6a8"): 2494269440,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "478dde139e27b6a8"): 2458328576,
+    ("grouped_gemm_gateup", "zipf-128e", "478dde139e27b6a8"): 1598989056,
+    ("grouped_gemm_down", "zipf-128e", "478dde139e27b6a8"): 1084371200,
+    ("grouped_gemm_gateup", "decode-256e-shared", "478dde139e27b6a8"): 12932950272,
+    ("grouped_gemm_down", "decode-256e-shared", "478dde139e27b6a8"): 6466513664,
+    ("grouped_gemm_gateup", "decode-256e-shared-mxfp4", "478dde139e27b6a8"): 3544724224,
+    ("grouped_gemm_down", "decode-256e-shared-mxfp4", "478dde139e27b6a8"): 1723772928,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "gemm_fp4.cuh", "gemm_fp4_mma.cuh",

@@ -87,10 +87,16 @@ struct GemmFp4WarpShape {
     }
 };
 
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-    uint32_t d;
-    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(d) : "r"(byte));
-    return d;
+// the four code pairs of a 32-bit word as four f16 pairs (bytes 0..3 in order): the hardware's exact E2M1 -> f16
+// conversion, low code to the low half. The bytes come from one unpacking move, which the compiler turns into byte
+// selects of the conversions themselves (measured: gate|up 0.806 -> 0.720 ms, down 0.450 -> 0.402 ms on the decode
+// layer, against a shift in front of every conversion)
+__device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t& o0, uint32_t& o1, uint32_t& o2, uint32_t& o3) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(o0), "=r"(o1), "=r"(o2), "=r"(o3)
+        : "r"(w));
 }
 
 __device__ __forceinline__ void mma_f16_m16n8k16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
@@ -389,10 +395,9 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
                             const uint32_t cb = sc[blk * S::S_BYTES + S::KSPL * i * S::BM + rb];
                             const float sa = S::SCALE_LUT ? scale_lut[ca] : e8m0_to_f32(ca);
                             const float sb = S::SCALE_LUT ? scale_lut[cb] : e8m0_to_f32(cb);
-                            const uint32_t a0[4] = {e2m1x2_to_f16x2(wa), e2m1x2_to_f16x2(wbv), e2m1x2_to_f16x2(wa >> 8),
-                                                    e2m1x2_to_f16x2(wbv >> 8)};
-                            const uint32_t a1[4] = {e2m1x2_to_f16x2(wa >> 16), e2m1x2_to_f16x2(wbv >> 16),
-                                                    e2m1x2_to_f16x2(wa >> 24), e2m1x2_to_f16x2(wbv >> 24)};
+                            uint32_t a0[4], a1[4];
+                            e2m1x8_to_f16x2x4(wa, a0[0], a0[2], a1[0], a1[2]);
+                            e2m1x8_to_f16x2x4(wbv, a0[1], a0[3], a1[1], a1[3]);
                             float d[4] = {0.f, 0.f, 0.f, 0.f};
                             mma_f16_m16n8k16(d, a0, xv.x, xv.y);
                             mma_f16_m16n8k16(d, a1, xv.z, xv.w);
