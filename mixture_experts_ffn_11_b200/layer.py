@@ -84,6 +84,7 @@ class MoEFFN:
         and side stream, so that two calls can be in flight at once."""
         twin = copy.copy(self)
         twin.buf, twin._T = {}, None
+        twin._gbuf, twin._gT, twin._gu_saved = None, None, False  # its own backward buffers too
         twin._side = torch.cuda.Stream(self.device) if self.shared_f else None
         return twin
 
