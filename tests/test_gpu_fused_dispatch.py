@@ -246,3 +246,26 @@ def test_fused_layer_bitwise_equals_separate(name, over):
     for key, v in g0.items():
         assert torch.equal(v.view(torch.int16) if v.dtype == torch.bfloat16 else v, g1[key].view(torch.int16)
                            if g1[key].dtype == torch.bfloat16 else g1[key]), key
+
+
+def test_empty_problems_launch_nothing():
+    """Zero rows: the gathering, combining and saving GEMMs and the row gather return at once (no launch, no
+    device error), as the other entry points do."""
+    dev = "cuda"
+    bf = torch.bfloat16
+    x = torch.empty(0, 64, dtype=bf, device=dev)
+    w = torch.zeros(2, 128, 64, dtype=bf, device=dev)
+    wd = torch.zeros(2, 64, 64, dtype=bf, device=dev)
+    off = torch.zeros(3, dtype=torch.int32, device=dev)
+    src = torch.empty(0, dtype=torch.int32, device=dev)
+    h = torch.empty(0, 64, dtype=bf, device=dev)
+    gu = torch.empty(0, 128, dtype=bf, device=dev)
+    N.grouped_gemm_gateup_gather(x, src, w, off, h, None)
+    N.grouped_gemm_gateup_save(x, w, off, h, gu)
+    N.gather_rows(x, src, torch.empty(0, 64, dtype=bf, device=dev))
+    tw = torch.empty(0, 2, dtype=torch.float32, device=dev)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    N.grouped_gemm_down_combine(h, wd, off, src, src, tw, None, torch.empty(0, 64, dtype=bf, device=dev),
+                                torch.empty(0, 64, dtype=bf, device=dev), ws)
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
