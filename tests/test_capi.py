@@ -90,6 +90,14 @@ def test_invalid_arguments_rejected_before_any_launch(native):
         native.MOE_ERR_INVALID_ARG
     assert lib.moe_grouped_gemm_gateup_gather(16, 16, 8, 16, 16, 1, 8, 8, 8, 16, null, 0, null) == \
         native.MOE_ERR_WORKSPACE
+    # down + combine: M != T*k; workspace missing
+    assert lib.moe_grouped_gemm_down_combine(16, 16, 16, 1, 8, 8, 8, 16, 16, 16, null, 3, 2, 16, 16, null, 0,
+                                             null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_down_combine(16, 16, 16, 1, 8, 8, 8, 16, 16, 16, null, 4, 2, 16, 16, null, 0,
+                                             null) == native.MOE_ERR_WORKSPACE
+    # gate|up keeping its pre-activations: no gu buffer; misaligned gu
+    assert lib.moe_grouped_gemm_gateup_save(16, 16, 16, 1, 8, 8, 8, 16, null, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_gateup_save(16, 16, 16, 1, 8, 8, 8, 16, 24, null) == native.MOE_ERR_INVALID_ARG
     # row gather: d not a multiple of 8; misaligned output
     assert lib.moe_gather_rows(16, 16, 4, 12, 4, 16, null) == native.MOE_ERR_INVALID_ARG
     assert lib.moe_gather_rows(16, 16, 4, 8, 4, 24, null) == native.MOE_ERR_INVALID_ARG
