@@ -26,11 +26,15 @@
 // token, block and t, 16 bytes of f16 in the order x0 x2 x4 x6 x1 x3 x5 x7 (x_i = element 32b + 8t + i), one
 // 16-byte load giving the B fragments of both MMAs. (A byte's low code goes to the low half of the f16 pair.)
 //
-// CTA (544 threads, one per SM, persistent over tiles): warps 0-15 compute, warp 16 is the TMA producer.
-// Tile = (group g, block of 8 token rows, run of `wpt` weight blocks of 128 rows; gate|up: 128 gate rows and the
-// matching 128 up rows). Per tile the producer loads the 8 token rows whole (one box per row) and then streams, per
-// weight block, stages of K = 256: codes [128 rows x 128 bytes] (128-byte swizzle) and scales [8 x 128] per
-// projection. Warps 0-7 scale and convert the token rows in place once per tile (warp w takes row w). Warps w and
+// CTA (544 threads, one per SM, persistent over its range of units): warps 0-15 compute, warp 16 is the TMA producer.
+// Work unit = (group g, block of 8 token rows, one weight block: 256 rows for down; 128 gate rows and the matching
+// 128 up rows for gate|up), numbered group by group, token block by token block, weight block by weight block.
+// Every unit streams the same bytes, so CTA b takes the contiguous range [U b / grid, U (b + 1) / grid) of the U
+// units (balanced to one unit whatever U; a fixed tile size left up to half an SM wave idle at the end). A range
+// splits into segments, one per token block it touches (usually two or three), and the token rows are loaded and
+// converted once per segment. Per segment the producer loads the 8 token rows whole (one box per row) and then
+// streams, per weight block, stages of K = 256: codes [128 rows x 128 bytes] (128-byte swizzle) and scales [8 x 128]
+// per projection. Warps 0-7 scale and convert the token rows in place once per segment (warp w takes row w). Warps w and
 // w + 8 compute weight rows 16w .. 16w+15 of each block, w the even and w + 8 the odd 32-element blocks of every
 // stage (four warps per SM sub-partition hide the MMA and load latencies); at the end of a weight block warp w + 8
 // hands its partial sums to warp w through shared memory, which adds them to its own (always in that order) and
@@ -43,7 +47,7 @@
 
 namespace moe {
 
-constexpr int FW_NT = 8;                      // token rows per tile (the MMA's N)
+constexpr int FW_NT = 8;                      // token rows per token block (the MMA's N)
 constexpr int FW_WARPS = 16;                  // compute warps
 constexpr int FW_THREADS = (FW_WARPS + 1) * 32;
 constexpr int FW_KS = GF_KS;                  // K per stage: 256 (128 bytes of codes per row)
@@ -138,7 +142,7 @@ template <bool GATEUP>
 __global__ void __launch_bounds__(FW_THREADS, 1)
     grouped_gemm_fp4_warp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ,
                                  const __grid_constant__ CUtensorMap tmS, const GemmArgs args,
-                                 int weights_streamed_once, int stages_n, int wpt) {
+                                 int weights_streamed_once, int stages_n) {
     using S = GemmFp4WarpShape<GATEUP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -150,7 +154,7 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
     uint64_t* empty_bar = full_bar + 8;
     uint64_t* bfull_bar = empty_bar + 8;
     uint64_t* bempty_bar = bfull_bar + 1;
-    uint64_t* bconv_bar = bempty_bar + 1;  // every token row of the tile converted
+    uint64_t* bconv_bar = bempty_bar + 1;  // every token row of the segment converted
     uint64_t* red_full = bconv_bar + 1;  // [8] (two warps per rows) partial sums of warp w + RW are in red[w]
     uint64_t* red_empty = red_full + 8;  // [8] red[w] has been read
     volatile int* abort_flag = reinterpret_cast<volatile int*>(red_empty + 8);
@@ -166,7 +170,6 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
     const int KB32 = K / 32;                    // scale blocks per row
     const int KS = (K + FW_KS - 1) / FW_KS;     // stages per weight block
     const int wblocks = args.n_tiles;           // weight blocks of S::BM output columns
-    const int wchunks = (wblocks + wpt - 1) / wpt;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages_n; ++s) {
@@ -200,14 +203,14 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         s_off[g] = v;
     }
     __syncthreads();
-    if (warp == 0) {  // tile prefix over groups: tiles(g) = ceil(rows / 8) * wchunks
+    if (warp == 0) {  // unit prefix over groups: units(g) = ceil(rows / 8) * wblocks
         const int per = (G + 31) / 32;
         const int g0 = lane * per, g1 = min(g0 + per, G);
         int local = 0;
         for (int g = g0; g < g1; ++g) {
             const int rows = s_off[g + 1] - s_off[g];
             if (rows < 0) flag_error(MOE_DEVERR_GROUP_RANGE);
-            local += (max(rows, 0) + FW_NT - 1) / FW_NT * wchunks;
+            local += (max(rows, 0) + FW_NT - 1) / FW_NT * wblocks;
         }
         int incl = local;
 #pragma unroll
@@ -218,27 +221,31 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         int run = incl - local;
         for (int g = g0; g < g1; ++g) {
             s_tp[g] = run;
-            run += (max(s_off[g + 1] - s_off[g], 0) + FW_NT - 1) / FW_NT * wchunks;
+            run += (max(s_off[g + 1] - s_off[g], 0) + FW_NT - 1) / FW_NT * wblocks;
         }
         if (lane == 31) s_tp[G] = incl;
     }
     __syncthreads();
     const int total = s_tp[G];
+    const int u_begin = (int)((long)total * blockIdx.x / gridDim.x);
+    const int u_end = (int)((long)total * (blockIdx.x + 1) / gridDim.x);
 
-    // tile -> group g, token block tb, weight chunk wc (tiles of one group: token block major, then weight chunk)
-    auto locate = [&](int tile, int& g, int& tb, int& wc) {
+    // the segment that starts at unit u: group g, token block tb, weight blocks [wb0, wb1) (up to the end of the
+    // token block or of this CTA's range)
+    auto segment = [&](int u, int& g, int& tb, int& wb0, int& wb1) {
         int lo = 0, hi = G - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (s_tp[mid] <= tile)
+            if (s_tp[mid] <= u)
                 lo = mid;
             else
                 hi = mid - 1;
         }
         g = lo;
-        const int local = tile - s_tp[g];
-        tb = local / wchunks;
-        wc = local - tb * wchunks;
+        const int local = u - s_tp[g];
+        tb = local / wblocks;
+        wb0 = local - tb * wblocks;
+        wb1 = min(wblocks, wb0 + (u_end - u));
     };
 
     if (warp == FW_WARPS) {
@@ -249,12 +256,12 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         uint32_t phase = 0, bphase = 0;
         long issued = 0;
         bool ok = true;
-        int tiles_done = 0;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++tiles_done) {
-            int g, tb, wc;
-            locate(tile, g, tb, wc);
+        int segs_done = 0;
+        int g, tb, wb0, wb1;
+        for (int u = u_begin; u < u_end && ok; u += wb1 - wb0) {
+            segment(u, g, tb, wb0, wb1);
             const int row0 = s_off[g] + tb * FW_NT;
-            // the token rows: after the compute warps are done with the previous tile's
+            // the token rows: after the compute warps are done with the previous segment's
             if (lane == 0) {
                 ok = mbar_wait_bounded(bempty_bar, bphase ^ 1u, abort_flag);
                 if (ok) {
@@ -266,8 +273,8 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
             bphase ^= 1u;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
-            const int wb_end = min(wblocks, (wc + 1) * wpt);
-            for (int wb = wc * wpt; wb < wb_end && ok; ++wb) {
+            ++segs_done;  // its token rows are in flight (drained below even if a later wait gives up)
+            for (int wb = wb0; wb < wb1 && ok; ++wb) {
                 const int wrow = wb * S::BM;
                 for (int ks = 0; ks < KS; ++ks) {
                     if (lane == 0) ok = mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, abort_flag);
@@ -297,7 +304,7 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         if (lane == 0) {
             for (long n = issued > stages_n ? issued - stages_n : 0; n < issued; ++n)
                 mbar_wait_drain(&full_bar[n % stages_n], (uint32_t)((n / stages_n) & 1));
-            if (tiles_done > 0) mbar_wait_drain(bfull_bar, (uint32_t)((tiles_done - 1) & 1));
+            if (segs_done > 0) mbar_wait_drain(bfull_bar, (uint32_t)((segs_done - 1) & 1));
         }
         __syncwarp();
     } else {
@@ -314,9 +321,9 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
         int stage = 0;
         uint32_t phase = 0, bphase = 0, rphase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-            int g, tb, wc;
-            locate(tile, g, tb, wc);
+        int g, tb, wb0, wb1;
+        for (int u = u_begin; u < u_end && ok; u += wb1 - wb0) {
+            segment(u, g, tb, wb0, wb1);
             const int row0 = s_off[g] + tb * FW_NT;
             const int rows = min(FW_NT, s_off[g + 1] - row0);
             if (lane == 0) ok = mbar_wait_bounded(bfull_bar, bphase, abort_flag);
@@ -370,8 +377,7 @@ __global__ void __launch_bounds__(FW_THREADS, 1)
             const int par = gq & 1;
             const uint8_t* bx0 = brows + gq * row_bytes + (((S::KSPL > 1 ? (kw ^ par) : par) * 4 + t) << 4);
             const uint8_t* bx1 = bx0 - (S::KSPL > 1 ? 0 : 2 * par * 64);  // odd i, one warp per rows
-            const int wb_end = min(wblocks, (wc + 1) * wpt);
-            for (int wb = wc * wpt; wb < wb_end && ok; ++wb) {
+            for (int wb = wb0; wb < wb1 && ok; ++wb) {
                 float acc_g[4] = {0.f, 0.f, 0.f, 0.f}, acc_u[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int ks = 0; ks < KS; ++ks) {
                     if (lane == 0) ok = mbar_wait_bounded(&full_bar[stage], phase, abort_flag);

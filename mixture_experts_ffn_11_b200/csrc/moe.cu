@@ -532,7 +532,7 @@ moe_status_t launch_fp4(const Fp4Problem& p, int sms, cudaStream_t stream) {
     return check_launch(GATEUP ? "grouped_gemm_gateup_mxfp4" : "grouped_gemm_down_mxfp4", e);
 }
 
-// Warp-MMA kernel (gemm_fp4_mma.cuh): 8-row token tiles, one weight block per tile.
+// Warp-MMA kernel (gemm_fp4_mma.cuh): 8-row token blocks, an equal share of the units per CTA.
 template <bool GATEUP>
 moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) {
     using S = GemmFp4WarpShape<GATEUP>;
@@ -564,20 +564,13 @@ moe_status_t launch_fp4_warp(const Fp4Problem& p, int sms, cudaStream_t stream) 
     args.f = p.f;
     args.n_tiles = (p.n_out + S::BM - 1) / S::BM;
     args.out = reinterpret_cast<__nv_bfloat16*>(p.out);
-    // weight blocks per tile: the token rows are loaded and converted once per tile, so a tile should stream
-    // several times their bytes (down: 278 KB of codes per 256-row block at d = 7168, f = 2048; gate|up about as
-    // much per 128 + 128-row block and 3.5x the K); fewer blocks per tile when that would leave fewer than 8
-    // tiles per SM
-    int wpt = 4;
-    // token blocks: at least one per non-empty group, and M / 8 in all
-    const long token_blocks = std::max<long>(std::min<long>(p.G, p.M), (p.M + FW_NT - 1) / FW_NT);
-    while (wpt > 1 && token_blocks * ((args.n_tiles + wpt - 1) / wpt) < 8L * sms) wpt >>= 1;
-    const long upper = ((long)p.M / FW_NT + p.G) * (long)((args.n_tiles + wpt - 1) / wpt);  // >= the tile count
+    // one CTA per SM, each with an equal share of the (token block, weight block) units
+    const long upper = ((long)p.M / FW_NT + p.G) * (long)args.n_tiles;  // >= the unit count
     const int grid = (int)(upper < sms ? upper : sms);
     const int streamed_once = (long)p.M <= (long)p.G * FW_NT ? 1 : 0;
     const cudaError_t e = launch_pdl(grouped_gemm_fp4_warp_kernel<GATEUP>, dim3(grid), dim3(FW_THREADS),
                                      (size_t)S::smem_bytes(p.K, stages, p.G), stream, tx, tq, ts, args, streamed_once,
-                                     stages, wpt);
+                                     stages);
     return check_launch(GATEUP ? "grouped_gemm_gateup_mxfp4 (warp MMA)" : "grouped_gemm_down_mxfp4 (warp MMA)", e);
 }
 
