@@ -216,12 +216,15 @@ def weight_bytes(wl) -> float:
     return 0.5 + 1.0 / 32 if wl.weights == "mxfp4" else 2.0
 
 
-def gemm_figures(wl, counts):
-    """Algorithmic FLOPs and DRAM bytes per launch of the two grouped GEMMs, from the realised routing."""
+def gemm_figures(wl, counts, folded_shared=False):
+    """Algorithmic FLOPs and DRAM bytes per launch of the two grouped GEMMs, from the realised routing; with
+    folded_shared the launches also compute the shared expert (as wide as a routed one) as one more group of T
+    rows."""
     R, d, f, wb = wl.R, wl.d, wl.f, weight_bytes(wl)
     active = int((counts > 0).sum())
-    gateup = {"flop": 4.0 * R * d * f, "bytes": active * 2 * f * d * wb + R * d * 2 + R * f * 2}
-    down = {"flop": 2.0 * R * f * d, "bytes": active * d * f * wb + R * f * 2 + R * d * 2}
+    groups, rows = active + (1 if folded_shared else 0), R + (wl.T if folded_shared else 0)
+    gateup = {"flop": 4.0 * rows * d * f, "bytes": groups * 2 * f * d * wb + rows * d * 2 + rows * f * 2}
+    down = {"flop": 2.0 * rows * f * d, "bytes": groups * d * f * wb + rows * f * 2 + rows * d * 2}
     return active, gateup, down
 
 
@@ -411,9 +414,9 @@ def run_kernel(args):
         launch = lambda: N.grouped_gemm_gateup_gather(inp["x"], b["perm_src"], layer.w_gateup, b["offsets"],  # noqa
                                                       b["h"], None, s)
     elif args.kernel == "gateup":
-        launch = lambda: layer._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)  # noqa: E731
+        launch = lambda: layer.routed_gateup(b, s)  # noqa: E731
     else:
-        launch = lambda: layer._down(b["h"], "routed", b["offsets"], b["y_perm"], s)  # noqa: E731
+        launch = lambda: layer.routed_down(b, s)  # noqa: E731
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -429,7 +432,7 @@ def run_kernel(args):
         raise SystemExit("device error word set")
     ms = statistics.mean(a.elapsed_time(c) for a, c in ev)
     counts = b["counts"].cpu().numpy()
-    active, fig_gu, fig_dn = gemm_figures(wl, counts)
+    active, fig_gu, fig_dn = gemm_figures(wl, counts, layer._fold(wl.T))
     peaks, src = load_peaks()
     fig = fig_gu if args.kernel == "gateup" else fig_dn
     roof = roofline_entry(f"grouped_gemm_{args.kernel}", fig, ms, peaks, "bf16_tflops", None)
@@ -579,7 +582,7 @@ def run_ours(args):
     clocks = sampler.summary(t0, t1)
 
     counts = layer.buf["counts"].cpu().numpy()
-    active, fig_gu, fig_dn = gemm_figures(wl, counts)
+    active, fig_gu, fig_dn = gemm_figures(wl, counts, layer._fold(wl.T))
     peaks, peak_src = load_peaks()
     peak_kind = "bf16_tflops_sustained" if total_ms > 1000.0 else "bf16_tflops"
     src_hash = kernel_source_hash()

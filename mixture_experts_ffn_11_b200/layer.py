@@ -18,12 +18,17 @@ import torch
 from . import _native as N
 
 
-def _encode_mxfp4(w):
-    """bf16 weights [G, N, K] -> (codes [G, N, K/2], scales [G, K/32, N]) on the weights' device."""
-    G, Nr, K = w.shape
-    q = torch.empty(G, Nr, K // 2, dtype=torch.uint8, device=w.device)
-    s = torch.empty(G, K // 32, Nr, dtype=torch.uint8, device=w.device)
-    N.mxfp4_quantize(w, q, s)
+def _encode_mxfp4(*ws):
+    """bf16 weights [G_i, N, K] (one or more tensors, stacked on dim 0 in the order given) -> (codes
+    [sum G_i, N, K/2], scales [sum G_i, K/32, N]) on the weights' device."""
+    G = sum(w.shape[0] for w in ws)
+    _, Nr, K = ws[0].shape
+    q = torch.empty(G, Nr, K // 2, dtype=torch.uint8, device=ws[0].device)
+    s = torch.empty(G, K // 32, Nr, dtype=torch.uint8, device=ws[0].device)
+    g = 0
+    for w in ws:
+        N.mxfp4_quantize(w, q[g:g + w.shape[0]], s[g:g + w.shape[0]])
+        g += w.shape[0]
     return q, s
 
 
@@ -61,12 +66,26 @@ class MoEFFN:
         self.w_gateup_shared, self.w_down_shared = w_gateup_shared, w_down_shared
         self.shared_f = w_gateup_shared.shape[0] // 2 if w_gateup_shared is not None else 0
         self.device = w_gateup.device
+        # MXFP4 with a shared expert as wide as a routed one: its weights are encoded as group E of the routed
+        # tensors; for decode-sized T (_fold) its T rows (x itself) follow the R routed rows, and the routed GEMM
+        # launches compute it as one more group, spread over every SM like the rest (on its own it is one group of
+        # T rows, which the MXFP4 kernels run on a few SMs: 139 us on the decode layer's side stream, half of it
+        # after the routing and grouping beside it; folded in, it adds 3-4% to the routed GEMMs and the decode
+        # layer takes 1.12 instead of 1.21 ms)
+        self.fold_shared = weights == "mxfp4" and self.shared_f == self.f and self.shared_f > 0
         if weights == "mxfp4":
-            self.mx_gateup = _encode_mxfp4(w_gateup)
-            self.mx_down = _encode_mxfp4(w_down)
-            if self.shared_f:
-                self.mx_gateup_shared = _encode_mxfp4(w_gateup_shared.unsqueeze(0))
-                self.mx_down_shared = _encode_mxfp4(w_down_shared.unsqueeze(0))
+            E = self.E
+            if self.fold_shared:  # the routed and shared names are views of the stacked tensors
+                qg, sg = self.mx_gateup_all = _encode_mxfp4(w_gateup, w_gateup_shared.unsqueeze(0))
+                qd, sd = self.mx_down_all = _encode_mxfp4(w_down, w_down_shared.unsqueeze(0))
+                self.mx_gateup, self.mx_down = (qg[:E], sg[:E]), (qd[:E], sd[:E])
+                self.mx_gateup_shared, self.mx_down_shared = (qg[E:], sg[E:]), (qd[E:], sd[E:])
+            else:
+                self.mx_gateup = _encode_mxfp4(w_gateup)
+                self.mx_down = _encode_mxfp4(w_down)
+                if self.shared_f:
+                    self.mx_gateup_shared = _encode_mxfp4(w_gateup_shared.unsqueeze(0))
+                    self.mx_down_shared = _encode_mxfp4(w_down_shared.unsqueeze(0))
             self.w_gateup = self.w_down = self.w_gateup_shared = self.w_down_shared = None
         self._T = None
         self.buf = {}
@@ -116,7 +135,18 @@ class MoEFFN:
                                       device=dev),
             "y": torch.empty(T, d, dtype=bf, device=dev),
         }
-        if self.shared_f:
+        if self._fold(T):
+            # the R routed rows, then the shared expert's T rows (group E, offsets[E + 1] = R + T); the routed-only
+            # names are views of the first R rows and E + 1 offsets
+            b["offsets_all"] = torch.full((E + 2,), R + T, dtype=i32, device=dev)
+            b["x_perm_all"] = torch.empty(R + T, d, dtype=bf, device=dev)
+            b["h_all"] = torch.empty(R + T, f, dtype=bf, device=dev)
+            b["y_perm_all"] = torch.empty(R + T, d, dtype=bf, device=dev)
+            b["offsets"] = b["offsets_all"][:E + 1]
+            b["x_perm"], b["h"], b["y_perm"] = b["x_perm_all"][:R], b["h_all"][:R], b["y_perm_all"][:R]
+            b["shared_rows"] = torch.arange(T, dtype=i32, device=dev)
+            b["shared"] = b["y_perm_all"][R:]
+        elif self.shared_f:
             b["shared_offsets"] = torch.tensor([0, T], dtype=i32, device=dev)
             b["h_shared"] = torch.empty(T, self.shared_f, dtype=bf, device=dev)
             b["shared"] = torch.empty(T, d, dtype=bf, device=dev)
@@ -131,7 +161,8 @@ class MoEFFN:
 
         timing: optional dict; if given, a (start, end) pair of CUDA events is recorded around each stage
         ("route", "permute", "gateup", "down", "combine" on the layer's stream; "shared", the always-on
-        expert, on the side stream where it overlaps routing and grouping).
+        expert, on the side stream where it overlaps routing and grouping: its GEMMs, or, folded into the routed
+        GEMMs (MXFP4), the copy of its rows).
         """
         T = x.shape[0]
         b = self.buffers(T)
@@ -154,8 +185,11 @@ class MoEFFN:
             if timing is not None:
                 timing["shared"] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 timing["shared"][0].record(side)
-            self._gateup(x, "shared", b["shared_offsets"], b["h_shared"], side)
-            self._down(b["h_shared"], "shared", b["shared_offsets"], b["shared"], side)
+            if self._fold(T):  # its rows after the routed ones; the routed GEMMs compute it
+                N.gather_rows(x, b["shared_rows"], b["x_perm_all"][T * self.k:], side)
+            else:
+                self._gateup(x, "shared", b["shared_offsets"], b["h_shared"], side)
+                self._down(b["h_shared"], "shared", b["shared_offsets"], b["shared"], side)
             shared_done = torch.cuda.Event()
             shared_done.record(side)
             if timing is not None:
@@ -182,6 +216,7 @@ class MoEFFN:
         mark("permute", False)
         if shared is not None:
             # the routed GEMMs are persistent kernels sized to every SM: they start once the shared expert is done
+            # (or, folded, its rows are in place)
             s.wait_event(shared_done)
         mark("gateup", True)
         if fused:
@@ -190,7 +225,7 @@ class MoEFFN:
             N.grouped_gemm_gateup_save(b["x_perm"], self.w_gateup, b["offsets"], b["h"], self._grad_buffers(T)["gu"], s)
             self._gu_saved = True
         else:
-            self._gateup(b["x_perm"], "routed", b["offsets"], b["h"], s)
+            self.routed_gateup(b, s)
         mark("gateup", False)
         mark("down", True)
         if fused:  # y_perm and, in the same kernel, y
@@ -198,7 +233,7 @@ class MoEFFN:
                                         b["topk_w"], shared, b["y_perm"], b["y"], b["combine_ws"], s)
             mark("down", False)
             return b["y"]
-        self._down(b["h"], "routed", b["offsets"], b["y_perm"], s)
+        self.routed_down(b, s)
         mark("down", False)
         mark("combine", True)
         N.unpermute_combine(b["y_perm"], b["inv_perm"], b["topk_w"], shared, b["y"], s)
@@ -212,6 +247,28 @@ class MoEFFN:
         T tokens."""
         return (self.fused and self.weights == "bf16" and T > 0
                 and N.grouped_gemm_gateup_gather_workspace_size(self.E, T * self.k, self.d) == 0)
+
+    def _fold(self, T: int) -> bool:
+        """Whether forward() computes the shared expert inside the routed MXFP4 GEMMs for T tokens: when the
+        R + T rows stay within the decode kernel's range (at most 8 rows per group on average, as the library's
+        dispatch decides), so that the routed experts keep that kernel."""
+        return self.fold_shared and T > 0 and T * self.k + T <= 8 * (self.E + 1)
+
+    def routed_gateup(self, b, stream):
+        """The routed gate|up GEMM of forward() on buffers b (with the folded shared expert as group E)."""
+        if "x_perm_all" in b:
+            q, sc = self.mx_gateup_all
+            N.grouped_gemm_gateup_mxfp4(b["x_perm_all"], q, sc, b["offsets_all"], b["h_all"], stream)
+        else:
+            self._gateup(b["x_perm"], "routed", b["offsets"], b["h"], stream)
+
+    def routed_down(self, b, stream):
+        """The routed down GEMM of forward() on buffers b (with the folded shared expert as group E)."""
+        if "x_perm_all" in b:
+            q, sc = self.mx_down_all
+            N.grouped_gemm_down_mxfp4(b["h_all"], q, sc, b["offsets_all"], b["y_perm_all"], stream)
+        else:
+            self._down(b["h"], "routed", b["offsets"], b["y_perm"], stream)
 
     def _gateup(self, a, which, offsets, h, stream):
         if self.weights == "mxfp4":
@@ -387,7 +444,7 @@ class MoEFFN:
         tensor-core path with fused top-k is taken (E <= 128, T >= 2048), else logits + top-k;
         permute 4, gate|up, down, combine 1 each (fused: permute 3, gate|up 1, down with combine 1; train: the
         gate|up that keeps its pre-activations is 1 kernel with 128 rows or more per expert, else 2); the shared
-        expert 2 more."""
+        expert 2 more (1 folded: the copy of its rows)."""
         if T <= 0:
             return 0
         route = 1 if (self.E <= 128 and T >= 2048) else 2
@@ -395,4 +452,4 @@ class MoEFFN:
             body = 4 + 3 + (0 if T * self.k >= 128 * self.E else 1)
         else:
             body = 3 + 2 if self._fused(T) else 4 + 3
-        return route + body + (2 if self.shared_f else 0)
+        return route + body + ((1 if self._fold(T) else 2) if self.shared_f else 0)

@@ -544,6 +544,33 @@ def test_mxfp4_large_scales_and_shared_expert():
     check_close(y, ref, "mxfp4 large scales + shared")
 
 
+def test_mxfp4_layer_folds_shared_expert_into_routed_gemms():
+    """A decode-sized MXFP4 layer whose shared expert is as wide as a routed one computes the shared expert as group
+    E of the routed GEMM launches (its rows after the routed rows): every token against the oracle, and the same
+    layer with the shared expert run on its own within the same bar."""
+    wl = synth.Workload(**{**synth.workload("tiny").__dict__, "name": "tiny-mxfp4-shared", "E": 32, "shared_f": 512,
+                           "weights": "mxfp4", "route": "sigmoid_topk_norm"})
+    ref = oracle.LayerReference(wl)
+    inp = synth.device_inputs(wl)
+    layer = MoEFFN(inp["w_router"], inp["w_gateup"], inp["w_down"], wl.k, wl.route, inp["bias"],
+                   inp["w_gateup_shared"], inp["w_down_shared"], weights="mxfp4")
+    twin = layer.sibling()
+    twin.fold_shared = False
+    assert layer._fold(wl.T) and not twin._fold(wl.T)
+    assert layer.kernel_launches(wl.T) == twin.kernel_launches(wl.T) - 1
+    y = bf16_to_host_f32(layer(inp["x"]).clone())
+    y_own = bf16_to_host_f32(twin(inp["x"]).clone())
+    torch.cuda.synchronize()
+    assert N.get_device_error() == 0
+    ties = set(ref.near_ties(NEAR_TIE).tolist())
+    toks = np.array([t for t in range(wl.T) if t not in ties], dtype=np.int32)
+    assert len(toks) >= wl.T - 4
+    assert (layer.buf["topk_idx"].cpu().numpy()[toks] == ref.idx[toks]).all()
+    want = ref.outputs(toks)
+    check_close(y[toks], want, "shared expert folded into the routed GEMMs")
+    check_close(y_own[toks], want, "shared expert on its own")
+
+
 def test_mxfp4_gateup_matches_bf16_gemm_on_decoded_weights():
     """Decode-shaped problem: h from the MXFP4 kernel equals h from the bf16 grouped GEMM given the decoded
     weights, up to fp32 summation order (both round h to bf16 from fp32 sums of the same products)."""
