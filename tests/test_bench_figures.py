@@ -34,6 +34,20 @@ def test_gemm_figures_count_only_active_experts_and_mxfp4_bytes():
     assert gu["bytes"] == pytest.approx(201 * 2 * wl.f * wl.d * wb + wl.R * wl.d * 2 + wl.R * wl.f * 2)
 
 
+def test_gemm_figures_count_a_folded_shared_expert_once():
+    wl = synth.workload("decode-256e-shared-mxfp4")
+    counts = np.zeros(wl.E, dtype=np.int64)
+    counts[:wl.R // 2] = 2
+    a0, gu0, dn0 = bench.gemm_figures(wl, counts)
+    a1, gu1, dn1 = bench.gemm_figures(wl, counts, folded_shared=True)
+    assert a1 == a0 == wl.R // 2
+    T, d, f, wb = wl.T, wl.d, wl.f, bench.weight_bytes(wl)
+    # one more group: its weights once, its T rows in and out
+    assert gu1["bytes"] - gu0["bytes"] == pytest.approx(2 * f * d * wb + T * d * 2 + T * f * 2)
+    assert dn1["bytes"] - dn0["bytes"] == pytest.approx(d * f * wb + T * f * 2 + T * d * 2)
+    assert gu1["flop"] - gu0["flop"] == 4.0 * T * d * f and dn1["flop"] - dn0["flop"] == 2.0 * T * d * f
+
+
 def test_roofline_entry_picks_the_slower_bound():
     peaks = {"bf16_tflops": 1000.0, "hbm_gbs": 5000.0}
     # 1 TFLOP and 1 GB: 1 ms of tensor work against 0.2 ms of bytes -> tensor-bound; 2 ms measured -> 0.5
