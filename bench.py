@@ -46,16 +46,16 @@ L2_FLUSH_BYTES = 256 << 20
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none -k regex:grouped_gemm -s 4 -c 1
 #       python bench.py --kernel K --workload W --steps 2 --warmup 3
 TRAFFIC = {
-    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "478dde139e27b6a8"): 1248200960,
-    ("grouped_gemm_down", "gpt-oss-20b-prefill", "478dde139e27b6a8"): 713675520,
-    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "478dde139e27b6a8"): 2494269440,
-    ("grouped_gemm_down", "mixtral-8x7b-prefill", "478dde139e27b6a8"): 2458328576,
-    ("grouped_gemm_gateup", "zipf-128e", "478dde139e27b6a8"): 1598989056,
-    ("grouped_gemm_down", "zipf-128e", "478dde139e27b6a8"): 1084371200,
-    ("grouped_gemm_gateup", "decode-256e-shared", "478dde139e27b6a8"): 12932950272,
-    ("grouped_gemm_down", "decode-256e-shared", "478dde139e27b6a8"): 6466513664,
-    ("grouped_gemm_gateup", "decode-256e-shared-mxfp4", "478dde139e27b6a8"): 3544724224,
-    ("grouped_gemm_down", "decode-256e-shared-mxfp4", "478dde139e27b6a8"): 1723772928,
+    ("grouped_gemm_gateup", "gpt-oss-20b-prefill", "e1c4dc9759352dbe"): 1248905472,
+    ("grouped_gemm_down", "gpt-oss-20b-prefill", "e1c4dc9759352dbe"): 713312000,
+    ("grouped_gemm_gateup", "mixtral-8x7b-prefill", "e1c4dc9759352dbe"): 2874045952,
+    ("grouped_gemm_down", "mixtral-8x7b-prefill", "e1c4dc9759352dbe"): 2457829376,
+    ("grouped_gemm_gateup", "zipf-128e", "e1c4dc9759352dbe"): 1593265664,
+    ("grouped_gemm_down", "zipf-128e", "e1c4dc9759352dbe"): 1083839744,
+    ("grouped_gemm_gateup", "decode-256e-shared", "e1c4dc9759352dbe"): 12932052992,
+    ("grouped_gemm_down", "decode-256e-shared", "e1c4dc9759352dbe"): 6467805184,
+    ("grouped_gemm_gateup", "decode-256e-shared-mxfp4", "e1c4dc9759352dbe"): 3671495936,
+    ("grouped_gemm_down", "decode-256e-shared-mxfp4", "e1c4dc9759352dbe"): 1772047616,
 }
 KERNEL_SOURCES = ["mixture_experts_ffn_11_b200/csrc/" + f for f in
                   ("gemm.cuh", "gemm_pair.cuh", "gemm_wide.cuh", "gemm_swap.cuh", "gemm_fp4.cuh", "gemm_fp4_mma.cuh",
