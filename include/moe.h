@@ -204,8 +204,8 @@ moe_status_t moe_permute_static_ws(const moe_bf16_t* x, const int32_t* topk_idx,
  *                  rows at or past group_offsets[G] are not written
  *   h              [M][f] bf16
  * M is the number of rows the caller allocated (T*k after moe_permute, T for
- * a shared expert with G = 1 and offsets {0, T}). Limits: G >= 1, d, f >= 8,
- * multiples of 8. */
+ * a shared expert with G = 1 and offsets {0, T}). Limits: 1 <= G <= 1024
+ * (the other grouped GEMMs below share it), d, f >= 8, multiples of 8. */
 moe_status_t moe_grouped_gemm_gateup(const moe_bf16_t* a, const moe_bf16_t* w_gateup, const int32_t* group_offsets,
                                      int G, int M, int d, int f, moe_bf16_t* h, cudaStream_t stream);
 

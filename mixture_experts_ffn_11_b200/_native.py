@@ -195,6 +195,7 @@ def permute(x, topk_idx, E, counts, offsets, perm_src, inv_perm, x_perm, ws, str
 
 
 PERMUTE_STATIC_WS_BYTES = 1 << 20  # MOE_PERMUTE_STATIC_WS_BYTES in include/moe.h
+MAX_GEMM_GROUPS = 1024  # the grouped GEMMs' limit on G (include/moe.h)
 
 
 def permute_static_ws(x, topk_idx, E, counts, offsets, perm_src, inv_perm, x_perm, stream=None):

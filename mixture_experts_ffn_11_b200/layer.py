@@ -251,8 +251,10 @@ class MoEFFN:
     def _fold(self, T: int) -> bool:
         """Whether forward() computes the shared expert inside the routed MXFP4 GEMMs for T tokens: when the
         R + T rows stay within the decode kernel's range (at most 8 rows per group on average, as the library's
-        dispatch decides), so that the routed experts keep that kernel."""
-        return self.fold_shared and T > 0 and T * self.k + T <= 8 * (self.E + 1)
+        dispatch decides), so that the routed experts keep that kernel, and E + 1 groups are within the grouped
+        GEMMs' limit of 1024."""
+        return (self.fold_shared and T > 0 and T * self.k + T <= 8 * (self.E + 1)
+                and self.E + 1 <= N.MAX_GEMM_GROUPS)
 
     def routed_gateup(self, b, stream):
         """The routed gate|up GEMM of forward() on buffers b (with the folded shared expert as group E)."""

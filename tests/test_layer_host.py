@@ -41,6 +41,15 @@ def test_fold_stops_where_the_routed_experts_would_leave_the_decode_kernel(MoEFF
     assert lay.kernel_launches(t_max + 1) == 2 + 4 + 3 + 2
 
 
+def test_no_fold_past_the_group_limit(MoEFFN):
+    from mixture_experts_ffn_11_b200 import _native as N
+
+    wl = synth.Workload(**{**synth.workload("decode-256e-shared-mxfp4").__dict__, "E": N.MAX_GEMM_GROUPS})
+    assert not _host_layer(MoEFFN, wl)._fold(64)  # E + 1 groups would pass the grouped GEMMs' limit
+    wl = synth.Workload(**{**wl.__dict__, "E": N.MAX_GEMM_GROUPS - 1})
+    assert _host_layer(MoEFFN, wl)._fold(64)
+
+
 def test_bf16_and_narrower_shared_experts_are_not_folded(MoEFFN):
     bf = _host_layer(MoEFFN, synth.workload("decode-256e-shared"))
     assert not bf.fold_shared and not bf._fold(64)
