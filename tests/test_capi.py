@@ -71,8 +71,12 @@ def test_invalid_arguments_rejected_before_any_launch(native):
     assert lib.moe_grouped_gemm_gateup(16, 16, 16, 1, 8, 12, 8, 16, null) == native.MOE_ERR_INVALID_ARG
     # misaligned pointer
     assert lib.moe_grouped_gemm_down(16, 16 + 2, 16, 1, 8, 8, 8, 16, null) == native.MOE_ERR_INVALID_ARG
-    # too many groups
+    # too many groups (the limit is 1024)
     assert lib.moe_grouped_gemm_down(16, 16, 16, 4096, 8, 8, 8, 16, null) == native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_gateup(16, 16, 16, native.MAX_GEMM_GROUPS + 1, 8, 8, 8, 16, null) == \
+        native.MOE_ERR_INVALID_ARG
+    assert lib.moe_grouped_gemm_gateup_mxfp4(16, 16, 16, 16, native.MAX_GEMM_GROUPS + 1, 8, 64, 64, 16, null) == \
+        native.MOE_ERR_INVALID_ARG
     # k > 32 in combine
     assert lib.moe_unpermute_combine(16, 16, 16, null, 4, 8, 33, 16, null) == native.MOE_ERR_INVALID_ARG
     # split router: no pieces; E out of range for the split
