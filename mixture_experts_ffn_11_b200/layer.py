@@ -70,8 +70,8 @@ class MoEFFN:
         # tensors; for decode-sized T (_fold) its T rows (x itself) follow the R routed rows, and the routed GEMM
         # launches compute it as one more group, spread over every SM like the rest (on its own it is one group of
         # T rows, which the MXFP4 kernels run on a few SMs: 139 us on the decode layer's side stream, half of it
-        # after the routing and grouping beside it; folded in, it adds 3-4% to the routed GEMMs and the decode
-        # layer takes 1.12 instead of 1.21 ms)
+        # after the routing and grouping beside it; folded in, it adds 3.6% to the routed GEMMs' work, and on one
+        # box the decode layer took 1.206-1.212 ms against 1.210-1.216 ms, at a power-capped clock 2-3% lower)
         self.fold_shared = weights == "mxfp4" and self.shared_f == self.f and self.shared_f > 0
         if weights == "mxfp4":
             E = self.E
